@@ -1,0 +1,214 @@
+"""CPU oracle for the quantized-attention hot path (ctypes over ``liboracle.so``).
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference arm import this package.  The product
+path (the CUDA library and its binding) never imports it and shares no code
+with it.
+
+Every array here is numpy.  bf16 tensors travel as their uint16 bit patterns.
+Layouts follow the library's logical layout [B, H, N, D]; V codes are
+token-major [N_kv, D] here (the device library stores them in its own order).
+"""
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+MASK_NONE, MASK_CAUSAL, MASK_BLOCK_CAUSAL = 0, 1, 2
+BLK = 64          # Q/K quantization block (tokens)
+TKV = 128         # KV tile width of the online softmax (the device kernel's)
+
+# Relative uncertainty of the device's exp2 result plus one fp32 rounding of
+# the oracle's own exp2.  The device uses the hardware ex2.approx.ftz.f32; its
+# measured worst relative error over the softmax's argument range is checked
+# by a GPU test to stay below EXP2_REL_ERR.  The slack derived from EPS marks
+# every e4m3 rounding of p*256 that the two sides may take differently.
+EXP2_REL_ERR = 2.0 ** -21
+EPS = EXP2_REL_ERR + 2.0 ** -24
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i64, i32, f64 = ctypes.c_long, ctypes.c_int, ctypes.c_double
+        L.orc_e4m3_decode.restype = f64
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e4m3_encode_n.restype = None
+        L.orc_e4m3_encode_n.argtypes = [P, i64, P]
+        L.orc_quant_head.restype = i32
+        L.orc_quant_head.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P]
+        L.orc_qk_int32.restype = None
+        L.orc_qk_int32.argtypes = [P, P, i32, i64, i64, i64, i64, P]
+        L.orc_row_limit.restype = i64
+        L.orc_row_limit.argtypes = [i64, i64, i64, i32, i64]
+        L.orc_attn_rows.restype = i32
+        L.orc_attn_rows.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
+                                    P, i64, P, P, P, i32]
+        L.orc_attn_rows_identity.restype = i32
+        L.orc_attn_rows_identity.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
+                                             P, i64, P, P, i32]
+        L.orc_attn_fp64_rows.restype = i32
+        L.orc_attn_fp64_rows.argtypes = [P, P, P, i64, i64, i32, i32, i64, P, i64, P, i32]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _threads(n):
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+# ---------------------------------------------------------------- e4m3
+
+def e4m3_encode(x):
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().orc_e4m3_encode_n(_p(x), x.size, _p(out))
+    return out
+
+
+def e4m3_decode(codes):
+    L = lib()
+    table = np.array([L.orc_e4m3_decode(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+# ---------------------------------------------------------------- quantization
+
+def quant_head(q, k, v):
+    """Quantize one head.  q [nq, D], k/v [nkv, D] as uint16 bf16 bits.
+
+    Returns a dict: q8 [nq_pad, D] int8, qs [nq_blk] f32, k8 [nkv_pad, D] int8,
+    ks [nkv_blk] f32, mu [D] f32, v8 [nkv, D] uint8 e4m3 codes, vs [D] f32.
+    """
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    nq, D = q.shape
+    nkv = k.shape[0]
+    nqb, nkb = -(-nq // BLK), -(-nkv // BLK)
+    out = dict(q8=np.empty((nqb * BLK, D), np.int8), qs=np.empty(nqb, np.float32),
+               k8=np.empty((nkb * BLK, D), np.int8), ks=np.empty(nkb, np.float32),
+               mu=np.empty(D, np.float32), v8=np.empty((nkv, D), np.uint8),
+               vs=np.empty(D, np.float32))
+    rc = lib().orc_quant_head(_p(q), _p(k), _p(v), nq, nkv, D,
+                              _p(out["q8"]), _p(out["qs"]), _p(out["k8"]), _p(out["ks"]),
+                              _p(out["mu"]), _p(out["v8"]), _p(out["vs"]))
+    if rc:
+        raise MemoryError("orc_quant_head failed")
+    out["nq"], out["nkv"], out["D"] = nq, nkv, D
+    return out
+
+
+def quant(q, k, v):
+    """Quantize [B, H, N, D] bf16-bit tensors head by head; returns stacked arrays."""
+    B, H = q.shape[:2]
+    heads = [quant_head(q[b, h], k[b, h], v[b, h]) for b in range(B) for h in range(H)]
+    out = {}
+    for key in ("q8", "qs", "k8", "ks", "mu", "v8", "vs"):
+        a = np.stack([hd[key] for hd in heads])
+        out[key] = a.reshape((B, H) + a.shape[1:])
+    return out
+
+
+def qk_int32(q8, k8, i0, ni, j0, nj):
+    q8 = np.ascontiguousarray(q8, np.int8)
+    k8 = np.ascontiguousarray(k8, np.int8)
+    out = np.empty((ni, nj), np.int32)
+    lib().orc_qk_int32(_p(q8), _p(k8), q8.shape[1], i0, ni, j0, nj, _p(out))
+    return out
+
+
+def row_limit(i, nq, nkv, mask, mb):
+    return lib().orc_row_limit(i, nq, nkv, mask, mb)
+
+
+# ---------------------------------------------------------------- attention
+
+def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
+              threads=None):
+    """Same-quantization attention of one quantized head on the given rows.
+
+    Returns (o [n, D] float64 of the fp32 recipe, slack [n, D] or None, lse [n]).
+    """
+    rows = np.ascontiguousarray(rows, np.int64)
+    n, D = rows.size, qh["D"]
+    o = np.empty((n, D), np.float64)
+    slack = np.empty((n, D), np.float64) if with_slack else None
+    lse = np.empty(n, np.float64)
+    q8 = np.ascontiguousarray(qh["q8"])
+    k8 = np.ascontiguousarray(qh["k8"])
+    v8 = np.ascontiguousarray(qh["v8"])
+    qs = np.ascontiguousarray(qh["qs"])
+    ks = np.ascontiguousarray(qh["ks"])
+    vs = np.ascontiguousarray(qh["vs"])
+    rc = lib().orc_attn_rows(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
+                             qh["nq"], qh["nkv"], D, mask, mb, tkv, eps,
+                             _p(rows), n, _p(o), _p(slack) if slack is not None else None,
+                             _p(lse), _threads(threads))
+    if rc:
+        raise ValueError("orc_attn_rows: invalid arguments")
+    return o, slack, lse
+
+
+def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=None):
+    """The oracle's tiled loop with identity quantizers, fp64 throughout."""
+    q = np.ascontiguousarray(q, np.float64)
+    k = np.ascontiguousarray(k, np.float64)
+    v = np.ascontiguousarray(v, np.float64)
+    rows = np.ascontiguousarray(rows, np.int64)
+    n, D = rows.size, q.shape[1]
+    o = np.empty((n, D), np.float64)
+    lse = np.empty(n, np.float64)
+    rc = lib().orc_attn_rows_identity(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
+                                      mask, mb, tkv, _p(rows), n, _p(o), _p(lse),
+                                      _threads(threads))
+    if rc:
+        raise ValueError("orc_attn_rows_identity: invalid arguments")
+    return o, lse
+
+
+def attn_fp64_rows(q, k, v, rows, mask=MASK_NONE, mb=0, threads=None):
+    """Full-precision softmax attention of one head from bf16 bits, fp64."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    rows = np.ascontiguousarray(rows, np.int64)
+    n, D = rows.size, q.shape[1]
+    o = np.empty((n, D), np.float64)
+    rc = lib().orc_attn_fp64_rows(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D, mask, mb,
+                                  _p(rows), n, _p(o), _threads(threads))
+    if rc:
+        raise ValueError("orc_attn_fp64_rows: invalid arguments")
+    return o
+
+
+def bf16_bits_to_f64(x):
+    return (np.asarray(x, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def accuracy(o, ref):
+    """cosine similarity and mean relative L1 of o against ref (flattened)."""
+    o = np.asarray(o, np.float64).ravel()
+    ref = np.asarray(ref, np.float64).ravel()
+    cos = float(o @ ref / (np.linalg.norm(o) * np.linalg.norm(ref)))
+    rel_l1 = float(np.abs(o - ref).sum() / np.abs(ref).sum())
+    return cos, rel_l1
+
+
+def c0(D):
+    """fp32(log2(e)/sqrt(D)) as the recipe defines it (for tests)."""
+    return np.float32(math.log2(math.e) / math.sqrt(D))

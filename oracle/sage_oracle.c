@@ -1,0 +1,651 @@
+/*
+ * sage_oracle.c -- plain, slow CPU reference for SageAttention-style
+ * quantized attention (INT8 per-block Q/K with K mean-smoothing, FP8 e4m3
+ * per-channel V, FP8 P, fp32 online softmax).
+ *
+ * TEST INFRASTRUCTURE.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline / reference arm may load this library.  The GPU
+ * product path never calls it and shares no code, header or table with it.
+ *
+ * Sources of the method:
+ *   - "Vidu S1: A Real-Time Interactive Video Generation Model" digest
+ *     (zhao9797.github.io), section "Infra": SageAttention is the attention
+ *     accelerator; per-block 8-bit quantization is chosen because per-tensor
+ *     and per-channel scales are stretched by outliers.
+ *   - reportify.cn TurboDiffusion notes: SageAttention is low-bit quantized
+ *     attention; 8-bit block-wise quantization runs on INT8 tensor cores.
+ *   - The finer recipe (64-token INT8 blocks with absmax/127 and
+ *     round-half-to-even, K mean-smoothing over tokens, e4m3 V with a
+ *     per-channel absmax/448 scale, FP8 P, fp32 online softmax with exp2) is
+ *     not printed on the pages; the readings taken here are listed in the
+ *     design notes and restated next to each function below.
+ *
+ * Build: plain C11, no FMA contraction (-ffp-contract=off), no fast-math, so
+ * that every float expression below is one IEEE binary32 operation rounded
+ * to nearest-even (x86-64 SSE: FLT_EVAL_METHOD == 0).
+ *
+ * Parity status of each exported function (what pins it in the tests):
+ *   orc_e4m3_encode / decode : OCP OFP8 E4M3 special points + brute-force
+ *                              nearest-even search + torch float8 cast.
+ *   orc_quant_head           : quantizer invariants, numpy mean for mu.
+ *   orc_qk_int32             : numpy int64 brute force.
+ *   orc_attn_rows (identity) : textbook softmax attention to 1e-12.
+ *   orc_attn_rows (quant)    : closed forms (Q = 0, single visible key) and
+ *                              the error bound against fp64 attention.
+ *   orc_attn_fp64_rows       : textbook softmax attention (torch) to 1e-12.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_BLK 64 /* Q/K quantization block: 64 tokens */
+
+enum { ORC_MASK_NONE = 0, ORC_MASK_CAUSAL = 1, ORC_MASK_BLOCK_CAUSAL = 2 };
+
+/* ------------------------------------------------------------------ */
+/* bf16                                                               */
+/* ------------------------------------------------------------------ */
+
+static float bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 E4M3 (OCP OFP8): 1 sign bit, 4 exponent bits with bias 7,       */
+/* 3 mantissa bits.  Exponent field 0 holds subnormals m/8 * 2^-6.     */
+/* No infinities; S.1111.111 is NaN, so the largest finite is          */
+/* 1.75 * 2^8 = 448.                                                   */
+/* ------------------------------------------------------------------ */
+
+double orc_e4m3_decode(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Round a non-negative finite double to e4m3 with round-to-nearest-even and
+ * saturation to the largest finite value (the "satfinite" convention). */
+static uint8_t e4m3_encode_abs(double a)
+{
+    int e2, E;
+    double quantum, n, r, v;
+    if (a >= 448.0)
+        return 0x7E;
+    if (a == 0.0)
+        return 0x00;
+    frexp(a, &e2);      /* a = f * 2^e2, f in [0.5, 1) */
+    E = e2 - 1;         /* a in [2^E, 2^(E+1)) */
+    if (E < -6)
+        E = -6;         /* subnormal range shares the 2^-9 quantum */
+    quantum = ldexp(1.0, E - 3);
+    n = a / quantum;    /* exact: power-of-two division */
+    r = nearbyint(n);   /* ties to even on the integer = on the mantissa */
+    v = r * quantum;
+    if (v == 0.0)
+        return 0x00;
+    if (v >= 448.0)
+        return 0x7E;
+    /* encode the representable value v */
+    frexp(v, &e2);
+    E = e2 - 1;
+    if (E < -6) {       /* subnormal: v = m/8 * 2^-6 */
+        int m = (int)(v / ldexp(1.0, -9));
+        return (uint8_t)m;
+    } else {
+        int m = (int)((v / ldexp(1.0, E) - 1.0) * 8.0);
+        return (uint8_t)(((E + 7) << 3) | m);
+    }
+}
+
+static uint8_t e4m3_encode_d(double x)
+{
+    if (isnan(x))
+        return 0x7F;
+    if (signbit(x))
+        return (uint8_t)(0x80 | e4m3_encode_abs(-x));
+    return e4m3_encode_abs(x);
+}
+
+uint8_t orc_e4m3_encode(float x) { return e4m3_encode_d((double)x); }
+
+void orc_e4m3_encode_n(const float *x, long n, uint8_t *out)
+{
+    for (long i = 0; i < n; i++)
+        out[i] = orc_e4m3_encode(x[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* Quantization                                                        */
+/* ------------------------------------------------------------------ */
+
+/* Symmetric per-block INT8 over blocks of 64 rows of an [n, D] matrix:
+ * a = max |x| over the block's valid rows, scale = a/127, inv = 127/a,
+ * q = clamp(round_half_even(x * inv), -127, 127).  An all-zero block gets
+ * scale 0 and q = 0; rows past n (padding up to the next multiple of 64)
+ * are 0.  Reading: no zero point, -128 unused, multiply by the rounded
+ * inverse rather than divide per element. */
+static void quant_blocks_i8(const float *x, long n, int D, int8_t *q, float *scale)
+{
+    long nblk = (n + ORC_BLK - 1) / ORC_BLK;
+    for (long b = 0; b < nblk; b++) {
+        long r0 = b * ORC_BLK, r1 = r0 + ORC_BLK;
+        long rv = r1 < n ? r1 : n;
+        float a = 0.0f;
+        for (long r = r0; r < rv; r++)
+            for (int d = 0; d < D; d++) {
+                float t = fabsf(x[r * D + d]);
+                if (t > a)
+                    a = t;
+            }
+        memset(q + r0 * D, 0, (size_t)(ORC_BLK * D));
+        if (a == 0.0f) {
+            scale[b] = 0.0f;
+            continue;
+        }
+        scale[b] = a / 127.0f;
+        float inv = 127.0f / a;
+        for (long r = r0; r < rv; r++)
+            for (int d = 0; d < D; d++) {
+                float y = x[r * D + d] * inv;
+                float t = nearbyintf(y);
+                if (t > 127.0f)
+                    t = 127.0f;
+                if (t < -127.0f)
+                    t = -127.0f;
+                q[r * D + d] = (int8_t)t;
+            }
+    }
+}
+
+/* Quantize one (batch, head): Q [nq, D], K [nkv, D], V [nkv, D] as bf16 bits.
+ *
+ * Outputs (caller-allocated):
+ *   q8 [ceil(nq/64)*64, D] int8, qs [ceil(nq/64)]
+ *   k8 [ceil(nkv/64)*64, D] int8, ks [ceil(nkv/64)], mu [D]
+ *   v8 [nkv, D] e4m3 codes (logical token-major order), vs [D]
+ *
+ * K mean-smoothing: mu[d] = fp32(sum_n K[n,d] / nkv) where the sum is taken
+ * in fp64 in a fixed order: each 64-token block summed in ascending token
+ * order, then the block sums added in ascending block order.  The smoothed
+ * key ks = fp32(K - mu) is what gets block-quantized.  Q is not smoothed.
+ *
+ * V: per channel d over all nkv tokens, a = max |V[:,d]|, vs = a/448,
+ * inv = 448/a, v8 = e4m3_rne_satfinite(V * inv); a == 0 gives vs = 0, v8 = 0.
+ */
+int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                   long nq, long nkv, int D,
+                   int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
+                   uint8_t *v8, float *vs)
+{
+    float *x = (float *)malloc(sizeof(float) * (size_t)((nq > nkv ? nq : nkv) * D));
+    if (!x)
+        return 1;
+    /* Q */
+    for (long i = 0; i < nq * D; i++)
+        x[i] = bf16_to_f32(q[i]);
+    quant_blocks_i8(x, nq, D, q8, qs);
+    /* K channel mean in the canonical fp64 order */
+    long nblk = (nkv + ORC_BLK - 1) / ORC_BLK;
+    for (int d = 0; d < D; d++) {
+        double total = 0.0;
+        for (long b = 0; b < nblk; b++) {
+            double s = 0.0;
+            long r1 = (b + 1) * ORC_BLK < nkv ? (b + 1) * ORC_BLK : nkv;
+            for (long r = b * ORC_BLK; r < r1; r++)
+                s += (double)bf16_to_f32(k[r * D + d]);
+            total += s;
+        }
+        mu[d] = (float)(total / (double)nkv);
+    }
+    /* smoothed K, then block quantization */
+    for (long r = 0; r < nkv; r++)
+        for (int d = 0; d < D; d++)
+            x[r * D + d] = bf16_to_f32(k[r * D + d]) - mu[d];
+    quant_blocks_i8(x, nkv, D, k8, ks);
+    /* V per channel */
+    for (int d = 0; d < D; d++) {
+        float a = 0.0f;
+        for (long r = 0; r < nkv; r++) {
+            float t = fabsf(bf16_to_f32(v[r * D + d]));
+            if (t > a)
+                a = t;
+        }
+        if (a == 0.0f) {
+            vs[d] = 0.0f;
+            for (long r = 0; r < nkv; r++)
+                v8[r * D + d] = 0;
+            continue;
+        }
+        vs[d] = a / 448.0f;
+        float inv = 448.0f / a;
+        for (long r = 0; r < nkv; r++)
+            v8[r * D + d] = orc_e4m3_encode(bf16_to_f32(v[r * D + d]) * inv);
+    }
+    free(x);
+    return 0;
+}
+
+/* Exact integer scores S[i,j] = sum_d q8[i,d] * k8[j,d] for rows i0..i0+ni-1
+ * and keys j0..j0+nj-1 (brute force in int64, stored as int32). */
+void orc_qk_int32(const int8_t *q8, const int8_t *k8, int D,
+                  long i0, long ni, long j0, long nj, int32_t *out)
+{
+    for (long a = 0; a < ni; a++)
+        for (long b = 0; b < nj; b++) {
+            int64_t s = 0;
+            for (int d = 0; d < D; d++)
+                s += (int64_t)q8[(i0 + a) * D + d] * (int64_t)k8[(j0 + b) * D + d];
+            out[a * nj + b] = (int32_t)s;
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Masks                                                               */
+/* ------------------------------------------------------------------ */
+
+/* Keys j < limit are visible to query row i.  Queries are the newest nq
+ * tokens of a cache of nkv (bottom-right alignment: query i sits at cache
+ * position g = i + nkv - nq).
+ *   none          : limit = nkv
+ *   causal        : limit = g + 1
+ *   block-causal  : every key of the query's own block (of mb tokens) and of
+ *                   all earlier blocks: limit = min(nkv, (g/mb + 1) * mb). */
+long orc_row_limit(long i, long nq, long nkv, int mask, long mb)
+{
+    long g = i + (nkv - nq);
+    long lim;
+    switch (mask) {
+    case ORC_MASK_CAUSAL:
+        lim = g + 1;
+        break;
+    case ORC_MASK_BLOCK_CAUSAL:
+        lim = (g / mb + 1) * mb;
+        break;
+    default:
+        lim = nkv;
+    }
+    return lim < nkv ? lim : nkv;
+}
+
+/* ------------------------------------------------------------------ */
+/* Attention, one query row at a time                                  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int identity; /* 1: quantizers replaced by identity, arithmetic in fp64 */
+    long nq, nkv;
+    int D, mask;
+    long mb, tkv;
+    double eps; /* relative exp2 uncertainty used for the rounding slack */
+    /* quantized operands (identity == 0) */
+    const int8_t *q8;
+    const float *qs;
+    const int8_t *k8;
+    const float *ks;
+    const uint8_t *v8; /* [nkv, D] */
+    const float *vs;
+    /* full-precision operands (identity == 1), [n, D] doubles */
+    const double *qd, *kd, *vd;
+    /* rows and outputs */
+    const long *rows;
+    long nrows;
+    double *o;     /* [nrows, D] */
+    double *slack; /* [nrows, D] or NULL */
+    double *lse;   /* [nrows] natural-log log-sum-exp, or NULL */
+} attn_job;
+
+static float exp2_f32(float x) { return (float)exp2((double)x); }
+
+/* Width, in units of p*256, of the set of e4m3 codes that p*256*(1 +- eps)
+ * can round to; zero when the uncertainty interval does not straddle a
+ * rounding boundary. */
+static double e4m3_flip_gap(double y, double eps)
+{
+    uint8_t lo = e4m3_encode_d(y * (1.0 - eps));
+    uint8_t hi = e4m3_encode_d(y * (1.0 + eps));
+    if (lo == hi)
+        return 0.0;
+    return fabs(orc_e4m3_decode(hi) - orc_e4m3_decode(lo));
+}
+
+/* One query row i with the flash-style online softmax over KV tiles of
+ * width tkv, visiting tiles in ascending order, only those holding a
+ * visible key.  Per tile k (scores in the log2 domain):
+ *   m_k   = max(m_{k-1}, max_j t_ij)                  (m_{-1} = -inf)
+ *   alpha = 0 if m_{k-1} = -inf else exp2(m_{k-1} - m_k)
+ *   p_ij  = exp2(t_ij - m_k)
+ *   l     = l * alpha + sum_j p_ij
+ *   O     = O * alpha + sum_j w_ij V_j
+ * and finally O / l.
+ *
+ * Quantized mode (the same-quantization result):
+ *   C0    = fp32(log2(e) / sqrt(D))             (fp64, rounded once)
+ *   sqC   = fp32(sq[i/64] * C0); c_ij = fp32(sqC * sk[j/64])
+ *   S_ij  = sum_d q8 k8 (exact integer)
+ *   t_ij  = fp32(fp32(S_ij) * c_ij)             (for the max)
+ *   x_ij  = fmaf(fp32(S_ij), c_ij, -m_k); p_ij = fp32(exp2(x_ij))
+ *   l is accumulated in fp32 from p (before quantization),
+ *   w_ij  = e4m3(p_ij * 256) (P scale 2^8), V_j = e4m3 code values,
+ *   O     = O_acc * vs[d] / (256 * l).
+ * Identity mode: t_ij = (q_i . k_j) * log2(e)/sqrt(D), w = p, all fp64.
+ */
+static void attend_row(const attn_job *J, long r)
+{
+    const long i = J->rows[r];
+    const int D = J->D;
+    const long lim = orc_row_limit(i, J->nq, J->nkv, J->mask, J->mb);
+    const long tkv = J->tkv;
+    double *o = J->o + r * D;
+    double *sl = J->slack ? J->slack + r * D : NULL;
+    double *acc = (double *)calloc((size_t)D, sizeof(double));
+    double *sacc = (double *)calloc((size_t)D, sizeof(double));
+    int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)tkv);
+    float *c = (float *)malloc(sizeof(float) * (size_t)tkv);
+    double *t = (double *)malloc(sizeof(double) * (size_t)tkv);
+
+    const double C64 = 1.4426950408889634 / sqrt((double)D); /* log2(e)/sqrt(D) */
+    const float C0 = (float)C64;
+    float sqC = 0.0f;
+    if (!J->identity)
+        sqC = J->qs[i / ORC_BLK] * C0;
+
+    double m = -INFINITY, l = 0.0;
+    float mf = -INFINITY, lf = 0.0f;
+    for (int d = 0; d < D; d++)
+        o[d] = 0.0;
+
+    for (long j0 = 0; j0 < lim; j0 += tkv) {
+        long j1 = j0 + tkv < lim ? j0 + tkv : lim; /* visible keys of this tile */
+        long nj = j1 - j0;
+        /* scores */
+        for (long jj = 0; jj < nj; jj++) {
+            long j = j0 + jj;
+            if (J->identity) {
+                double s = 0.0;
+                for (int d = 0; d < D; d++)
+                    s += J->qd[i * D + d] * J->kd[j * D + d];
+                t[jj] = s * C64;
+            } else {
+                int64_t s = 0;
+                for (int d = 0; d < D; d++)
+                    s += (int64_t)J->q8[i * D + d] * (int64_t)J->k8[j * D + d];
+                S[jj] = (int32_t)s;
+                c[jj] = sqC * J->ks[j / ORC_BLK];
+                t[jj] = (double)((float)S[jj] * c[jj]);
+            }
+        }
+        /* running max and rescale factor */
+        double tmax = -INFINITY;
+        for (long jj = 0; jj < nj; jj++)
+            if (t[jj] > tmax)
+                tmax = t[jj];
+        double alpha;
+        if (J->identity) {
+            double mn = m > tmax ? m : tmax;
+            alpha = (m == -INFINITY) ? 0.0 : exp2(m - mn);
+            m = mn;
+        } else {
+            float mn = mf > (float)tmax ? mf : (float)tmax;
+            alpha = (mf == -INFINITY) ? 0.0 : (double)exp2_f32(mf - mn);
+            mf = mn;
+        }
+        /* probabilities and the P.V contribution */
+        for (int d = 0; d < D; d++) {
+            acc[d] = 0.0;
+            sacc[d] = 0.0;
+        }
+        double rowsum = 0.0;
+        float rowsum_f = 0.0f;
+        for (long jj = 0; jj < nj; jj++) {
+            long j = j0 + jj;
+            if (J->identity) {
+                double p = exp2(t[jj] - m);
+                rowsum += p;
+                for (int d = 0; d < D; d++)
+                    acc[d] += p * J->vd[j * D + d];
+            } else {
+                float x = fmaf((float)S[jj], c[jj], -mf);
+                float p = exp2_f32(x);
+                rowsum_f += p;
+                float y = p * 256.0f;
+                double w = orc_e4m3_decode(orc_e4m3_encode(y));
+                double gap = sl ? e4m3_flip_gap((double)y, J->eps) : 0.0;
+                for (int d = 0; d < D; d++) {
+                    double vv = orc_e4m3_decode(J->v8[j * D + d]);
+                    acc[d] += w * vv;
+                    if (gap != 0.0)
+                        sacc[d] += gap * fabs(vv);
+                }
+            }
+        }
+        for (int d = 0; d < D; d++) {
+            o[d] = o[d] * alpha + acc[d];
+            if (sl)
+                sl[d] = sl[d] * alpha + sacc[d];
+        }
+        if (J->identity)
+            l = l * alpha + rowsum;
+        else
+            lf = lf * (float)alpha + rowsum_f;
+    }
+    /* output */
+    if (J->identity) {
+        for (int d = 0; d < D; d++)
+            o[d] = o[d] / l;
+        if (J->lse)
+            J->lse[r] = (m + log2(l)) * 0.6931471805599453;
+    } else {
+        for (int d = 0; d < D; d++) {
+            double f = (double)J->vs[d] / (256.0 * (double)lf);
+            o[d] = o[d] * f;
+            if (sl)
+                sl[d] = sl[d] * f;
+        }
+        if (J->lse)
+            J->lse[r] = ((double)mf + log2((double)lf)) * 0.6931471805599453;
+    }
+    free(acc);
+    free(sacc);
+    free(S);
+    free(c);
+    free(t);
+}
+
+/* ------------------------------------------------------------------ */
+/* Thread fan-out over rows (rows are independent)                     */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const void *job;
+    void (*fn)(const void *, long);
+    long r0, r1;
+} span;
+
+static void *span_run(void *arg)
+{
+    span *s = (span *)arg;
+    for (long r = s->r0; r < s->r1; r++)
+        s->fn(s->job, r);
+    return NULL;
+}
+
+static void for_rows(const void *job, void (*fn)(const void *, long), long nrows, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > nrows)
+        nthreads = (int)(nrows > 0 ? nrows : 1);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    span *sp = (span *)malloc(sizeof(span) * (size_t)nthreads);
+    long per = (nrows + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; t++) {
+        sp[t].job = job;
+        sp[t].fn = fn;
+        sp[t].r0 = t * per < nrows ? t * per : nrows;
+        sp[t].r1 = (t + 1) * per < nrows ? (t + 1) * per : nrows;
+        if (t == 0)
+            continue;
+        pthread_create(&th[t], NULL, span_run, &sp[t]);
+    }
+    span_run(&sp[0]);
+    for (int t = 1; t < nthreads; t++)
+        pthread_join(th[t], NULL);
+    free(th);
+    free(sp);
+}
+
+static void attend_row_cb(const void *job, long r) { attend_row((const attn_job *)job, r); }
+
+/* Same-quantization attention for the given query rows of one head.
+ * q8/qs/k8/ks/v8/vs as produced by orc_quant_head (v8 token-major [nkv, D]).
+ * o, slack: [nrows, D] doubles; lse: [nrows] or NULL; slack may be NULL.
+ * eps: relative uncertainty of the device exp2 (plus one fp32 rounding) used
+ * to mark e4m3 rounding decisions of p*256 that may go either way. */
+int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
+                  const uint8_t *v8, const float *vs, long nq, long nkv, int D,
+                  int mask, long mb, long tkv, double eps,
+                  const long *rows, long nrows, double *o, double *slack, double *lse,
+                  int nthreads)
+{
+    if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0)
+        return 1;
+    if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
+        return 1;
+    if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
+        return 1;
+    attn_job J = {0};
+    J.identity = 0;
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = mask;
+    J.mb = mb;
+    J.tkv = tkv;
+    J.eps = eps;
+    J.q8 = q8;
+    J.qs = qs;
+    J.k8 = k8;
+    J.ks = ks;
+    J.v8 = v8;
+    J.vs = vs;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.slack = slack;
+    J.lse = lse;
+    if (slack)
+        memset(slack, 0, sizeof(double) * (size_t)(nrows * D));
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
+}
+
+/* The same tiled online-softmax loop with the quantizers replaced by
+ * identity and all arithmetic in fp64 (q, k, v: [n, D] doubles). */
+int orc_attn_rows_identity(const double *q, const double *k, const double *v,
+                           long nq, long nkv, int D, int mask, long mb, long tkv,
+                           const long *rows, long nrows, double *o, double *lse,
+                           int nthreads)
+{
+    if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0)
+        return 1;
+    if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
+        return 1;
+    if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
+        return 1;
+    attn_job J = {0};
+    J.identity = 1;
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = mask;
+    J.mb = mb;
+    J.tkv = tkv;
+    J.qd = q;
+    J.kd = k;
+    J.vd = v;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.lse = lse;
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Full-precision attention: the plain definition                       */
+/* O_i = sum_j softmax_j(q_i . k_j / sqrt(D) over visible j) v_j, fp64 */
+/* from the bf16 inputs.                                               */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    long nq, nkv;
+    int D, mask;
+    long mb;
+    const long *rows;
+    double *o;
+} fp64_job;
+
+static void fp64_row(const void *job, long r)
+{
+    const fp64_job *J = (const fp64_job *)job;
+    const int D = J->D;
+    const long i = J->rows[r];
+    const long lim = orc_row_limit(i, J->nq, J->nkv, J->mask, J->mb);
+    double *s = (double *)malloc(sizeof(double) * (size_t)lim);
+    double *qi = (double *)malloc(sizeof(double) * (size_t)D);
+    double *o = J->o + r * D;
+    const double scale = 1.0 / sqrt((double)D);
+    for (int d = 0; d < D; d++)
+        qi[d] = (double)bf16_to_f32(J->q[i * D + d]);
+    double mx = -INFINITY;
+    for (long j = 0; j < lim; j++) {
+        double a = 0.0;
+        for (int d = 0; d < D; d++)
+            a += qi[d] * (double)bf16_to_f32(J->k[j * D + d]);
+        s[j] = a * scale;
+        if (s[j] > mx)
+            mx = s[j];
+    }
+    double den = 0.0;
+    for (int d = 0; d < D; d++)
+        o[d] = 0.0;
+    for (long j = 0; j < lim; j++) {
+        double p = exp(s[j] - mx);
+        den += p;
+        for (int d = 0; d < D; d++)
+            o[d] += p * (double)bf16_to_f32(J->v[j * D + d]);
+    }
+    for (int d = 0; d < D; d++)
+        o[d] /= den;
+    free(s);
+    free(qi);
+}
+
+int orc_attn_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       long nq, long nkv, int D, int mask, long mb,
+                       const long *rows, long nrows, double *o, int nthreads)
+{
+    if (nq <= 0 || nkv <= 0 || D <= 0)
+        return 1;
+    if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
+        return 1;
+    if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
+        return 1;
+    fp64_job J = {q, k, v, nq, nkv, D, mask, mb, rows, o};
+    for_rows(&J, fp64_row, nrows, nthreads);
+    return 0;
+}
