@@ -1,0 +1,411 @@
+"""Benchmark of the quantized-attention hot path on B200.
+
+One step = the whole path on one batch of synthetic input already resident in
+HBM: sage_quant_qk (Q/K INT8 per block, K smoothing, V e4m3) followed by
+sage_attn_fwd (fused INT8 QK^T, fp32 online softmax, FP8 P V).  The metric is
+quantized-attention TOPS = 4 * D * B * H * (visible query-key pairs) per
+second of step time, summed over all ranks.
+
+Default workload: the 720p video-DiT shape (B1 H40 N75600 D128, K with four
+x20 outlier channels); the 480p shape (B1 H12 N32760) is timed alongside.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank processes its own
+full workload (weak scaling, no data-path collective) and the step time is
+the max over ranks.  `--impl reference` times the CPU oracle (the only
+reference of this method here) on a bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_attention_sage_b200 import synth  # noqa: E402
+
+METRIC = "quantized-attention TOPS at 32k/75k tokens (H=12/40, D=128); % of INT8/FP8 peak"
+UNIT = "TOPS"
+KERNELS_PER_STEP = 4  # quant pass1, finalize, pass2, attention
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=synth.P720.name, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="approximate CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def peaks():
+    """8-bit tensor peak (TOPS) and HBM GB/s from the measured file."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        m = json.load(open(path))
+        return {"i8_sustained": 2.0 * m["bf16_tflops_sustained"], "i8_burst": 2.0 * m["bf16_tflops"],
+                "hbm": m["hbm_gbs"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"i8_sustained": 2.0 * 1400.0, "i8_burst": 2.0 * 1590.0, "hbm": 6650.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in ("attn.cu", "sm100.cuh", "attn.cuh"):
+        h.update(open(os.path.join(ROOT, "bit_quantized_attention_sage_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "attn_traffic.json")))
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec
+
+
+class Runner:
+    """Device buffers and one step of the hot path for a workload."""
+
+    def __init__(self, w, seed_offset, device):
+        import torch
+        import bit_quantized_attention_sage_b200 as sage
+        self.torch, self.sage, self.w = torch, sage, w
+        wr = synth.Workload(w.name, w.B, w.H, w.Nq, w.Nkv, w.D, w.mask, w.mask_block,
+                            w.k_offset_var, w.outlier_mag, w.seed + seed_offset)
+        q, k, v = synth.full(wr)
+
+        def pin(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        self.h_q, self.h_k, self.h_v = pin(q), pin(k), pin(v)
+        del q, k, v
+        self.q = self.h_q.to(device)
+        self.k = self.h_k.to(device)
+        self.v = self.h_v.to(device)
+        self.shape = sage.make_shape(w.B, w.H, w.Nq, w.Nkv, w.D)
+        self.qkv = sage.QuantizedQKV(self.shape, device)
+        self.ws = torch.empty(max(sage.workspace_bytes(self.shape), 16), dtype=torch.uint8,
+                              device=device)
+        self.o = torch.empty((w.B, w.H, w.Nq, w.D), dtype=torch.bfloat16, device=device)
+        self.h_o = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
+        self.stream = torch.cuda.current_stream()
+
+    def step(self, ev=None):
+        s = self.sage
+        if ev is not None:
+            ev[0].record(self.stream)
+        s.quant_qk(self.q, self.k, self.v, out=self.qkv, workspace=self.ws, stream=self.stream)
+        if ev is not None:
+            ev[1].record(self.stream)
+        s.attn_fwd(self.qkv, self.w.mask, self.w.mask_block, out=self.o, stream=self.stream)
+        if ev is not None:
+            ev[2].record(self.stream)
+
+    def step_e2e(self):
+        self.q.copy_(self.h_q, non_blocking=True)
+        self.k.copy_(self.h_k, non_blocking=True)
+        self.v.copy_(self.h_v, non_blocking=True)
+        self.step()
+        self.h_o.copy_(self.o, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.h_q, self.h_k, self.h_v))
+
+    def d2h_bytes(self):
+        return self.h_o.numel() * self.h_o.element_size()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(runner, steps, warmup, world, e2e=False, per_kernel=False):
+    torch = runner.torch
+    fn = runner.step_e2e if e2e else runner.step
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)] \
+        if per_kernel else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(runner.stream)
+    for i in range(steps):
+        if e2e:
+            fn()
+        else:
+            runner.step(evs[i] if per_kernel else None)
+    end.record(runner.stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end) / steps
+    out = {"ms": max_over_ranks(ms, world)}
+    if per_kernel:
+        out["quant_ms"] = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+        out["attn_ms"] = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    return out
+
+
+def cpu_baseline(w, target_s):
+    """Time the CPU oracle on a bounded sample of the workload: quantize one
+    head, attend a set of its query rows; throughput in the metric's unit."""
+    import oracle
+    q, k, v = synth.head(w, 0, 0)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    qh = oracle.quant_head(q, k, v)
+    t_quant = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    # calibrate on one row per thread, then size the sample to ~target_s
+    cal = rng.choice(w.Nq, size=min(threads, w.Nq), replace=False)
+    t0 = time.perf_counter()
+    oracle.attn_rows(qh, cal, w.mask, w.mask_block, with_slack=False, threads=threads)
+    t_cal = max(time.perf_counter() - t0, 1e-3)
+    n_rows = int(min(w.Nq, max(threads, len(cal) * target_s / t_cal)))
+    rows = np.sort(rng.choice(w.Nq, size=n_rows, replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_rows(qh, rows, w.mask, w.mask_block, with_slack=False, threads=threads)
+    t_attn = time.perf_counter() - t0
+    pairs = sum(oracle.row_limit(int(i), w.Nq, w.Nkv, w.mask, max(w.mask_block, 1)) for i in rows)
+    ops = 4 * w.D * pairs
+    # charge the whole head's quantization pro rata to the sampled rows
+    t = t_attn + t_quant * n_rows / w.Nq
+    return {"value": ops / t / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%s: oracle quantization of head 0 and same-quantization attention of %d "
+                      "of its %d query rows (%d threads, %.1f s)" % (w.name, n_rows, w.Nq,
+                                                                      threads, t)}
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import bit_quantized_attention_sage_b200 as sage
+    sage.lib()
+    w = synth.WORKLOADS[args.workload]
+    runner = Runner(w, 1000 * rank, device)
+    ops_rank = w.ops()
+    pk = peaks()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    t = time_steps(runner, args.steps, args.warmup, world, per_kernel=True)
+    clk = clocks.stop()
+    if sage.sync_status() != 0:
+        raise RuntimeError("device status error during the timed steps")
+
+    in_gb = runner.h2d_bytes() / 1e9
+    e2e = None
+    if not args.no_e2e:
+        te = time_steps(runner, args.steps, max(1, args.warmup), world, e2e=True)
+        e2e = {"value": ops_rank * world / (te["ms"] / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
+               "ms_per_step": te["ms"]}
+
+    secondary = {}
+    if not args.no_secondary and w.name != synth.P480.name:
+        del runner
+        torch.cuda.empty_cache()
+        r2 = Runner(synth.P480, 1000 * rank, device)
+        t2 = time_steps(r2, args.steps, args.warmup, world, per_kernel=True)
+        secondary[synth.P480.name] = {
+            "value": synth.P480.ops() * world / (t2["ms"] / 1e3) / 1e12, "unit": UNIT,
+            "ms_per_step": t2["ms"], "attn_ms": t2["attn_ms"], "quant_ms": t2["quant_ms"],
+            "attn_frac_of_peak": synth.P480.ops() / (t2["attn_ms"] / 1e3) / 1e12 / pk["i8_sustained"]}
+        del r2
+
+    value = ops_rank * world / (t["ms"] / 1e3) / 1e12
+    achieved = ops_rank / (t["attn_ms"] / 1e3) / 1e12
+    traffic = recorded_traffic()
+    # algorithmic bytes of sage_quant_qk: read bf16 (2 B) and write one 8-bit
+    # code (1 B) per element of Q, K and V, plus the scales and the K mean
+    quant_bytes = 3 * w.B * w.H * (w.Nq + 2 * w.Nkv) * w.D + 4 * w.B * w.H * (
+        (w.Nq + 63) // 64 + (w.Nkv + 63) // 64 + 2 * w.D)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t["ms"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8+e4m3 (fp32 softmax)", "data": "synthetic (seeded N(0,1) bf16, K outliers)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nkv": w.Nkv, "D": w.D,
+                   "mask": ["none", "causal", "block_causal"][w.mask],
+                   "mask_block": w.mask_block, "ops_per_step_per_gpu": ops_rank,
+                   "l2": "inputs (%.2f GB bf16 Q/K/V per GPU) larger than the 126 MB L2; no flush"
+                         % in_gb,
+                   "parallelism": "replica per GPU (dp%d, no collective)" % world},
+        "roofline": {"bound": "tensor", "kernel": "k_attn (sage_attn_fwd)",
+                     "achieved": round(achieved, 2), "peak": round(pk["i8_sustained"], 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / pk["i8_sustained"], 4),
+                     "peak_note": "8-bit dense = 2 x %s sustained cuBLAS bf16 (of %s)" % (
+                         "measured" if pk["source"] == "measured" else "fallback", pk["source"]),
+                     "attn_ms_per_launch": round(t["attn_ms"], 4),
+                     "traffic": traffic["bytes_per_launch"] if traffic else None},
+        "roofline_quant": {"bound": "hbm", "kernel": "sage_quant_qk (3 kernels)",
+                           "achieved": round(quant_bytes / (t["quant_ms"] / 1e3) / 1e9, 1),
+                           "peak": pk["hbm"], "unit": "GB/s",
+                           "frac": round(quant_bytes / (t["quant_ms"] / 1e3) / 1e9 / pk["hbm"], 4),
+                           "ms_per_step": round(t["quant_ms"], 4),
+                           "algorithmic_bytes": quant_bytes},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if secondary:
+        line["also"] = secondary
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    per_step = max(2.0, min(15.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, per_step / 4)
+    vals, secs = [], []
+    last = None
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        last = cpu_baseline(w, per_step)
+        secs.append(time.perf_counter() - t0)
+        vals.append(last["value"])
+    value = float(np.mean(vals))
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(secs)),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "i8+e4m3 (fp32 softmax), CPU", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nkv": w.Nkv,
+                       "D": w.D, "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,231 @@
+"""B200-native SageAttention-style quantized attention.
+
+Thin ctypes binding of ``libsage_b200.so`` (the C ABI in ``include/sage.h``).
+This module only marshals arguments: torch provides device memory and the
+stream, every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback -- if the library is missing or the device is not an
+sm_100a GPU the calls raise.
+
+One-line use, in place of a FlashAttention call on [B, H, N, D] bf16 tensors:
+
+    o = attention(q, k, v)                          # bidirectional
+    o = attention(q, k, v, mask="causal")
+    o = attention(q, k, v, mask=("block_causal", 2040))   # streaming KV cache
+"""
+import ctypes
+import os
+
+MASK_NONE, MASK_CAUSAL, MASK_BLOCK_CAUSAL = 0, 1, 2
+TILE_M, TILE_N = 128, 128   # attention kernel's query rows per CTA / keys per KV tile
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
+          4: "device wait timed out"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage_b200.so")
+_lib = None
+
+
+class SageError(RuntimeError):
+    def __init__(self, code, what):
+        super().__init__("%s: %s (status %d)" % (what, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("Nq", ctypes.c_int),
+                ("Nkv", ctypes.c_int), ("D", ctypes.c_int)]
+
+
+class _QKV(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q_i8", "q_scale", "k_i8", "k_scale", "k_mean", "v_f8", "v_scale")]
+
+
+BUFFERS = ("q_i8", "q_scale", "k_i8", "k_scale", "k_mean", "v_f8", "v_scale")
+
+
+def lib():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libsage_b200.so is not built; run "
+                              "`python -m bit_quantized_attention_sage_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.sage_abi_version.restype = I
+        L.sage_status_string.restype = ctypes.c_char_p
+        L.sage_status_string.argtypes = [I]
+        L.sage_quant_buffer_bytes.restype = I
+        L.sage_quant_buffer_bytes.argtypes = [P, P]
+        L.sage_quant_workspace_bytes.restype = SZ
+        L.sage_quant_workspace_bytes.argtypes = [P]
+        L.sage_quant_qk.restype = I
+        L.sage_quant_qk.argtypes = [P, P, P, P, P, P, SZ, P]
+        L.sage_attn_fwd.restype = I
+        L.sage_attn_fwd.argtypes = [P, P, I, I, P, P, P, P]
+        L.sage_debug_qk_int32.restype = I
+        L.sage_debug_qk_int32.argtypes = [P, P, P, I, P, P]
+        L.sage_debug_timeout_probe.restype = I
+        L.sage_debug_timeout_probe.argtypes = [ctypes.c_longlong, P]
+        L.sage_debug_e4m3.restype = I
+        L.sage_debug_e4m3.argtypes = [P, P, SZ, P]
+        L.sage_debug_exp2.restype = I
+        L.sage_debug_exp2.argtypes = [P, P, SZ, P]
+        L.sage_sync_status.restype = I
+        L.sage_sync_status.argtypes = [P]
+        _lib = L
+    return _lib
+
+
+def _check(code, what):
+    if code != 0:
+        raise SageError(code, what)
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def make_shape(B, H, Nq, Nkv, D):
+    return Shape(int(B), int(H), int(Nq), int(Nkv), int(D))
+
+
+def buffer_bytes(shape):
+    sizes = (ctypes.c_size_t * 7)()
+    _check(lib().sage_quant_buffer_bytes(ctypes.byref(shape), sizes), "sage_quant_buffer_bytes")
+    return dict(zip(BUFFERS, (int(x) for x in sizes)))
+
+
+def workspace_bytes(shape):
+    return int(lib().sage_quant_workspace_bytes(ctypes.byref(shape)))
+
+
+class QuantizedQKV:
+    """The seven device buffers sage_quant_qk fills (torch uint8 storage)."""
+
+    def __init__(self, shape, device):
+        import torch
+        self.shape = shape
+        self.bufs = {n: torch.empty(b, dtype=torch.uint8, device=device)
+                     for n, b in buffer_bytes(shape).items()}
+
+    def struct(self):
+        return _QKV(*(self.bufs[n].data_ptr() for n in BUFFERS))
+
+    # typed views (for inspection and tests)
+    def view(self, name):
+        import torch
+        s = self.shape
+        bh = s.B * s.H
+        nqp, nkp = -(-s.Nq // 64) * 64, -(-s.Nkv // 64) * 64
+        t = self.bufs[name]
+        if name == "q_i8":
+            return t.view(torch.int8).view(s.B, s.H, nqp, s.D)
+        if name == "k_i8":
+            return t.view(torch.int8).view(s.B, s.H, nkp, s.D)
+        if name == "v_f8":
+            return t.view(s.B, s.H, s.D, nkp)
+        if name == "q_scale":
+            return t.view(torch.float32).view(s.B, s.H, nqp // 64)
+        if name == "k_scale":
+            return t.view(torch.float32).view(s.B, s.H, nkp // 64)
+        return t.view(torch.float32).view(s.B, s.H, s.D)
+
+
+def quant_qk(q, k, v, out=None, workspace=None, stream=None):
+    """sage_quant_qk on bf16 CUDA tensors [B, H, N, D]; returns QuantizedQKV."""
+    import torch
+    B, H, Nq, D = q.shape
+    Nkv = k.shape[2]
+    shape = make_shape(B, H, Nq, Nkv, D)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if out is None:
+        out = QuantizedQKV(shape, q.device)
+    ws_need = workspace_bytes(shape)
+    if workspace is None:
+        workspace = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=q.device)
+    qs = out.struct()
+    _check(lib().sage_quant_qk(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(qs),
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sage_quant_qk")
+    return out
+
+
+def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, stream=None):
+    """sage_attn_fwd on a QuantizedQKV; returns the bf16 output tensor."""
+    import torch
+    s = qkv.shape
+    dev = qkv.bufs["q_i8"].device
+    if out is None:
+        out = torch.empty((s.B, s.H, s.Nq, s.D), dtype=torch.bfloat16, device=dev)
+    st = qkv.struct()
+    _check(lib().sage_attn_fwd(ctypes.byref(st), ctypes.byref(s), int(mask), int(mask_block),
+                               _ptr(out), _ptr(o_f32), _ptr(lse), _stream(stream)),
+           "sage_attn_fwd")
+    return out
+
+
+def attention(q, k, v, mask=None, stream=None):
+    """Drop-in quantized attention: bf16 [B, H, N, D] in, bf16 out."""
+    if mask is None or mask == "none":
+        m, mb = MASK_NONE, 0
+    elif mask == "causal":
+        m, mb = MASK_CAUSAL, 0
+    elif isinstance(mask, tuple) and mask[0] == "block_causal":
+        m, mb = MASK_BLOCK_CAUSAL, int(mask[1])
+    else:
+        raise ValueError("mask must be None, 'causal' or ('block_causal', n)")
+    qkv = quant_qk(q, k, v, stream=stream)
+    return attn_fwd(qkv, m, mb, stream=stream)
+
+
+def debug_qk_int32(qkv, tiles, stream=None):
+    """int32 score tiles left in tensor memory by the attention kernel.
+
+    tiles: sequence of (bh, qt, kt); returns a torch int32 [n, 128, 128]."""
+    import torch
+    n = len(tiles)
+    flat = (ctypes.c_int * (3 * n))(*[int(x) for t in tiles for x in t])
+    out = torch.empty((n, TILE_M, TILE_N), dtype=torch.int32, device=qkv.bufs["q_i8"].device)
+    st = qkv.struct()
+    _check(lib().sage_debug_qk_int32(ctypes.byref(st), ctypes.byref(qkv.shape), flat, n,
+                                     _ptr(out), _stream(stream)), "sage_debug_qk_int32")
+    return out
+
+
+def debug_e4m3(x, stream=None):
+    """Device e4m3 codes of a float32 CUDA tensor (the kernels' conversion)."""
+    import torch
+    x = x.contiguous()
+    y = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib().sage_debug_e4m3(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "sage_debug_e4m3")
+    return y
+
+
+def debug_exp2(x, stream=None):
+    """Device 2^x of a float32 CUDA tensor (the softmax's exp2)."""
+    import torch
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check(lib().sage_debug_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "sage_debug_exp2")
+    return y
+
+
+def timeout_probe(budget_cycles, stream=None):
+    _check(lib().sage_debug_timeout_probe(int(budget_cycles), _stream(stream)),
+           "sage_debug_timeout_probe")
+
+
+def sync_status(stream=None):
+    """Synchronize the stream and return (and clear) the device status code."""
+    return int(lib().sage_sync_status(_stream(stream)))

@@ -1,0 +1,325 @@
+// api.cu -- the C ABI declared in include/sage.h: argument validation, TMA
+// descriptor encoding, kernel launches and the device status word.
+//
+// Nothing here allocates device memory: every buffer comes from the caller.
+// No exception crosses the ABI; errors are returned as sage_status codes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.cuh"
+#include "quant.cuh"
+#include "sage.h"
+#include "sm100.cuh"
+
+#define SAGE_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace sage {
+namespace {
+
+// {code, site} -- see WaitCtx.  One copy per device that loads the library.
+__device__ int g_status[2];
+
+constexpr long long kWaitBudget = 1ll << 31;  // ~1 s of SM clock per wait
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t init_err = cudaSuccess;
+  int* status = nullptr;  // device address of g_status
+};
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device one-time setup: the status word's device address and the
+// attention kernels' shared-memory attribute.
+DeviceState* device_state() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& d = g_dev[dev];
+  std::call_once(d.once, [&d] {
+    void* p = nullptr;
+    d.init_err = cudaGetSymbolAddress(&p, g_status);
+    d.status = static_cast<int*>(p);
+    if (d.init_err == cudaSuccess) d.init_err = attn_prepare(128);
+    if (d.init_err == cudaSuccess) d.init_err = attn_prepare(64);
+  });
+  if (d.init_err != cudaSuccess) return nullptr;
+  return &d;
+}
+
+inline bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t pad64(int n) { return (static_cast<size_t>(n) + 63) / 64 * 64; }
+
+bool shape_ok(const sage_shape* s) {
+  if (!s) return false;
+  if (s->B < 1 || s->H < 1 || s->Nq < 1 || s->Nkv < 1) return false;
+  if (s->D != 64 && s->D != 128) return false;
+  if (static_cast<long long>(s->B) * s->H > 65535) return false;
+  if (s->Nq > (1 << 30) || s->Nkv > (1 << 30)) return false;
+  return true;
+}
+
+void buffer_bytes(const sage_shape* s, size_t sz[7]) {
+  const size_t bh = static_cast<size_t>(s->B) * s->H, D = s->D;
+  sz[0] = bh * pad64(s->Nq) * D;         // q_i8
+  sz[1] = bh * (pad64(s->Nq) / 64) * 4;  // q_scale
+  sz[2] = bh * pad64(s->Nkv) * D;        // k_i8
+  sz[3] = bh * (pad64(s->Nkv) / 64) * 4; // k_scale
+  sz[4] = bh * D * 4;                    // k_mean
+  sz[5] = bh * D * pad64(s->Nkv);        // v_f8
+  sz[6] = bh * D * 4;                    // v_scale
+}
+
+size_t workspace_bytes(const sage_shape* s) {
+  const size_t bh = static_cast<size_t>(s->B) * s->H, D = s->D;
+  return bh * (pad64(s->Nkv) / 64) * D * 12 + bh * D * 4;
+}
+
+bool qkv_ok(const sage_qkv_quant* q) {
+  return q && aligned16(q->q_i8) && aligned16(q->q_scale) && aligned16(q->k_i8) &&
+         aligned16(q->k_scale) && aligned16(q->k_mean) && aligned16(q->v_f8) &&
+         aligned16(q->v_scale);
+}
+
+// 3-D tiled map over a contiguous uint8 array [d2][d1][d0] with a
+// box0 x box1 x 1 box.
+bool encode_u8_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0, d0 * d1};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_maps(const sage_qkv_quant* q, const sage_shape* s, AttnMaps* m) {
+  const uint64_t bh = static_cast<uint64_t>(s->B) * s->H, D = s->D;
+  const CUtensorMapSwizzle swqk =
+      D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return encode_u8_3d(&m->q, q->q_i8, D, pad64(s->Nq), bh, static_cast<uint32_t>(D), kAttnBM,
+                      swqk) &&
+         encode_u8_3d(&m->k, q->k_i8, D, pad64(s->Nkv), bh, static_cast<uint32_t>(D), kAttnBN,
+                      swqk) &&
+         encode_u8_3d(&m->v, q->v_f8, pad64(s->Nkv), D, bh, kAttnBN, static_cast<uint32_t>(D),
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+AttnParams base_params(const sage_qkv_quant* q, const sage_shape* s, const DeviceState* d) {
+  AttnParams p{};
+  p.BH = s->B * s->H;
+  p.Nq = s->Nq;
+  p.Nkv = s->Nkv;
+  p.D = s->D;
+  p.nq_blocks = static_cast<int>(pad64(s->Nq) / 64);
+  p.nkv_blocks = static_cast<int>(pad64(s->Nkv) / 64);
+  p.q_scale = q->q_scale;
+  p.k_scale = q->k_scale;
+  p.v_scale = q->v_scale;
+  // fp32(log2(e) / sqrt(D)), the log2-domain softmax scale, rounded once
+  p.c0 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s->D)));
+  p.budget = kWaitBudget;
+  p.status = d->status;
+  return p;
+}
+
+__global__ void k_timeout_probe(long long budget, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  const WaitCtx w{budget, status, &abort_flag};
+  // Nothing arrives on `bar`: the bounded wait must give up and report.
+  (void)mbar_wait(&bar, 0, w, 0x7F001);
+}
+
+// Debug: the same e4m3 conversion and exp2 the kernels use, elementwise.
+__global__ void k_e4m3(const float* x, uint8_t* y, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = static_cast<uint8_t>(cvt_e4m3x2(x[i], 0.0f) & 0xFF);
+}
+
+__global__ void k_exp2(const float* x, float* y, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = ex2_approx(x[i]);
+}
+
+}  // namespace
+}  // namespace sage
+
+using namespace sage;
+
+SAGE_EXPORT int sage_abi_version(void) { return SAGE_ABI_VERSION; }
+
+SAGE_EXPORT const char* sage_status_string(sage_status st) {
+  switch (st) {
+    case SAGE_OK: return "ok";
+    case SAGE_ERR_INVALID_ARG: return "invalid argument";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported";
+    case SAGE_ERR_CUDA: return "CUDA error";
+    case SAGE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+SAGE_EXPORT sage_status sage_quant_buffer_bytes(const sage_shape* shape, size_t sizes[7]) {
+  if (!shape_ok(shape) || !sizes) return SAGE_ERR_INVALID_ARG;
+  buffer_bytes(shape, sizes);
+  return SAGE_OK;
+}
+
+SAGE_EXPORT size_t sage_quant_workspace_bytes(const sage_shape* shape) {
+  return shape_ok(shape) ? workspace_bytes(shape) : 0;
+}
+
+SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, const void* v_bf16,
+                                      const sage_shape* shape, const sage_qkv_quant* out,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  if (!shape_ok(shape) || !qkv_ok(out)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(workspace))
+    return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape)) return SAGE_ERR_INVALID_ARG;
+  if (!device_state()) return SAGE_ERR_CUDA;
+  QuantArgs a{};
+  a.q = static_cast<const uint16_t*>(q_bf16);
+  a.k = static_cast<const uint16_t*>(k_bf16);
+  a.v = static_cast<const uint16_t*>(v_bf16);
+  a.BH = shape->B * shape->H;
+  a.Nq = shape->Nq;
+  a.Nkv = shape->Nkv;
+  a.D = shape->D;
+  a.q_i8 = out->q_i8;
+  a.q_scale = out->q_scale;
+  a.k_i8 = out->k_i8;
+  a.k_scale = out->k_scale;
+  a.k_mean = out->k_mean;
+  a.v_f8 = out->v_f8;
+  a.v_scale = out->v_scale;
+  const size_t cells = static_cast<size_t>(a.BH) * (pad64(a.Nkv) / 64) * a.D;
+  a.ws_ksum = static_cast<double*>(workspace);
+  a.ws_vmax = reinterpret_cast<float*>(static_cast<char*>(workspace) + cells * 8);
+  a.ws_vinv = reinterpret_cast<float*>(static_cast<char*>(workspace) + cells * 12);
+  return launch_quant(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
+                                                                           : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_attn_fwd(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
+                                      int mask_block, void* o_bf16, float* o_f32, float* lse,
+                                      void* stream) {
+  if (!shape_ok(shape) || !qkv_ok(qkv) || !aligned16(o_bf16)) return SAGE_ERR_INVALID_ARG;
+  if (o_f32 && !aligned16(o_f32)) return SAGE_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SAGE_ERR_INVALID_ARG;
+  if (mask < SAGE_MASK_NONE || mask > SAGE_MASK_BLOCK_CAUSAL) return SAGE_ERR_INVALID_ARG;
+  if (mask != SAGE_MASK_NONE && shape->Nkv < shape->Nq) return SAGE_ERR_INVALID_ARG;
+  if (mask == SAGE_MASK_BLOCK_CAUSAL && mask_block < 1) return SAGE_ERR_INVALID_ARG;
+  DeviceState* d = device_state();
+  if (!d) return SAGE_ERR_CUDA;
+  AttnMaps maps;
+  if (!make_maps(qkv, shape, &maps)) return SAGE_ERR_CUDA;
+  AttnParams p = base_params(qkv, shape, d);
+  p.mask = mask;
+  p.mask_block = mask == SAGE_MASK_BLOCK_CAUSAL ? mask_block : 1;
+  p.o = static_cast<__nv_bfloat16*>(o_bf16);
+  p.o_f32 = o_f32;
+  p.lse = lse;
+  return launch_attn(maps, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
+                                                                                : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_debug_qk_int32(const sage_qkv_quant* qkv, const sage_shape* shape,
+                                            const int* tiles, int n_tiles, int32_t* out,
+                                            void* stream) {
+  if (!shape_ok(shape) || !qkv_ok(qkv) || !aligned16(out) || !tiles) return SAGE_ERR_INVALID_ARG;
+  if (n_tiles < 0 || n_tiles > 65535) return SAGE_ERR_INVALID_ARG;
+  const int bh = shape->B * shape->H;
+  const int nqt = static_cast<int>((pad64(shape->Nq) + kAttnBM - 1) / kAttnBM);
+  const int nkt = static_cast<int>((pad64(shape->Nkv) + kAttnBN - 1) / kAttnBN);
+  for (int t = 0; t < n_tiles; t++) {
+    const int* tt = tiles + 3 * t;
+    if (tt[0] < 0 || tt[0] >= bh || tt[1] < 0 || tt[1] >= nqt || tt[2] < 0 || tt[2] >= nkt)
+      return SAGE_ERR_INVALID_ARG;
+  }
+  DeviceState* d = device_state();
+  if (!d) return SAGE_ERR_CUDA;
+  AttnMaps maps;
+  if (!make_maps(qkv, shape, &maps)) return SAGE_ERR_CUDA;
+  AttnParams p = base_params(qkv, shape, d);
+  p.mask_block = 1;
+  for (int t = 0; t < n_tiles; t++) {
+    p.dbg_bh = tiles[3 * t];
+    p.dbg_qt = tiles[3 * t + 1];
+    p.dbg_kt = tiles[3 * t + 2];
+    p.dbg_out = out + static_cast<size_t>(t) * kAttnBM * kAttnBN;
+    if (launch_attn_dump(maps, p, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+  }
+  return SAGE_OK;
+}
+
+SAGE_EXPORT sage_status sage_debug_timeout_probe(long long budget_cycles, void* stream) {
+  if (budget_cycles < 1 || budget_cycles > (1ll << 40)) return SAGE_ERR_INVALID_ARG;
+  DeviceState* d = device_state();
+  if (!d) return SAGE_ERR_CUDA;
+  k_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_cycles, d->status);
+  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_debug_e4m3(const float* x, uint8_t* y, size_t n, void* stream) {
+  if (!x || !y) return SAGE_ERR_INVALID_ARG;
+  if (n == 0) return SAGE_OK;
+  k_e4m3<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_debug_exp2(const float* x, float* y, size_t n, void* stream) {
+  if (!x || !y) return SAGE_ERR_INVALID_ARG;
+  if (n == 0) return SAGE_OK;
+  k_exp2<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_sync_status(void* stream) {
+  DeviceState* d = device_state();
+  if (!d) return SAGE_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGE_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpy(h, d->status, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  if (h[0] != 0) {
+    const int z[2] = {0, 0};
+    if (cudaMemcpy(d->status, z, sizeof z, cudaMemcpyHostToDevice) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+    return static_cast<sage_status>(h[0]);
+  }
+  return SAGE_OK;
+}

@@ -1,0 +1,445 @@
+// attn.cu -- sage_attn_fwd: fused SageAttention-style quantized attention
+// for sm_100a.
+//
+// The method (low-bit quantized attention that keeps FlashAttention's
+// streaming structure but runs its matmuls on 8-bit tensor cores; "Vidu S1"
+// digest section "Infra", TurboDiffusion notes): Q K^T on INT8 tensor cores
+// from per-block INT8 codes, an fp32 online softmax in the log2 domain, P
+// quantized to FP8 e4m3 with a fixed 2^8 scale and P V on FP8 tensor cores
+// with fp32 accumulation.
+//
+// One CTA owns 128 query rows of one (batch, head) and streams the visible
+// KV tiles of 128 keys.  Warp roles (192 threads, two CTAs per SM):
+//   warp 0      TMA producer: the Q tile once, then K and V^T tiles through
+//               a two-stage shared-memory ring (128-byte swizzle).
+//   warp 1      allocates 256 TMEM columns (S: 128 x 128 int32, O: 128 x D
+//               fp32) and one elected thread issues every tcgen05.mma:
+//               S = Q K^T (kind::i8) for tile k+1 while the softmax warps
+//               work on tile k, then O (+)= P V^T (kind::f8f6f4).
+//   warps 2-5   softmax: thread t of the warpgroup owns query row t (TMEM
+//               lane t).  Per tile: load the int32 score row from TMEM, take
+//               the masked max in the integer domain per 64-key scale group,
+//               update the running max, p = exp2(fma(S, c, -m)), row sum,
+//               e4m3(p * 256) into the swizzled shared-memory P tile, and
+//               rescale the O row in TMEM when the max moved.  Epilogue:
+//               O * v_scale / (256 l) -> bf16 (and optional fp32 O, lse).
+// Every wait is bounded (see WaitCtx); on a timeout the CTA drains its
+// in-flight copies and MMAs, frees TMEM and returns.
+#include "attn.cuh"
+#include "sm100.cuh"
+
+#include <cfloat>
+#include <climits>
+
+namespace sage {
+
+namespace {
+
+constexpr int BM = kAttnBM;
+constexpr int BN = kAttnBN;
+constexpr int NS = 2;              // K/V pipeline stages
+constexpr int kThreads = 192;      // 6 warps
+constexpr int kTmemCols = 256;
+constexpr uint32_t kFull = 0xffffffffu;
+
+// wait-site codes for the status word (kernel 1 = attention)
+enum : int {
+  kSiteProdKEmpty = 0x10101, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaSFree,
+  kSiteMmaV, kSiteMmaP, kSiteSmS, kSiteSmO, kSiteSmEpi, kSiteDrain
+};
+
+template <int D>
+struct alignas(1024) Smem {
+  uint8_t q[BM * D];         // int8 Q tile [128 rows][D]
+  uint8_t k[NS][BN * D];     // int8 K tiles [128 keys][D]
+  uint8_t v[NS][D * BN];     // e4m3 V^T tiles [D][128 keys]
+  uint8_t p[BM * BN];        // e4m3 P tile [128 rows][128 keys], 128-byte swizzle
+  uint64_t q_full;
+  uint64_t k_full[NS], k_empty[NS];
+  uint64_t v_full[NS], v_empty[NS];
+  uint64_t s_full, s_free, p_full, o_ready, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__host__ __device__ inline size_t smem_bytes_for(int D) {
+  return (D == 128 ? sizeof(Smem<128>) : sizeof(Smem<64>)) + 1024;  // + alignment slack
+}
+
+// A wait taken by all 32 threads of a warp that reports success only if it
+// succeeded for every lane, so that the warp never splits before the
+// warp-collective tcgen05.ld / tcgen05.st that follow.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                          int site) {
+  return __all_sync(kFull, mbar_wait(bar, parity, w, site));
+}
+
+// First key index that query row i (global row) may NOT see.
+__device__ __forceinline__ int row_limit(int i, const AttnParams& p) {
+  const int g = i + (p.Nkv - p.Nq);
+  int lim = p.Nkv;
+  if (p.mask == 1) lim = g + 1;
+  else if (p.mask == 2) lim = (g / p.mask_block + 1) * p.mask_block;
+  return lim < p.Nkv ? lim : p.Nkv;
+}
+
+// Bounded wait that ignores the abort flag: used while draining copies and
+// MMAs that were already issued, so that the CTA never frees shared memory
+// or TMEM under an operation in flight.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > w.budget) {
+      record_timeout(w.status, kSiteDrain);
+      return;
+    }
+  }
+}
+
+template <int D, bool DUMP>
+__device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int bh, int qt,
+                                         int kt0, int nk, const WaitCtx& w) {
+  tma_prefetch_desc(&maps.q);
+  tma_prefetch_desc(&maps.k);
+  tma_prefetch_desc(&maps.v);
+  mbar_arrive_expect_tx(&s.q_full, BM * D);
+  tma_load_3d(s.q, &maps.q, &s.q_full, 0, qt * BM, bh);
+  int k_issued = 0, v_issued = 0;
+  for (int it = 0; it < nk; it++) {
+    const int st = it % NS;
+    const uint32_t ph = (it / NS) & 1;
+    const int kt = kt0 + it;
+    if (it >= NS && !mbar_wait(&s.k_empty[st], ph ^ 1, w, kSiteProdKEmpty)) break;
+    mbar_arrive_expect_tx(&s.k_full[st], BN * D);
+    tma_load_3d(s.k[st], &maps.k, &s.k_full[st], 0, kt * BN, bh);
+    k_issued++;
+    if (DUMP) continue;
+    if (it >= NS && !mbar_wait(&s.v_empty[st], ph ^ 1, w, kSiteProdVEmpty)) break;
+    mbar_arrive_expect_tx(&s.v_full[st], D * BN);
+    tma_load_3d(s.v[st], &maps.v, &s.v_full[st], kt * BN, 0, bh);
+    v_issued++;
+  }
+  // Drain: every issued load must have landed before the CTA may exit.  A
+  // load is only issued once the previous load of its stage was consumed, so
+  // only the last NS loads of each kind can still be in flight.
+  drain_wait(&s.q_full, 0, w);
+  for (int it = (k_issued > NS ? k_issued - NS : 0); it < k_issued; it++)
+    drain_wait(&s.k_full[it % NS], (it / NS) & 1, w);
+  for (int it = (v_issued > NS ? v_issued - NS : 0); it < v_issued; it++)
+    drain_wait(&s.v_full[it % NS], (it / NS) & 1, w);
+}
+
+template <int D, bool DUMP>
+__device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t tmem_O, int nk,
+                                           const WaitCtx& w) {
+  constexpr uint32_t idesc_qk = idesc_i8_s32(BM, BN);
+  constexpr uint32_t idesc_pv = idesc_e4m3_f32(BM, D);
+  const uint32_t q_addr = smem_u32(s.q);
+  const uint32_t p_addr = smem_u32(s.p);
+  bool ok = mbar_wait(&s.q_full, 0, w, kSiteMmaQ);
+  for (int it = 0; ok && it <= nk; it++) {
+    if (it < nk) {  // S = Q K^T for tile it
+      const int st = it % NS;
+      const uint32_t ph = (it / NS) & 1;
+      if (!mbar_wait(&s.k_full[st], ph, w, kSiteMmaK)) break;
+      if (it > 0 && !mbar_wait(&s.s_free, (it - 1) & 1, w, kSiteMmaSFree)) break;
+      tc_fence_after();
+      const uint32_t k_addr = smem_u32(s.k[st]);
+#pragma unroll
+      for (int kk = 0; kk < D / 32; kk++)
+        mma_i8_ss(tmem_S, smem_desc_kmajor(q_addr + kk * 32, D),
+                  smem_desc_kmajor(k_addr + kk * 32, D), idesc_qk, kk > 0);
+      mma_commit(&s.k_empty[st]);
+      mma_commit(&s.s_full);
+    }
+    if (!DUMP && it > 0) {  // O (+)= P V^T for tile it - 1
+      const int j = it - 1;
+      const int st = j % NS;
+      const uint32_t ph = (j / NS) & 1;
+      if (!mbar_wait(&s.v_full[st], ph, w, kSiteMmaV)) break;
+      if (!mbar_wait(&s.p_full, j & 1, w, kSiteMmaP)) break;
+      tc_fence_after();
+      const uint32_t v_addr = smem_u32(s.v[st]);
+#pragma unroll
+      for (int kk = 0; kk < BN / 32; kk++)
+        mma_f8_ss(tmem_O, smem_desc_kmajor(p_addr + kk * 32, BN),
+                  smem_desc_kmajor(v_addr + kk * 32, BN), idesc_pv, (j > 0 || kk > 0));
+      mma_commit(&s.v_empty[st]);
+      mma_commit(&s.o_ready);
+    }
+  }
+  // Drain: all MMAs issued by this thread complete before TMEM is freed.
+  mma_commit(&s.drain);
+  drain_wait(&s.drain, 0, w);
+}
+
+// Softmax / correction / epilogue for one query row per thread.
+template <int D>
+__device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
+                                             uint32_t tmem_O, int bh, int qt, int nk,
+                                             const WaitCtx& w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3;               // TMEM lane quadrant of this warp
+  const int r = quad * 32 + lane;          // row within the tile
+  const int i = qt * BM + r;               // query row
+  const bool valid = i < p.Nq;
+  const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+  const uint32_t tS = tmem_S + lane_off, tO = tmem_O + lane_off;
+  const int lim = valid ? row_limit(i, p) : 0;
+  const float sqC = valid ? __fmul_rn(__ldg(p.q_scale + static_cast<size_t>(bh) * p.nq_blocks + i / 64), p.c0)
+                          : 0.0f;
+  const float* ksc = p.k_scale + static_cast<size_t>(bh) * p.nkv_blocks;
+  uint8_t* prow = s.p + r * BN;
+
+  float m = -INFINITY, l = 0.0f;
+  bool ok = true;
+  for (int it = 0; it < nk; it++) {
+    const int j0 = it * BN;
+    if (!warp_wait(&s.s_full, it & 1, w, kSiteSmS)) { ok = false; break; }
+    tc_fence_after();
+    uint32_t sv[128];
+    {
+      uint32_t (&h0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&sv[0]);
+      uint32_t (&h1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&sv[64]);
+      tmem_ld64(tS, h0);
+      tmem_ld64(tS + 64, h1);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.s_free);
+
+    // scale of each 64-key group of the tile (blocks past the end read as 0)
+    const int g0 = 2 * it, g1 = 2 * it + 1;
+    const float c0 = __fmul_rn(sqC, g0 < p.nkv_blocks ? __ldg(ksc + g0) : 0.0f);
+    const float c1 = __fmul_rn(sqC, g1 < p.nkv_blocks ? __ldg(ksc + g1) : 0.0f);
+    const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
+    const bool full = __all_sync(kFull, nvis == BN);
+
+    // masked max per group in the integer domain: for c >= 0,
+    // max_j fp32(S_j * c) = fp32(max_j S_j * c)
+    int mx0 = INT_MIN, mx1 = INT_MIN;
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 64; j++) mx0 = max(mx0, static_cast<int>(sv[j]));
+#pragma unroll
+      for (int j = 64; j < 128; j++) mx1 = max(mx1, static_cast<int>(sv[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 64; j++) if (j < nvis) mx0 = max(mx0, static_cast<int>(sv[j]));
+#pragma unroll
+      for (int j = 64; j < 128; j++) if (j < nvis) mx1 = max(mx1, static_cast<int>(sv[j]));
+    }
+    const float t0 = mx0 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mx0), c0);
+    const float t1 = mx1 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mx1), c1);
+    const float m_new = fmaxf(m, fmaxf(t0, t1));
+    const float alpha = (m == -INFINITY) ? 0.0f
+                        : (m == m_new)   ? 1.0f
+                                         : ex2_approx(__fsub_rn(m, m_new));
+    const float negm = -m_new;
+
+    // the P tile is free once P V of the previous tile has completed
+    if (it > 0 && !warp_wait(&s.o_ready, (it - 1) & 1, w, kSiteSmO)) { ok = false; break; }
+    tc_fence_after();
+
+    float rs = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 8; c++) {  // 16-key chunks
+      uint32_t pk[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; q4++) {
+        float pv[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const int j = c * 16 + q4 * 4 + e;
+          float x = __fmaf_rn(__int2float_rn(static_cast<int>(sv[j])), j < 64 ? c0 : c1, negm);
+          if (!full && j >= nvis) x = -INFINITY;
+          pv[e] = ex2_approx(x);
+          rs += pv[e];
+        }
+        pk[q4] = cvt_e4m3x2(pv[0] * 256.0f, pv[1] * 256.0f) |
+                 (cvt_e4m3x2(pv[2] * 256.0f, pv[3] * 256.0f) << 16);
+      }
+      *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+    fence_proxy_async_smem();
+
+    // rescale the O row when the running max moved (never before the first P V)
+    if (it > 0 && __any_sync(kFull, alpha != 1.0f)) {
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+#pragma unroll
+        for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), alpha));
+        tmem_st32(tO + c, o);
+      }
+    }
+    l = __fadd_rn(__fmul_rn(l, alpha), rs);
+    m = m_new;
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.p_full);
+  }
+
+  if (!ok || nk == 0) return;
+  if (!warp_wait(&s.o_ready, (nk - 1) & 1, w, kSiteSmEpi)) return;
+  tc_fence_after();
+  const float inv = __frcp_rn(__fmul_rn(256.0f, l));
+  const float* vsc = p.v_scale + static_cast<size_t>(bh) * D;
+  const size_t orow = (static_cast<size_t>(bh) * p.Nq + (valid ? i : 0)) * D;
+#pragma unroll 1
+  for (int c = 0; c < D; c += 32) {
+    uint32_t o[32];
+    tmem_ld32(tO + c, o);
+    if (!valid) continue;
+    float f[32];
+#pragma unroll
+    for (int e = 0; e < 32; e++) f[e] = __uint_as_float(o[e]) * (__ldg(vsc + c + e) * inv);
+    uint32_t b[16];
+#pragma unroll
+    for (int e = 0; e < 16; e++) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+      b[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.o + orow + c);
+#pragma unroll
+    for (int e = 0; e < 4; e++) dst[e] = make_uint4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+    if (p.o_f32) {
+      float4* d32 = reinterpret_cast<float4*>(p.o_f32 + orow + c);
+#pragma unroll
+      for (int e = 0; e < 8; e++) d32[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+    }
+  }
+  if (valid && p.lse)
+    p.lse[static_cast<size_t>(bh) * p.Nq + i] = (m + log2f(l)) * 0.69314718055994531f;
+}
+
+// Score dump (debug): copy the int32 S tile from TMEM to global memory.
+template <int D>
+__device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
+                                          const WaitCtx& w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  if (!warp_wait(&s.s_full, 0, w, kSiteSmS)) return;
+  tc_fence_after();
+  const uint32_t tS = tmem_S + (static_cast<uint32_t>(quad * 32) << 16);
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t v[32];
+    tmem_ld32(tS + c, v);
+    uint4* dst = reinterpret_cast<uint4*>(p.dbg_out + static_cast<size_t>(r) * BN + c);
+#pragma unroll
+    for (int e = 0; e < 8; e++) dst[e] = make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&s.s_free);
+}
+
+template <int D, bool DUMP>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D>& s = *reinterpret_cast<Smem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = DUMP ? p.dbg_qt : static_cast<int>(blockIdx.x);
+  const int bh = DUMP ? p.dbg_bh : static_cast<int>(blockIdx.y);
+
+  // KV tiles this CTA visits: those holding a key visible to its last valid
+  // row (the masks' limits grow with the row index).
+  int kt0 = 0, nk;
+  if (DUMP) {
+    kt0 = p.dbg_kt;
+    nk = 1;
+  } else {
+    const int last = min(p.Nq - 1, qt * BM + BM - 1);
+    nk = (row_limit(last, p) + BN - 1) / BN;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(&s.q_full, 1);
+    for (int i = 0; i < NS; i++) {
+      mbar_init(&s.k_full[i], 1);
+      mbar_init(&s.k_empty[i], 1);
+      mbar_init(&s.v_full[i], 1);
+      mbar_init(&s.v_empty[i], 1);
+    }
+    mbar_init(&s.s_full, 1);
+    mbar_init(&s.s_free, 4);
+    mbar_init(&s.p_full, 4);
+    mbar_init(&s.o_ready, 1);
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t tmem_S = tmem;        // columns [0, 128): int32 scores
+  const uint32_t tmem_O = tmem + 128;  // columns [128, 128 + D): fp32 output
+  const WaitCtx w{p.budget, p.status, &s.abort};
+
+  if (warp == 0) {
+    if (lane == 0) producer<D, DUMP>(s, maps, bh, qt, kt0, nk, w);
+  } else if (warp == 1) {
+    if (lane == 0) mma_issuer<D, DUMP>(s, tmem_S, tmem_O, nk, w);
+  } else {
+    if (DUMP) dump_rows<D>(s, p, tmem_S, w);
+    else softmax_rows<D>(s, p, tmem_S, tmem_O, bh, qt, nk, w);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int D) { return smem_bytes_for(D); }
+
+cudaError_t attn_prepare(int D) {
+  cudaError_t e;
+  if (D == 128) {
+    e = cudaFuncSetAttribute(k_attn<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for(128)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_attn<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes_for(128)));
+  } else {
+    e = cudaFuncSetAttribute(k_attn<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for(64)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_attn<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes_for(64)));
+  }
+  return e;
+}
+
+cudaError_t launch_attn(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
+  dim3 grid((p.Nq + BM - 1) / BM, p.BH);
+  if (p.D == 128)
+    k_attn<128, false><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
+  else
+    k_attn<64, false><<<grid, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_dump(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
+  if (p.D == 128)
+    k_attn<128, true><<<1, kThreads, smem_bytes_for(128), stream>>>(maps, p);
+  else
+    k_attn<64, true><<<1, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+}  // namespace sage

@@ -1,0 +1,279 @@
+// quant.cu -- sage_quant_qk: per-block INT8 quantization of Q and of the
+// mean-smoothed K, and per-channel FP8 e4m3 quantization of V.
+//
+// SageAttention's quantizer (low-bit attention, "Vidu S1" digest section
+// "Infra" and the TurboDiffusion notes on 8-bit block-wise quantization):
+// 64-token blocks, symmetric absmax/127 INT8 codes with round-half-to-even,
+// K smoothed by its per-channel mean over all tokens, V cast to e4m3 with a
+// per-channel absmax/448 scale.
+//
+// Three stream-ordered kernels (the K mean and the V maxima span all tokens
+// of a head, so the K and V codes need a second pass):
+//   pass1    one CTA per (head, 64-token block): Q block codes + scale; fp64
+//            per-channel sums of the K block in ascending token order; V
+//            block per-channel maxima.
+//   finalize one thread per (head, channel): ascending sum of the block sums
+//            -> k_mean; max of the block maxima -> v_scale, 448/absmax.
+//   pass2    one CTA per (head, 64-token block): K - mean block codes + scale;
+//            V codes written channel-major ([B,H,D,Nkv_pad]) through shared
+//            memory so that the attention kernel reads K-major V^T tiles.
+// Memory traffic: 16-byte vectorised bf16 loads; every fp32 operation is an
+// explicit IEEE round-to-nearest intrinsic so the codes match a plain CPU
+// implementation bit for bit.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "quant.cuh"
+#include "sm100.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr int kBlk = 64;
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
+  x[0] = bf16lo(u.x); x[1] = bf16hi(u.x);
+  x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
+  x[4] = bf16lo(u.z); x[5] = bf16hi(u.z);
+  x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Max over the CTA (kThreads threads); every thread gets the result.
+__device__ __forceinline__ float block_max(float v, float* red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();  // `red` may still be read by a previous call
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int i = 1; i < kThreads / 32; i++) r = fmaxf(r, red[i]);
+  return r;
+}
+
+__device__ __forceinline__ int8_t q_i8(float x, float inv) {
+  int q = __float2int_rn(__fmul_rn(x, inv));
+  q = q > 127 ? 127 : (q < -127 ? -127 : q);
+  return static_cast<int8_t>(q);
+}
+
+// Quantize the 64 x D block held as `ch` 16-byte chunks per thread (x[c][8],
+// chunk index c*kThreads + tid), write codes and the block scale.  Rows >=
+// `valid` are written as zero and excluded from the max.
+template <int D, int CH>
+__device__ __forceinline__ void quant_block_store(float (&x)[CH][8], int valid, int8_t* codes,
+                                                  float* scale_out, float* red) {
+  constexpr int kChunksPerRow = D / 8;
+  float a = 0.0f;
+#pragma unroll
+  for (int c = 0; c < CH; c++) {
+    const int chunk = c * kThreads + threadIdx.x;
+    const int row = chunk / kChunksPerRow;
+    if (row < valid) {
+#pragma unroll
+      for (int e = 0; e < 8; e++) a = fmaxf(a, fabsf(x[c][e]));
+    }
+  }
+  a = block_max(a, red);
+  const float scale = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
+  const float inv = (a == 0.0f) ? 0.0f : __fdiv_rn(127.0f, a);
+#pragma unroll
+  for (int c = 0; c < CH; c++) {
+    const int chunk = c * kThreads + threadIdx.x;
+    const int row = chunk / kChunksPerRow;
+    const int col = (chunk % kChunksPerRow) * 8;
+    uint32_t lo = 0, hi = 0;
+    if (row < valid && a != 0.0f) {
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        lo |= (static_cast<uint32_t>(static_cast<uint8_t>(q_i8(x[c][e], inv)))) << (8 * e);
+        hi |= (static_cast<uint32_t>(static_cast<uint8_t>(q_i8(x[c][e + 4], inv)))) << (8 * e);
+      }
+    }
+    *reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * D + col) = make_uint2(lo, hi);
+  }
+  if (threadIdx.x == 0) *scale_out = scale;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
+  constexpr int kChunksPerRow = D / 8;
+  constexpr int CH = kBlk * kChunksPerRow / kThreads;  // chunks per thread
+  __shared__ float red[kThreads / 32];
+  __shared__ __align__(16) uint16_t ks[kBlk * D];
+  __shared__ __align__(16) uint16_t vsm[kBlk * D];
+
+  const int blk = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int nqb = (a.Nq + kBlk - 1) / kBlk;
+  const int nkb = (a.Nkv + kBlk - 1) / kBlk;
+
+  if (blk < nqb) {  // Q block: codes and scale
+    const int valid = min(kBlk, a.Nq - blk * kBlk);
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.q + (static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(blk) * kBlk) * D);
+    float x[CH][8];
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (row < valid) u = __ldg(src + chunk);
+      unpack8(u, x[c]);
+    }
+    int8_t* codes = a.q_i8 + (static_cast<size_t>(bh) * nqb + blk) * kBlk * D;
+    quant_block_store<D, CH>(x, valid, codes, a.q_scale + static_cast<size_t>(bh) * nqb + blk,
+                             red);
+  }
+
+  if (blk < nkb) {  // K block sums and V block maxima
+    const int valid = min(kBlk, a.Nkv - blk * kBlk);
+    const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
+    const uint4* ksrc = reinterpret_cast<const uint4*>(a.k + base);
+    const uint4* vsrc = reinterpret_cast<const uint4*>(a.v + base);
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      if (row < valid) {
+        reinterpret_cast<uint4*>(ks)[chunk] = __ldg(ksrc + chunk);
+        reinterpret_cast<uint4*>(vsm)[chunk] = __ldg(vsrc + chunk);
+      }
+    }
+    __syncthreads();
+    const size_t ws = (static_cast<size_t>(bh) * nkb + blk) * D;
+    const int t = threadIdx.x;
+    if (t < D) {  // fp64 sum of channel t, ascending token order
+      double s = 0.0;
+      for (int r = 0; r < valid; r++)
+        s = __dadd_rn(s, static_cast<double>(__uint_as_float(static_cast<uint32_t>(ks[r * D + t]) << 16)));
+      a.ws_ksum[ws + t] = s;
+    } else if (t < 2 * D) {  // max |V| of channel t - D
+      const int d = t - D;
+      float m = 0.0f;
+      for (int r = 0; r < valid; r++)
+        m = fmaxf(m, fabsf(__uint_as_float(static_cast<uint32_t>(vsm[r * D + d]) << 16)));
+      a.ws_vmax[ws + d] = m;
+    }
+  }
+}
+
+__global__ void k_quant_finalize(QuantArgs a) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int D = a.D;
+  if (idx >= a.BH * D) return;
+  const int bh = idx / D, d = idx % D;
+  const int nkb = (a.Nkv + kBlk - 1) / kBlk;
+  double total = 0.0;
+  float m = 0.0f;
+  for (int b = 0; b < nkb; b++) {
+    const size_t w = (static_cast<size_t>(bh) * nkb + b) * D + d;
+    total = __dadd_rn(total, a.ws_ksum[w]);
+    m = fmaxf(m, a.ws_vmax[w]);
+  }
+  a.k_mean[idx] = __double2float_rn(__ddiv_rn(total, static_cast<double>(a.Nkv)));
+  a.v_scale[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 448.0f);
+  a.ws_vinv[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(448.0f, m);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
+  constexpr int kChunksPerRow = D / 8;
+  constexpr int CH = kBlk * kChunksPerRow / kThreads;
+  __shared__ float red[kThreads / 32];
+  __shared__ __align__(16) uint8_t vt[D * kBlk];  // [d][token] e4m3 codes
+
+  const int blk = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int nkb = (a.Nkv + kBlk - 1) / kBlk;
+  const int nkv_pad = nkb * kBlk;
+  const int valid = min(kBlk, a.Nkv - blk * kBlk);
+  const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
+
+  {  // K - mean, block codes and scale
+    const uint4* src = reinterpret_cast<const uint4*>(a.k + base);
+    const float* mu = a.k_mean + static_cast<size_t>(bh) * D;
+    float x[CH][8];
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      const int col = (chunk % kChunksPerRow) * 8;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (row < valid) u = __ldg(src + chunk);
+      unpack8(u, x[c]);
+#pragma unroll
+      for (int e = 0; e < 8; e++) x[c][e] = __fsub_rn(x[c][e], __ldg(mu + col + e));
+    }
+    int8_t* codes = a.k_i8 + (static_cast<size_t>(bh) * nkb + blk) * kBlk * D;
+    quant_block_store<D, CH>(x, valid, codes, a.k_scale + static_cast<size_t>(bh) * nkb + blk,
+                             red);
+  }
+
+  {  // V codes, transposed through shared memory
+    const uint4* src = reinterpret_cast<const uint4*>(a.v + base);
+    const float* inv = a.ws_vinv + static_cast<size_t>(bh) * D;
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      const int col = (chunk % kChunksPerRow) * 8;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (row < valid) u = __ldg(src + chunk);
+      float x[8];
+      unpack8(u, x);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float i0 = __ldg(inv + col + e), i1 = __ldg(inv + col + e + 1);
+        uint32_t p = cvt_e4m3x2(__fmul_rn(x[e], i0), __fmul_rn(x[e + 1], i1));
+        if (i0 == 0.0f || row >= valid) p &= 0xFF00u;  // zero channel or padding token
+        if (i1 == 0.0f || row >= valid) p &= 0x00FFu;
+        vt[(col + e) * kBlk + row] = static_cast<uint8_t>(p & 0xFF);
+        vt[(col + e + 1) * kBlk + row] = static_cast<uint8_t>(p >> 8);
+      }
+    }
+    __syncthreads();
+    // D rows of 64 bytes: 4 x 16-byte chunks per channel
+    uint8_t* dst = a.v_f8 + static_cast<size_t>(bh) * D * nkv_pad + static_cast<size_t>(blk) * kBlk;
+    for (int chunk = threadIdx.x; chunk < D * (kBlk / 16); chunk += kThreads) {
+      const int d = chunk / (kBlk / 16), part = chunk % (kBlk / 16);
+      *reinterpret_cast<uint4*>(dst + static_cast<size_t>(d) * nkv_pad + part * 16) =
+          reinterpret_cast<const uint4*>(vt)[chunk];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream) {
+  const int nqb = (a.Nq + kBlk - 1) / kBlk;
+  const int nkb = (a.Nkv + kBlk - 1) / kBlk;
+  dim3 g1(nqb > nkb ? nqb : nkb, a.BH);
+  dim3 g2(nkb, a.BH);
+  const int nfin = a.BH * a.D;
+  if (a.D == 128) {
+    k_quant_pass1<128><<<g1, kThreads, 0, stream>>>(a);
+    k_quant_finalize<<<(nfin + 255) / 256, 256, 0, stream>>>(a);
+    k_quant_pass2<128><<<g2, kThreads, 0, stream>>>(a);
+  } else {
+    k_quant_pass1<64><<<g1, kThreads, 0, stream>>>(a);
+    k_quant_finalize<<<(nfin + 255) / 256, 256, 0, stream>>>(a);
+    k_quant_pass2<64><<<g2, kThreads, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sage

@@ -1,0 +1,29 @@
+// quant.cuh -- launch interface of the quantization kernels (sage_quant_qk).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace sage {
+
+struct QuantArgs {
+  const uint16_t* q;  // bf16 bits [BH, Nq, D]
+  const uint16_t* k;  // bf16 bits [BH, Nkv, D]
+  const uint16_t* v;  // bf16 bits [BH, Nkv, D]
+  int BH, Nq, Nkv, D;
+  int8_t* q_i8;
+  float* q_scale;
+  int8_t* k_i8;
+  float* k_scale;
+  float* k_mean;
+  uint8_t* v_f8;
+  float* v_scale;
+  double* ws_ksum;  // [BH, nkb, D] fp64 per-block K channel sums
+  float* ws_vmax;   // [BH, nkb, D] per-block V channel maxima
+  float* ws_vinv;   // [BH, D] 448 / channel absmax (0 for an all-zero channel)
+};
+
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream);
+
+}  // namespace sage

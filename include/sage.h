@@ -1,0 +1,200 @@
+/*
+ * sage.h -- C ABI of the B200 (sm_100a) SageAttention-style quantized
+ * attention library (libsage_b200.so).
+ *
+ * What it computes.  Attention O = softmax(Q K^T / sqrt(D) + mask) V for bf16
+ * Q, K, V, approximated the SageAttention way: Q and K quantized to INT8 per
+ * block of 64 tokens (K after subtracting its per-channel mean over tokens),
+ * V cast to FP8 e4m3 with a per-channel scale, Q K^T on INT8 tensor cores,
+ * softmax taken online in fp32, P quantized to FP8 e4m3 and P V on FP8 tensor
+ * cores with fp32 accumulation.
+ *   - "SageAttention: low-bit quantized attention, plug-and-play in place of
+ *     FlashAttention" -- Crossing podcast show notes (wav.pub), section
+ *     "硬件上明明有更快的计算单元"; English notes (elsewhere.news), same section.
+ *   - Per-block 8-bit quantization because per-tensor and per-channel scales
+ *     are stretched by outliers -- "Vidu S1" technical digest
+ *     (zhao9797.github.io), section "Infra", linear-layer quantization bullet.
+ *   - 8-bit block-wise quantization on INT8 tensor cores -- reportify.cn
+ *     TurboDiffusion notes, "W8A8线性层量化" bullet.
+ *   - Streaming generation attends over a KV cache of earlier frames, which is
+ *     what the block-causal mask expresses -- "Vidu S1" digest, section
+ *     "Infra", sliding-window decoding paragraph.
+ * The pages print neither the block sizes nor the rounding rules; the values
+ * used here (64-token INT8 blocks, absmax/127 with round-half-to-even, K mean
+ * over all tokens, e4m3 V with absmax/448 per channel, P scale 2^8, KV tiles of
+ * 128) are this library's readings and are documented with each call.
+ *
+ * Conventions shared by every call.
+ *   - Memory: the library never allocates device memory.  The caller owns
+ *     every buffer (inputs, outputs, workspace).  All pointers named "device"
+ *     must be device-accessible addresses on the current CUDA device and
+ *     16-byte aligned.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *     default stream).  All device work is enqueued asynchronously on it; no
+ *     call synchronizes except sage_sync_status.
+ *   - Errors: argument errors are detected on the host before anything is
+ *     enqueued and return SAGE_ERR_INVALID_ARG or SAGE_ERR_UNSUPPORTED.
+ *     A failed launch returns SAGE_ERR_CUDA.  Every wait inside a kernel is
+ *     bounded; a wait that runs out records SAGE_ERR_TIMEOUT in a device-side
+ *     status word and the kernel returns early with its outputs undefined;
+ *     sage_sync_status reports and clears it.  No call throws or aborts.
+ *   - Layouts are row-major.  Padded token counts: N_pad = ceil(N/64)*64.
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SAGE_ABI_VERSION 1
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or mask   */
+    SAGE_ERR_UNSUPPORTED = 2, /* valid request outside this build's support  */
+    SAGE_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed         */
+    SAGE_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out           */
+} sage_status;
+
+typedef enum {
+    SAGE_MASK_NONE = 0,
+    /* key j visible to query i iff j <= i + (Nkv - Nq): queries are the
+     * newest Nq tokens of the Nkv-token cache (bottom-right alignment). */
+    SAGE_MASK_CAUSAL = 1,
+    /* block-causal over blocks of mask_block tokens (one latent frame in a
+     * streaming video step): key j visible to query i iff
+     * floor(j / mask_block) <= floor((i + Nkv - Nq) / mask_block). */
+    SAGE_MASK_BLOCK_CAUSAL = 2
+} sage_mask;
+
+/* Problem shape.  Inputs are [B, H, Nq, D] (Q) and [B, H, Nkv, D] (K, V).
+ * Supported: B, H, Nq, Nkv >= 1; D in {64, 128}; B*H <= 65535. */
+typedef struct {
+    int B, H, Nq, Nkv, D;
+} sage_shape;
+
+/* The quantized operands produced by sage_quant_qk and read by
+ * sage_attn_fwd.  All device pointers, caller-allocated, 16-byte aligned:
+ *   q_i8    int8  [B, H, Nq_pad,  D]  Q codes; rows >= Nq are 0
+ *   q_scale f32   [B, H, Nq_pad/64]   per-block Q scale (absmax/127)
+ *   k_i8    int8  [B, H, Nkv_pad, D]  codes of K - k_mean; rows >= Nkv are 0
+ *   k_scale f32   [B, H, Nkv_pad/64]  per-block K scale
+ *   k_mean  f32   [B, H, D]           per-channel mean of K over all Nkv tokens
+ *   v_f8    e4m3  [B, H, D, Nkv_pad]  V codes, CHANNEL-major (transposed):
+ *                                     byte ((b*H+h)*D + d)*Nkv_pad + n;
+ *                                     tokens n >= Nkv are 0
+ *   v_scale f32   [B, H, D]           per-channel V scale (absmax/448)
+ * Dequantization: q = q_i8 * q_scale[n/64]; k = k_i8 * k_scale[n/64] + k_mean;
+ * v = e4m3_value(v_f8) * v_scale[d]. */
+typedef struct {
+    int8_t *q_i8;
+    float *q_scale;
+    int8_t *k_i8;
+    float *k_scale;
+    float *k_mean;
+    uint8_t *v_f8;
+    float *v_scale;
+} sage_qkv_quant;
+
+/* Byte sizes of the seven sage_qkv_quant buffers, in struct order
+ * (q_i8, q_scale, k_i8, k_scale, k_mean, v_f8, v_scale).
+ * Returns SAGE_ERR_INVALID_ARG for a null pointer or an invalid shape. */
+sage_status sage_quant_buffer_bytes(const sage_shape *shape, size_t sizes[7]);
+
+/* Device workspace sage_quant_qk needs for `shape` (bytes; 0 on an invalid
+ * shape).  It holds per-64-token-block fp64 K channel sums and V channel
+ * maxima: B*H*ceil(Nkv/64)*D*12 + B*H*D*4 bytes. */
+size_t sage_quant_workspace_bytes(const sage_shape *shape);
+
+/* Quantize Q, K and V (all device, bf16, contiguous [B,H,N,D]).
+ *
+ *   Q: per (b, h, 64-token block): a = max|Q| over the block, q_scale = a/127,
+ *      q_i8 = clamp(round_half_even(Q * fp32(127/a)), -127, 127); a = 0 gives
+ *      scale 0 and codes 0.
+ *   K: k_mean[d] = fp32(S/Nkv) with S the fp64 sum of K[:, d] taken as
+ *      ascending 64-token block sums (each summed in ascending token order)
+ *      added in ascending block order; then the block quantization above on
+ *      fp32(K - k_mean).
+ *   V: per channel, a = max|V[:, d]| over all tokens, v_scale = a/448,
+ *      v_f8 = e4m3_rne_satfinite(V * fp32(448/a)).
+ * All fp32 operations are single IEEE operations rounded to nearest-even, so
+ * the outputs are reproducible bit for bit.
+ *
+ * `out` points to caller-allocated buffers sized by sage_quant_buffer_bytes;
+ * `workspace` to at least sage_quant_workspace_bytes(shape) device bytes
+ * (contents need not be initialised; they are overwritten).
+ * Enqueues three kernels on `stream`.  Returns SAGE_OK or an error (above). */
+sage_status sage_quant_qk(const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                          const sage_shape *shape, const sage_qkv_quant *out,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Fused quantized attention over the output of sage_quant_qk.
+ *
+ * Per query row i (row limit lim_i from `mask`, see sage_mask), over KV tiles
+ * of 128 keys in ascending order (only tiles holding a visible key):
+ *   S    = q_i8 . k_i8 (exact int32 on the INT8 tensor cores)
+ *   c    = fp32(fp32(q_scale * C0) * k_scale), C0 = fp32(log2(e)/sqrt(D))
+ *   m    = max(m, max_j fp32(S*c))   (running max in the log2 domain)
+ *   p    = exp2(fma(S, c, -m)) in fp32; l = l*alpha + sum_j p
+ *   P    = e4m3(p * 256); O_acc = O_acc*alpha + P . v_f8 (FP8 tensor cores,
+ *          fp32 accumulation), alpha = exp2(m_old - m_new)
+ *   O    = O_acc * v_scale[d] / (256 * l), rounded to bf16.
+ * Softmax invariance makes the K-mean subtraction exact in real arithmetic.
+ *
+ *   mask        a sage_mask value; CAUSAL and BLOCK_CAUSAL need Nkv >= Nq
+ *   mask_block  block length for SAGE_MASK_BLOCK_CAUSAL (>= 1), else ignored
+ *   o_bf16      device bf16 [B, H, Nq, D] output (required)
+ *   o_f32       device f32  [B, H, Nq, D] output before bf16 rounding, or NULL
+ *   lse         device f32  [B, H, Nq] natural-log log-sum-exp of the
+ *               dequantized scaled scores, or NULL
+ * One kernel launch on `stream`. */
+sage_status sage_attn_fwd(const sage_qkv_quant *qkv, const sage_shape *shape, int mask,
+                          int mask_block, void *o_bf16, float *o_f32, float *lse, void *stream);
+
+/* Debug: run the attention kernel's load + INT8 MMA path on selected tiles
+ * and copy the int32 score tile it leaves in tensor memory to `out`.
+ *   tiles  host int array of n_tiles triples (bh, qt, kt): head index b*H+h,
+ *          query tile (rows qt*128 .. qt*128+127), KV tile (keys kt*128 ..)
+ *   out    device int32 [n_tiles, 128, 128]: out[t][r][c] = S of query row
+ *          qt*128+r and key kt*128+c (rows/keys past the padded ends read
+ *          as zero codes).
+ * Tiles outside the shape give SAGE_ERR_INVALID_ARG.  n_tiles <= 65535. */
+sage_status sage_debug_qk_int32(const sage_qkv_quant *qkv, const sage_shape *shape,
+                                const int *tiles, int n_tiles, int32_t *out, void *stream);
+
+/* Debug: launch one CTA that waits on a shared-memory barrier nothing ever
+ * arrives at, with a budget of `budget_cycles` SM clock cycles (1 .. 2^40).
+ * The wait gives up, records SAGE_ERR_TIMEOUT in the status word and the
+ * kernel returns.  Exercises the bounded-wait path every kernel uses. */
+sage_status sage_debug_timeout_probe(long long budget_cycles, void *stream);
+
+/* Debug: y[i] = e4m3 code of x[i] (round to nearest even, saturating to
+ * +-448, NaN to NaN), computed with the conversion instruction the kernels
+ * use for V and P.  x: device f32 [n], y: device uint8 [n]. */
+sage_status sage_debug_e4m3(const float *x, uint8_t *y, size_t n, void *stream);
+
+/* Debug: y[i] = 2^x[i] as the attention kernel's softmax computes it (the
+ * hardware approximate base-2 exponential, subnormal results flushed to
+ * zero).  x, y: device f32 [n]. */
+sage_status sage_debug_exp2(const float *x, float *y, size_t n, void *stream);
+
+/* Synchronize `stream`, then return and clear the device-side status word:
+ * SAGE_ERR_TIMEOUT if any kernel's bounded wait ran out since the last call,
+ * SAGE_ERR_CUDA if the synchronization failed, else SAGE_OK. */
+sage_status sage_sync_status(void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *sage_status_string(sage_status status);
+
+/* SAGE_ABI_VERSION of the loaded library. */
+int sage_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H */

@@ -1,0 +1,86 @@
+"""The C-ABI library loads and exports every symbol include/sage.h declares,
+and its host-side logic (sizes, argument validation, status strings) works
+without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_quantized_attention_sage_b200 as sage
+from bit_quantized_attention_sage_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "sage.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return sage.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.sage_abi_version() == 1
+    for code in range(5):
+        assert L.sage_status_string(code)
+    assert L.sage_status_string(99) == b"unknown status"
+
+
+def test_buffer_and_workspace_sizes(L):
+    s = sage.make_shape(1, 2, 1000, 3000, 128)
+    b = sage.buffer_bytes(s)
+    nqp, nkp = 1024, 3008
+    assert b["q_i8"] == 2 * nqp * 128 and b["q_scale"] == 2 * 16 * 4
+    assert b["k_i8"] == 2 * nkp * 128 and b["k_scale"] == 2 * 47 * 4
+    assert b["k_mean"] == 2 * 128 * 4 and b["v_scale"] == 2 * 128 * 4
+    assert b["v_f8"] == 2 * 128 * nkp
+    assert sage.workspace_bytes(s) == 2 * 47 * 128 * 12 + 2 * 128 * 4
+
+
+@pytest.mark.parametrize("shape", [(0, 1, 8, 8, 128), (1, 1, 8, 8, 96), (1, 1, 0, 8, 64),
+                                   (300, 300, 8, 8, 64)])
+def test_invalid_shapes(L, shape):
+    s = sage.make_shape(*shape)
+    sizes = (ctypes.c_size_t * 7)()
+    assert L.sage_quant_buffer_bytes(ctypes.byref(s), sizes) == 1
+    assert L.sage_quant_workspace_bytes(ctypes.byref(s)) == 0
+
+
+def test_invalid_arguments_are_rejected_before_any_launch(L):
+    s = sage.make_shape(1, 1, 64, 64, 128)
+    null = sage._QKV()
+    assert L.sage_quant_qk(None, None, None, ctypes.byref(s), ctypes.byref(null), None, 0,
+                           None) == 1
+    assert L.sage_attn_fwd(ctypes.byref(null), ctypes.byref(s), 0, 0, None, None, None, None) == 1
+    # misaligned pointers
+    fake = sage._QKV(*([16 * 1024 + 4] * 7))
+    assert L.sage_attn_fwd(ctypes.byref(fake), ctypes.byref(s), 0, 0, ctypes.c_void_p(4096),
+                           None, None, None) == 1
+    ok = sage._QKV(*([16 * 1024] * 7))
+    # bad mask, causal with Nkv < Nq, block-causal without a block length
+    assert L.sage_attn_fwd(ctypes.byref(ok), ctypes.byref(s), 7, 0, ctypes.c_void_p(4096),
+                           None, None, None) == 1
+    s2 = sage.make_shape(1, 1, 128, 64, 128)
+    assert L.sage_attn_fwd(ctypes.byref(ok), ctypes.byref(s2), 1, 0, ctypes.c_void_p(4096),
+                           None, None, None) == 1
+    assert L.sage_attn_fwd(ctypes.byref(ok), ctypes.byref(s), 2, 0, ctypes.c_void_p(4096),
+                           None, None, None) == 1
+    assert L.sage_debug_timeout_probe(0, None) == 1
+    # tile outside the shape
+    tiles = (ctypes.c_int * 3)(0, 5, 0)
+    assert L.sage_debug_qk_int32(ctypes.byref(ok), ctypes.byref(s), tiles, 1,
+                                 ctypes.c_void_p(4096), None) == 1
