@@ -63,6 +63,8 @@ def lib():
         L.sage_quant_workspace_bytes.argtypes = [P]
         L.sage_quant_qk.restype = I
         L.sage_quant_qk.argtypes = [P, P, P, P, P, P, SZ, P]
+        L.sage_quant_qk_noalloc.restype = I
+        L.sage_quant_qk_noalloc.argtypes = [P, P, P, P, P, P]
         L.sage_attn_fwd.restype = I
         L.sage_attn_fwd.argtypes = [P, P, I, I, P, P, P, P]
         L.sage_debug_qk_int32.restype = I
@@ -158,6 +160,26 @@ def quant_qk(q, k, v, out=None, workspace=None, stream=None):
     _check(lib().sage_quant_qk(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(qs),
                                _ptr(workspace), workspace.numel(), _stream(stream)),
            "sage_quant_qk")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # SAGE_NOALLOC_SCRATCH_BYTES in include/sage.h
+
+
+def quant_qk_noalloc(q, k, v, out, stream=None):
+    """sage_quant_qk_noalloc: quantize into caller-provided outputs without
+    any workspace, for callers that cannot allocate device memory (the
+    library's fixed 16 MiB scratch array is used instead; calls on one device
+    share it, so do not overlap them across streams)."""
+    shape = out.shape
+    need = workspace_bytes(shape)
+    if need > NOALLOC_SCRATCH_BYTES:
+        raise SageError(2, "sage_quant_qk_noalloc: this shape needs %d bytes of scratch, more "
+                           "than the fixed %d-byte array" % (need, NOALLOC_SCRATCH_BYTES))
+    qs = out.struct()
+    _check(lib().sage_quant_qk_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape),
+                                       ctypes.byref(qs), _stream(stream)),
+           "sage_quant_qk_noalloc")
     return out
 
 

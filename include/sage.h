@@ -132,6 +132,42 @@ sage_status sage_quant_qk(const void *q_bf16, const void *k_bf16, const void *v_
                           const sage_shape *shape, const sage_qkv_quant *out,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the fixed device scratch array sage_quant_qk_noalloc uses: 16 MiB
+ * on every GPU that loads the library, held until the process exits. */
+#define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* sage_quant_qk for callers that cannot allocate device memory.
+ *
+ * The pages describe no such call; it exists for callers that are handed only
+ * their input and output buffers and are not allowed to allocate -- for
+ * example code running inside a memory pool that has been sized and locked in
+ * advance, a real-time loop that must not enter the allocator, or a plugin of
+ * a host framework that owns all device memory.  Such callers cannot supply
+ * the workspace sage_quant_qk needs, so this variant keeps it in one fixed,
+ * library-owned device array of SAGE_NOALLOC_SCRATCH_BYTES.  It computes
+ * exactly what sage_quant_qk computes (same kernels, same results) and calls
+ * no allocation routine.
+ *
+ *   q_bf16, k_bf16, v_bf16, shape, out, stream: as for sage_quant_qk.
+ *
+ * Errors: SAGE_ERR_INVALID_ARG for a bad shape or pointer;
+ * SAGE_ERR_UNSUPPORTED if sage_quant_workspace_bytes(shape) exceeds
+ * SAGE_NOALLOC_SCRATCH_BYTES (e.g. B1 H24 Nkv26520 D128 fits, B1 H40 Nkv75600
+ * D128 does not) -- nothing is enqueued then; SAGE_ERR_CUDA if a launch
+ * fails.
+ *
+ * Sharing: all calls on a device use the same array, which keeps whatever
+ * the last call left in it.  Nothing in it needs to start at zero (each call
+ * writes every cell it later reads), but two calls whose work can overlap on
+ * the GPU (e.g. on two streams with no ordering between them) race on it and
+ * give undefined results; order such calls on one stream.
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current).  Make that first call
+ * before any stream capture. */
+sage_status sage_quant_qk_noalloc(const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                                  const sage_shape *shape, const sage_qkv_quant *out,
+                                  void *stream);
+
 /* Fused quantized attention over the output of sage_quant_qk.
  *
  * Per query row i (row limit lim_i from `mask`, see sage_mask), over KV tiles
