@@ -309,7 +309,7 @@ typedef struct {
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
 
-/* Width, in units of p*256, of the set of e4m3 codes that p*256*(1 +- eps)
+/* Width, in units of y = p*2^8, of the set of e4m3 codes that y*(1 +- eps)
  * can round to; zero when the uncertainty interval does not straddle a
  * rounding boundary. */
 static double e4m3_flip_gap(double y, double eps)
@@ -336,10 +336,11 @@ static double e4m3_flip_gap(double y, double eps)
  *   sqC   = fp32(sq[i/64] * C0); c_ij = fp32(sqC * sk[j/64])
  *   S_ij  = sum_d q8 k8 (exact integer)
  *   t_ij  = fp32(fp32(S_ij) * c_ij)             (for the max)
- *   x_ij  = fmaf(fp32(S_ij), c_ij, -m_k); p_ij = fp32(exp2(x_ij))
- *   l is accumulated in fp32 from p (before quantization),
- *   w_ij  = e4m3(p_ij * 256) (P scale 2^8), V_j = e4m3 code values,
- *   O     = O_acc * vs[d] / (256 * l).
+ *   P is quantized with the fixed scale 2^8, folded into the exponent:
+ *   y_ij  = fp32(exp2(fmaf(fp32(S_ij), c_ij, fp32(8 - m_k))))   (~ 256 p_ij)
+ *   l is accumulated in fp32 from y (before quantization),
+ *   w_ij  = e4m3(y_ij), V_j = e4m3 code values,
+ *   O     = O_acc * vs[d] / l;  lse = (m + log2(l) - 8) * ln 2.
  * Identity mode: t_ij = (q_i . k_j) * log2(e)/sqrt(D), w = p, all fp64.
  */
 static void attend_row(const attn_job *J, long r)
@@ -402,7 +403,8 @@ static void attend_row(const attn_job *J, long r)
             alpha = (mf == -INFINITY) ? 0.0 : (double)exp2_f32(mf - mn);
             mf = mn;
         }
-        /* probabilities and the P.V contribution */
+        /* probabilities (scaled by 2^8 in quantized mode) and the P.V contribution */
+        const float nm8 = 8.0f - mf;
         for (int d = 0; d < D; d++) {
             acc[d] = 0.0;
             sacc[d] = 0.0;
@@ -417,10 +419,9 @@ static void attend_row(const attn_job *J, long r)
                 for (int d = 0; d < D; d++)
                     acc[d] += p * J->vd[j * D + d];
             } else {
-                float x = fmaf((float)S[jj], c[jj], -mf);
-                float p = exp2_f32(x);
-                rowsum_f += p;
-                float y = p * 256.0f;
+                float x = fmaf((float)S[jj], c[jj], nm8);
+                float y = exp2_f32(x);
+                rowsum_f += y;
                 double w = orc_e4m3_decode(orc_e4m3_encode(y));
                 double gap = sl ? e4m3_flip_gap((double)y, J->eps) : 0.0;
                 for (int d = 0; d < D; d++) {
@@ -449,13 +450,13 @@ static void attend_row(const attn_job *J, long r)
             J->lse[r] = (m + log2(l)) * 0.6931471805599453;
     } else {
         for (int d = 0; d < D; d++) {
-            double f = (double)J->vs[d] / (256.0 * (double)lf);
+            double f = (double)J->vs[d] / (double)lf;
             o[d] = o[d] * f;
             if (sl)
                 sl[d] = sl[d] * f;
         }
         if (J->lse)
-            J->lse[r] = ((double)mf + log2((double)lf)) * 0.6931471805599453;
+            J->lse[r] = ((double)mf + log2((double)lf) - 8.0) * 0.6931471805599453;
     }
     free(acc);
     free(sacc);
