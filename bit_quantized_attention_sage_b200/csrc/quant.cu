@@ -12,8 +12,8 @@
 //   pass1    one CTA per (head, 64-token block): Q block codes + scale; fp64
 //            per-channel sums of the K block in ascending token order; V
 //            block per-channel maxima.
-//   finalize one thread per (head, channel): ascending sum of the block sums
-//            -> k_mean; max of the block maxima -> v_scale, 448/absmax.
+//   finalize one CTA per (head, 32 channels): ascending sum of the block
+//            sums -> k_mean; max of the block maxima -> v_scale, 448/absmax.
 //   pass2    one CTA per (head, 64-token block): K - mean block codes + scale;
 //            V codes written channel-major ([B,H,D,Nkv_pad]) through shared
 //            memory so that the attention kernel reads K-major V^T tiles.
@@ -171,22 +171,47 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
   }
 }
 
-__global__ void k_quant_finalize(QuantArgs a) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+// One CTA per (head, 32 channels).  The fp64 block sums of a channel must be
+// added one after the other in ascending block order (the canonical order
+// that makes the mean reproducible), so the CTA stages chunks of block sums
+// in shared memory with coalesced loads by all its threads, and then one
+// thread per channel adds its chunk in order.  The V block maxima are
+// reduced on the fly (max is order-free).
+constexpr int kFinChunk = 128;  // blocks per staged chunk
+constexpr int kFinCh = 32;      // channels per CTA
+
+__global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
+  __shared__ double part[kFinChunk][kFinCh];
+  __shared__ float vred[kThreads / kFinCh][kFinCh];
   const int D = a.D;
-  if (idx >= a.BH * D) return;
-  const int bh = idx / D, d = idx % D;
+  const int bh = blockIdx.y;
+  const int d0 = blockIdx.x * kFinCh;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
+  const int lane = threadIdx.x % kFinCh;       // channel d0 + lane
+  const int rowg = threadIdx.x / kFinCh;       // 0 .. 7
   double total = 0.0;
   float m = 0.0f;
-  for (int b = 0; b < nkb; b++) {
-    const size_t w = (static_cast<size_t>(bh) * nkb + b) * D + d;
-    total = __dadd_rn(total, a.ws_ksum[w]);
-    m = fmaxf(m, a.ws_vmax[w]);
+  for (int b0 = 0; b0 < nkb; b0 += kFinChunk) {
+    const int nb = min(kFinChunk, nkb - b0);
+    for (int r = rowg; r < nb; r += kThreads / kFinCh) {
+      const size_t w = (static_cast<size_t>(bh) * nkb + b0 + r) * D + d0 + lane;
+      part[r][lane] = a.ws_ksum[w];
+      m = fmaxf(m, a.ws_vmax[w]);
+    }
+    __syncthreads();
+    if (threadIdx.x < kFinCh)
+      for (int r = 0; r < nb; r++) total = __dadd_rn(total, part[r][threadIdx.x]);
+    __syncthreads();
   }
-  a.k_mean[idx] = __double2float_rn(__ddiv_rn(total, static_cast<double>(a.Nkv)));
-  a.v_scale[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 448.0f);
-  a.ws_vinv[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(448.0f, m);
+  vred[rowg][lane] = m;
+  __syncthreads();
+  if (threadIdx.x < kFinCh) {
+    for (int g = 1; g < kThreads / kFinCh; g++) m = fmaxf(m, vred[g][threadIdx.x]);
+    const int idx = bh * D + d0 + threadIdx.x;
+    a.k_mean[idx] = __double2float_rn(__ddiv_rn(total, static_cast<double>(a.Nkv)));
+    a.v_scale[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 448.0f);
+    a.ws_vinv[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(448.0f, m);
+  }
 }
 
 template <int D>
@@ -224,25 +249,30 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   }
 
   {  // V codes, transposed through shared memory
-    const uint4* src = reinterpret_cast<const uint4*>(a.v + base);
-    const float* inv = a.ws_vinv + static_cast<size_t>(bh) * D;
+    // thread t owns token row t % 64 and channels [g*DG, g*DG + DG) with
+    // g = t / 64; a warp then stores 32 consecutive tokens of one channel per
+    // instruction (32 bytes, no bank conflict), and the rows are written out
+    // as 16-byte chunks.
+    constexpr int DG = D / (kThreads / kBlk);  // channels per thread: 32 (D=128) or 16
+    const int row = threadIdx.x % kBlk;
+    const int g = threadIdx.x / kBlk;
+    const uint4* src = reinterpret_cast<const uint4*>(a.v + base + static_cast<size_t>(row) * D + g * DG);
+    const float* inv = a.ws_vinv + static_cast<size_t>(bh) * D + g * DG;
 #pragma unroll
-    for (int c = 0; c < CH; c++) {
-      const int chunk = c * kThreads + threadIdx.x;
-      const int row = chunk / kChunksPerRow;
-      const int col = (chunk % kChunksPerRow) * 8;
+    for (int c = 0; c < DG / 8; c++) {
       uint4 u = make_uint4(0, 0, 0, 0);
-      if (row < valid) u = __ldg(src + chunk);
+      if (row < valid) u = __ldg(src + c);
       float x[8];
       unpack8(u, x);
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
-        const float i0 = __ldg(inv + col + e), i1 = __ldg(inv + col + e + 1);
+        const int d = c * 8 + e;
+        const float i0 = __ldg(inv + d), i1 = __ldg(inv + d + 1);
         uint32_t p = cvt_e4m3x2(__fmul_rn(x[e], i0), __fmul_rn(x[e + 1], i1));
         if (i0 == 0.0f || row >= valid) p &= 0xFF00u;  // zero channel or padding token
         if (i1 == 0.0f || row >= valid) p &= 0x00FFu;
-        vt[(col + e) * kBlk + row] = static_cast<uint8_t>(p & 0xFF);
-        vt[(col + e + 1) * kBlk + row] = static_cast<uint8_t>(p >> 8);
+        vt[(g * DG + d) * kBlk + row] = static_cast<uint8_t>(p & 0xFF);
+        vt[(g * DG + d + 1) * kBlk + row] = static_cast<uint8_t>(p >> 8);
       }
     }
     __syncthreads();
@@ -263,14 +293,14 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream) {
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
   dim3 g1(nqb > nkb ? nqb : nkb, a.BH);
   dim3 g2(nkb, a.BH);
-  const int nfin = a.BH * a.D;
+  dim3 gf(a.D / kFinCh, a.BH);
   if (a.D == 128) {
     k_quant_pass1<128><<<g1, kThreads, 0, stream>>>(a);
-    k_quant_finalize<<<(nfin + 255) / 256, 256, 0, stream>>>(a);
+    k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
     k_quant_pass2<128><<<g2, kThreads, 0, stream>>>(a);
   } else {
     k_quant_pass1<64><<<g1, kThreads, 0, stream>>>(a);
-    k_quant_finalize<<<(nfin + 255) / 256, 256, 0, stream>>>(a);
+    k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
     k_quant_pass2<64><<<g2, kThreads, 0, stream>>>(a);
   }
   return cudaGetLastError();
