@@ -8,42 +8,26 @@
 // quantized to FP8 e4m3 with a fixed 2^8 scale and P V on FP8 tensor cores
 // with fp32 accumulation.
 //
-// One CTA per SM owns two 128-row query tiles (A and B) of one (batch, head)
-// and streams the visible KV tiles of 128 keys.  512 threads, launched at
-// 128 registers each and re-split per warpgroup with setmaxnreg (the shares
-// add up to at most the launch allocation):
-//   WG0  (56 regs)  warp 0: TMA producer of both Q tiles (once) and of K
-//                   through a 4-stage shared-memory ring; warp 2: producer of
-//                   V^T through its own 4-stage ring (separate threads, so a
-//                   full V ring never holds back K loads).  Tiles further
-//                   ahead are prefetched into L2, since the CTAs of a head
-//                   run in step and would otherwise all wait for the same
-//                   DRAM fetch.
-//                   warp 1: owns all 512 TMEM columns (S_A, S_B: 128 x 128
-//                   int32; O_A, O_B: 128 x D fp32); one elected thread
-//                   issues every tcgen05.mma: S_X = Q_X K^T (kind::i8),
-//                   O_X (+)= P_X V^T (kind::f8f6f4).
-//   WG1, WG2 (184)  softmax of tile A and tile B: thread t owns query row t
-//                   (TMEM lane t).  The S columns are seeded with the bit
-//                   pattern of 1.5 * 2^23 before every Q K^T, so the int32
-//                   accumulator reads as the fp32 value 12582912 + S: no
-//                   conversion per score.  Per KV tile: load S, re-seed,
-//                   masked max per 64-key scale group (3-input maxima),
-//                   running max, rescale factor alpha to the correction
-//                   warps, then -- taking turns with the other softmax
-//                   warpgroup so that one warpgroup's exp2-heavy phase runs
-//                   while the other does its loads and maxima --
-//                   y = exp2(fma(S, c, 8 - m)) (P scale 2^8) with packed
-//                   fp32x2 arithmetic, row sum, e4m3(y) into the
-//                   128-byte-swizzled shared-memory P tile of its query tile.
-//   WG3  (80 regs)  correction and epilogue: rescales O_X in TMEM by alpha
-//                   when a row's max moved (between P V of consecutive
-//                   tiles), and finally writes O * v_scale / l as bf16 (plus
-//                   optional fp32 O and lse).
+// One CTA owns 128 query rows of one (batch, head) and streams the visible
+// KV tiles of 128 keys.  Warp roles (192 threads, two CTAs per SM):
+//   warp 0      TMA producer: the Q tile once, then K and V^T tiles through
+//               a two-stage shared-memory ring (128-byte swizzle).
+//   warp 1      allocates 256 TMEM columns (S: 128 x 128 int32, O: 128 x D
+//               fp32) and one elected thread issues every tcgen05.mma:
+//               S = Q K^T (kind::i8) for tile k+1 while the softmax warps
+//               work on tile k, then O (+)= P V^T (kind::f8f6f4).
+//   warps 2-5   softmax: thread t of the warpgroup owns query row t (TMEM
+//               lane t).  Per tile: load the int32 score row from TMEM, take
+//               the masked max in the integer domain per 64-key scale group,
+//               update the running max, y = exp2(fma(S, c, 8 - m)) (P scale
+//               2^8 folded into the exponent; S converted exactly without
+//               the conversion unit as as_float(S + 0x4B400000) - 1.5*2^23)
+//               with packed fp32x2 arithmetic, row sum, e4m3(y) into the
+//               swizzled shared-memory P tile, and rescale the O row in TMEM
+//               when the max moved.  Epilogue: O * v_scale / l -> bf16 (and
+//               optional fp32 O, lse).
 // Every wait is bounded (see WaitCtx); on a timeout the CTA drains its
-// in-flight copies and MMAs, frees TMEM and returns.  Every mbarrier is
-// waited by one role only and can never run two phases ahead of its waiter
-// (double-buffered signals use one barrier per buffer).
+// in-flight copies and MMAs, frees TMEM and returns.
 #include "attn.cuh"
 #include "sm100.cuh"
 
@@ -54,50 +38,29 @@ namespace sage {
 
 namespace {
 
-constexpr int BM = kAttnBM;        // rows per query tile
-constexpr int BN = kAttnBN;        // keys per KV tile
-constexpr int NQT = 2;             // query tiles per CTA
-constexpr int NK = 4;              // K stages
-constexpr int NV = 4;              // V stages
-constexpr int kPrefetch = 6;       // KV tiles prefetched into L2 ahead of the loads
-constexpr int kThreads = 512;      // 16 warps = 4 warpgroups
-constexpr int kLaunchRegs = 128;   // registers per thread at launch (1 CTA per SM)
-constexpr int kRegsRoles = 56;     // WG0
-constexpr int kRegsSoftmax = 184;  // WG1, WG2
-constexpr int kRegsCorr = 80;      // WG3
-static_assert(128 * kRegsRoles + 256 * kRegsSoftmax + 128 * kRegsCorr <= kThreads * kLaunchRegs,
-              "register shares must fit in the launch allocation");
-constexpr int kTmemCols = 512;
+constexpr int BM = kAttnBM;
+constexpr int BN = kAttnBN;
+constexpr int NS = 2;              // K/V pipeline stages
+constexpr int kThreads = 192;      // 6 warps
+constexpr int kTmemCols = 256;
 constexpr uint32_t kFull = 0xffffffffu;
-// Seed of the S accumulator: the int32 bit pattern of 1.5 * 2^23.  For
-// |S| < 2^22 the word 0x4B400000 + S is the fp32 value 12582912 + S.
-constexpr uint32_t kBiasBits = 0x4B400000u;
-constexpr float kBias = 12582912.0f;
 
 // wait-site codes for the status word (kernel 1 = attention)
 enum : int {
   kSiteProdKEmpty = 0x10101, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaSFree,
-  kSiteMmaV, kSiteMmaP, kSiteMmaCorr, kSiteSmS, kSiteSmPFree, kSiteSmTurn, kSiteCorrAlpha,
-  kSiteCorrO, kSiteEpiO, kSiteEpiFin, kSiteDrain
+  kSiteMmaV, kSiteMmaP, kSiteSmS, kSiteSmO, kSiteSmEpi, kSiteDrain
 };
 
 template <int D>
 struct alignas(1024) Smem {
-  uint8_t q[NQT][BM * D];        // int8 Q tiles [128 rows][D]
-  uint8_t k[NK][BN * D];         // int8 K tiles [128 keys][D]
-  uint8_t v[NV][D * BN];         // e4m3 V^T tiles [D][128 keys]
-  uint8_t p[NQT][BM * BN];       // e4m3 P tiles [128 rows][128 keys], 128-byte swizzle
-  float alpha[NQT][2][BM];       // rescale factor per row and tile parity
-  float fin_m[NQT][BM];          // final running max per row
-  float fin_l[NQT][BM];          // final row sum (units of 2^8 p)
+  uint8_t q[BM * D];         // int8 Q tile [128 rows][D]
+  uint8_t k[NS][BN * D];     // int8 K tiles [128 keys][D]
+  uint8_t v[NS][D * BN];     // e4m3 V^T tiles [D][128 keys]
+  uint8_t p[BM * BN];        // e4m3 P tile [128 rows][128 keys], 128-byte swizzle
   uint64_t q_full;
-  uint64_t k_full[NK], k_empty[NK];
-  uint64_t v_full[NV], v_empty[NV];
-  uint64_t s_full[NQT], s_free[NQT];
-  uint64_t p_full[NQT], p_free[NQT];
-  uint64_t alpha_full[NQT][2], corr_done[NQT], o_done[NQT];
-  uint64_t turn[NQT], fin_ready[NQT];
-  uint64_t drain;
+  uint64_t k_full[NS], k_empty[NS];
+  uint64_t v_full[NS], v_empty[NS];
+  uint64_t s_full, s_free, p_full, o_ready, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -114,12 +77,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(kFull, mbar_wait(bar, parity, w, site));
 }
 
-// Warp-level arrival: the warp's prior work is ordered before lane 0 arrives.
-__device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
-  __syncwarp();
-  if (lane == 0) mbar_arrive(bar);
-}
-
 // First key index that query row i (global row) may NOT see.
 __device__ __forceinline__ int row_limit(int i, const AttnParams& p) {
   const int g = i + (p.Nkv - p.Nq);
@@ -134,7 +91,7 @@ __device__ __forceinline__ int row_limit(int i, const AttnParams& p) {
 // or TMEM under an operation in flight.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   const long long t0 = clock64();
-  while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
+  while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > w.budget) {
       record_timeout(w.status, kSiteDrain);
       return;
@@ -142,101 +99,76 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
   }
 }
 
-// ------------------------------------------------------------------ producer
-
-// K producer (and both Q tiles) when load_k, else the V producer.
 template <int D, bool DUMP>
-__device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int bh, int q0,
-                                         int kt0, int nk, bool load_k, const WaitCtx& w) {
-  constexpr int nqt = DUMP ? 1 : NQT;
-  int issued = 0;
-  if (load_k) {
-    tma_prefetch_desc(&maps.q);
-    tma_prefetch_desc(&maps.k);
-    mbar_arrive_expect_tx(&s.q_full, nqt * BM * D);
-    for (int x = 0; x < nqt; x++) tma_load_3d(s.q[x], &maps.q, &s.q_full, 0, q0 + x * BM, bh);
-    if (!DUMP)
-      for (int it = 0; it < kPrefetch && it < nk; it++)
-        tma_prefetch_l2_3d(&maps.k, 0, (kt0 + it) * BN, bh);
-    for (int it = 0; it < nk; it++) {
-      const int kt = kt0 + it, st = it % NK;
-      if (!DUMP && it + kPrefetch < nk) tma_prefetch_l2_3d(&maps.k, 0, (kt + kPrefetch) * BN, bh);
-      if (it >= NK && !mbar_wait(&s.k_empty[st], ((it / NK) & 1) ^ 1, w, kSiteProdKEmpty)) break;
-      mbar_arrive_expect_tx(&s.k_full[st], BN * D);
-      tma_load_3d(s.k[st], &maps.k, &s.k_full[st], 0, kt * BN, bh);
-      issued++;
-    }
-  } else {
-    tma_prefetch_desc(&maps.v);
-    for (int it = 0; it < kPrefetch && it < nk; it++)
-      tma_prefetch_l2_3d(&maps.v, (kt0 + it) * BN, 0, bh);
-    for (int it = 0; it < nk; it++) {
-      const int kt = kt0 + it, st = it % NV;
-      if (it + kPrefetch < nk) tma_prefetch_l2_3d(&maps.v, (kt + kPrefetch) * BN, 0, bh);
-      if (it >= NV && !mbar_wait(&s.v_empty[st], ((it / NV) & 1) ^ 1, w, kSiteProdVEmpty)) break;
-      mbar_arrive_expect_tx(&s.v_full[st], D * BN);
-      tma_load_3d(s.v[st], &maps.v, &s.v_full[st], kt * BN, 0, bh);
-      issued++;
-    }
+__device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int bh, int qt,
+                                         int kt0, int nk, const WaitCtx& w) {
+  tma_prefetch_desc(&maps.q);
+  tma_prefetch_desc(&maps.k);
+  tma_prefetch_desc(&maps.v);
+  mbar_arrive_expect_tx(&s.q_full, BM * D);
+  tma_load_3d(s.q, &maps.q, &s.q_full, 0, qt * BM, bh);
+  int k_issued = 0, v_issued = 0;
+  for (int it = 0; it < nk; it++) {
+    const int st = it % NS;
+    const uint32_t ph = (it / NS) & 1;
+    const int kt = kt0 + it;
+    if (it >= NS && !mbar_wait(&s.k_empty[st], ph ^ 1, w, kSiteProdKEmpty)) break;
+    mbar_arrive_expect_tx(&s.k_full[st], BN * D);
+    tma_load_3d(s.k[st], &maps.k, &s.k_full[st], 0, kt * BN, bh);
+    k_issued++;
+    if (DUMP) continue;
+    if (it >= NS && !mbar_wait(&s.v_empty[st], ph ^ 1, w, kSiteProdVEmpty)) break;
+    mbar_arrive_expect_tx(&s.v_full[st], D * BN);
+    tma_load_3d(s.v[st], &maps.v, &s.v_full[st], kt * BN, 0, bh);
+    v_issued++;
   }
   // Drain: every issued load must have landed before the CTA may exit.  A
   // load is only issued once the previous load of its stage was consumed, so
-  // only the last NK (NV) loads can still be in flight.
-  const int ns = load_k ? NK : NV;
-  if (load_k) drain_wait(&s.q_full, 0, w);
-  for (int it = (issued > ns ? issued - ns : 0); it < issued; it++)
-    drain_wait(load_k ? &s.k_full[it % NK] : &s.v_full[it % NV], (it / ns) & 1, w);
+  // only the last NS loads of each kind can still be in flight.
+  drain_wait(&s.q_full, 0, w);
+  for (int it = (k_issued > NS ? k_issued - NS : 0); it < k_issued; it++)
+    drain_wait(&s.k_full[it % NS], (it / NS) & 1, w);
+  for (int it = (v_issued > NS ? v_issued - NS : 0); it < v_issued; it++)
+    drain_wait(&s.v_full[it % NS], (it / NS) & 1, w);
 }
 
-// ------------------------------------------------------------------ MMA issuer
-
 template <int D, bool DUMP>
-__device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem, int nk, const WaitCtx& w) {
+__device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t tmem_O, int nk,
+                                           const WaitCtx& w) {
   constexpr uint32_t idesc_qk = idesc_i8_s32(BM, BN);
   constexpr uint32_t idesc_pv = idesc_e4m3_f32(BM, D);
-  constexpr int nqt = DUMP ? 1 : NQT;
+  const uint32_t q_addr = smem_u32(s.q);
+  const uint32_t p_addr = smem_u32(s.p);
   bool ok = mbar_wait(&s.q_full, 0, w, kSiteMmaQ);
   for (int it = 0; ok && it <= nk; it++) {
-    if (it < nk) {  // S_X = Q_X K^T for tile it
-      const int st = it % NK;
-      if (!mbar_wait(&s.k_full[st], (it / NK) & 1, w, kSiteMmaK)) break;
+    if (it < nk) {  // S = Q K^T for tile it
+      const int st = it % NS;
+      const uint32_t ph = (it / NS) & 1;
+      if (!mbar_wait(&s.k_full[st], ph, w, kSiteMmaK)) break;
+      if (it > 0 && !mbar_wait(&s.s_free, (it - 1) & 1, w, kSiteMmaSFree)) break;
+      tc_fence_after();
       const uint32_t k_addr = smem_u32(s.k[st]);
-      for (int x = 0; x < nqt; x++) {
-        // softmax X has read S_X of the previous tile and re-seeded it
-        if (!mbar_wait(&s.s_free[x], it & 1, w, kSiteMmaSFree)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(s.q[x]);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; kk++)
-          mma_i8_ss(tmem + x * BN, smem_desc_kmajor(q_addr + kk * 32, D),
-                    smem_desc_kmajor(k_addr + kk * 32, D), idesc_qk, 1u);
-        mma_commit(&s.s_full[x]);
-      }
-      if (!ok) break;
+      for (int kk = 0; kk < D / 32; kk++)
+        mma_i8_ss(tmem_S, smem_desc_kmajor(q_addr + kk * 32, D),
+                  smem_desc_kmajor(k_addr + kk * 32, D), idesc_qk, kk > 0);
       mma_commit(&s.k_empty[st]);
+      mma_commit(&s.s_full);
     }
-    if (!DUMP && it > 0) {  // O_X (+)= P_X V^T for tile it - 1
+    if (!DUMP && it > 0) {  // O (+)= P V^T for tile it - 1
       const int j = it - 1;
-      const int stv = j % NV;
-      if (!mbar_wait(&s.v_full[stv], (j / NV) & 1, w, kSiteMmaV)) break;
-      const uint32_t v_addr = smem_u32(s.v[stv]);
-      for (int x = 0; x < NQT; x++) {
-        if (!mbar_wait(&s.p_full[x], j & 1, w, kSiteMmaP) ||
-            !mbar_wait(&s.corr_done[x], j & 1, w, kSiteMmaCorr)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t p_addr = smem_u32(s.p[x]);
+      const int st = j % NS;
+      const uint32_t ph = (j / NS) & 1;
+      if (!mbar_wait(&s.v_full[st], ph, w, kSiteMmaV)) break;
+      if (!mbar_wait(&s.p_full, j & 1, w, kSiteMmaP)) break;
+      tc_fence_after();
+      const uint32_t v_addr = smem_u32(s.v[st]);
 #pragma unroll
-        for (int kk = 0; kk < BN / 32; kk++)
-          mma_f8_ss(tmem + 2 * BN + x * BN, smem_desc_kmajor(p_addr + kk * 32, BN),
-                    smem_desc_kmajor(v_addr + kk * 32, BN), idesc_pv, (j > 0 || kk > 0));
-        mma_commit(&s.p_free[x]);
-        mma_commit(&s.o_done[x]);
-      }
-      if (!ok) break;
-      mma_commit(&s.v_empty[stv]);
+      for (int kk = 0; kk < BN / 32; kk++)
+        mma_f8_ss(tmem_O, smem_desc_kmajor(p_addr + kk * 32, BN),
+                  smem_desc_kmajor(v_addr + kk * 32, BN), idesc_pv, (j > 0 || kk > 0));
+      mma_commit(&s.v_empty[st]);
+      mma_commit(&s.o_ready);
     }
   }
   // Drain: all MMAs issued by this thread complete before TMEM is freed.
@@ -244,295 +176,191 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem, int nk, co
   drain_wait(&s.drain, 0, w);
 }
 
-// ------------------------------------------------------------------ softmax
-
-// Seed the warp's 32 rows of the S columns with kBiasBits (asynchronous
-// TMEM store; see release_scores).
-__device__ __forceinline__ void seed_scores(uint32_t tS) { tmem_fill128_nowait(tS, kBiasBits); }
-
-// Wait for the seed to land and tell the MMA issuer that S may be written.
-__device__ __forceinline__ void release_scores(uint64_t* s_free, int lane) {
-  tmem_wait_st();
-  tc_fence_before();
-  warp_arrive(s_free, lane);
-}
-
-// Max of 32 biased scores (all > 0), 3-input maxima in two chains.
-__device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
-  float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
-  float b = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
-#pragma unroll
-  for (int j = 6; j < 30; j += 4) {
-    a = fmax3(a, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-    b = fmax3(b, __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-  }
-  return fmax3(a, b, fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31])));
-}
-
-// Keys at or past `nvis` (masked) read as 0, below every seeded score.
-__device__ __forceinline__ void mask_chunk(uint32_t (&v)[32], int j0, int nvis) {
-#pragma unroll
-  for (int e = 0; e < 32; e++) v[e] = (j0 + e < nvis) ? v[e] : 0u;
-}
-
-// Online softmax of query tile X (0 = A, 1 = B), one row per thread.  The
-// score row is read from TMEM in 32-column chunks (double-buffered), once
-// for the maximum and once for the exponentials, so that few registers are
-// live at any time.
+// Softmax / correction / epilogue for one query row per thread.
 template <int D>
-__device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem,
-                                             int X, int bh, int q0, int nk, const WaitCtx& w) {
+__device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
+                                             uint32_t tmem_O, int bh, int qt, int nk,
+                                             const WaitCtx& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;               // TMEM lane quadrant of this warp
   const int r = quad * 32 + lane;          // row within the tile
-  const int i = q0 + X * BM + r;           // query row
+  const int i = qt * BM + r;               // query row
   const bool valid = i < p.Nq;
-  const uint32_t tS = tmem + (static_cast<uint32_t>(quad * 32) << 16) + X * BN;
+  const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+  const uint32_t tS = tmem_S + lane_off, tO = tmem_O + lane_off;
   const int lim = valid ? row_limit(i, p) : 0;
   const float sqC = valid ? __fmul_rn(__ldg(p.q_scale + static_cast<size_t>(bh) * p.nq_blocks + i / 64), p.c0)
                           : 0.0f;
   const float* ksc = p.k_scale + static_cast<size_t>(bh) * p.nkv_blocks;
+  uint8_t* prow = s.p + r * BN;
 
-  seed_scores(tS);  // S seed for the first tile
-  release_scores(&s.s_free[X], lane);
-  if (X == 1) warp_arrive(&s.turn[0], lane);  // tile A takes the first turn
-
-  // K scales of a tile's two 64-key groups, loaded one tile ahead (blocks
-  // past the end read as 0)
-  float sk0 = __ldg(ksc), sk1 = p.nkv_blocks > 1 ? __ldg(ksc + 1) : 0.0f;
   float m = -INFINITY, l = 0.0f;
+  bool ok = true;
   for (int it = 0; it < nk; it++) {
     const int j0 = it * BN;
-    const int pb = it & 1;
-    const float c0 = __fmul_rn(sqC, sk0), c1 = __fmul_rn(sqC, sk1);
-    {
-      const int g0 = 2 * it + 2, g1 = 2 * it + 3;
-      sk0 = g0 < p.nkv_blocks ? __ldg(ksc + g0) : 0.0f;
-      sk1 = g1 < p.nkv_blocks ? __ldg(ksc + g1) : 0.0f;
-    }
-    if (!warp_wait(&s.s_full[X], it & 1, w, kSiteSmS)) return;
+    if (!warp_wait(&s.s_full, it & 1, w, kSiteSmS)) { ok = false; break; }
     tc_fence_after();
+    uint32_t sv[128];
+    {
+      uint32_t (&h0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&sv[0]);
+      uint32_t (&h1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&sv[64]);
+      tmem_ld64(tS, h0);
+      tmem_ld64(tS + 64, h1);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.s_free);
+
+    // scale of each 64-key group of the tile (blocks past the end read as 0)
+    const int g0 = 2 * it, g1 = 2 * it + 1;
+    const float c0 = __fmul_rn(sqC, g0 < p.nkv_blocks ? __ldg(ksc + g0) : 0.0f);
+    const float c1 = __fmul_rn(sqC, g1 < p.nkv_blocks ? __ldg(ksc + g1) : 0.0f);
     const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
     const bool full = __all_sync(kFull, nvis == BN);
 
-    // ---- maximum per 64-key scale group (biased scores; 0 = all masked)
-    float mb[2];
-    {
-      uint32_t b0[32], b1[32];
-      tmem_ld32_async(tS, b0);
+    // masked max per group in the integer domain: for c >= 0,
+    // max_j fp32(S_j * c) = fp32(max_j S_j * c)
+    int mx0 = INT_MIN, mx1 = INT_MIN;
+    if (full) {
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t (&cur)[32] = (c & 1) ? b1 : b0;
-        uint32_t (&nxt)[32] = (c & 1) ? b0 : b1;
-        tmem_wait_ld(cur);
-        if (c < 3) tmem_ld32_async(tS + 32 * (c + 1), nxt);
-        if (!full) mask_chunk(cur, 32 * c, nvis);
-        const float cm = max32(cur);
-        if (c & 1) mb[c >> 1] = fmaxf(mb[c >> 1], cm);
-        else mb[c >> 1] = cm;
-      }
+      for (int j = 0; j < 64; j++) mx0 = max(mx0, static_cast<int>(sv[j]));
+#pragma unroll
+      for (int j = 64; j < 128; j++) mx1 = max(mx1, static_cast<int>(sv[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 64; j++) if (j < nvis) mx0 = max(mx0, static_cast<int>(sv[j]));
+#pragma unroll
+      for (int j = 64; j < 128; j++) if (j < nvis) mx1 = max(mx1, static_cast<int>(sv[j]));
     }
-    // max_j fp32(S_j * c) = fp32(max_j S_j * c) for c >= 0 (rounding is monotone)
-    const float t0 = mb[0] > 0.0f ? __fmul_rn(__fsub_rn(mb[0], kBias), c0) : -INFINITY;
-    const float t1 = mb[1] > 0.0f ? __fmul_rn(__fsub_rn(mb[1], kBias), c1) : -INFINITY;
-    const float m_new = fmax3(m, t0, t1);
+    const float t0 = mx0 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mx0), c0);
+    const float t1 = mx1 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mx1), c1);
+    const float m_new = fmaxf(m, fmaxf(t0, t1));
     const float alpha = (m == -INFINITY) ? 0.0f
                         : (m == m_new)   ? 1.0f
                                          : ex2_approx(__fsub_rn(m, m_new));
     const float nm8 = __fsub_rn(8.0f, m_new);  // P scale 2^8 folded into the exponent
-    s.alpha[X][pb][r] = alpha;
-    warp_arrive(&s.alpha_full[X][pb], lane);
 
-    // the P tile is free once P V of the previous tile has read it; then
-    // wait for this warpgroup's turn at the exp2 phase
-    if (it >= 1 && !warp_wait(&s.p_free[X], (it - 1) & 1, w, kSiteSmPFree)) return;
-    if (!warp_wait(&s.turn[X], it & 1, w, kSiteSmTurn)) return;
+    // the P tile is free once P V of the previous tile has completed
+    if (it > 0 && !warp_wait(&s.o_ready, (it - 1) & 1, w, kSiteSmO)) { ok = false; break; }
+    tc_fence_after();
 
-    // ---- y = 2^(S c + 8 - m), row sum, e4m3 codes into the swizzled P tile
-    uint8_t* prow = s.p[X] + r * BN;
-    const float2 nb2 = make_float2(-kBias, -kBias);
-    const float2 nm2 = make_float2(nm8, nm8);
     float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-    {
-      uint32_t b0[32], b1[32];
-      tmem_ld32_async(tS, b0);
+    const float2 nm2 = make_float2(nm8, nm8);
+    const float2 nb2 = make_float2(-12582912.0f, -12582912.0f);
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t (&cur)[32] = (c & 1) ? b1 : b0;
-        uint32_t (&nxt)[32] = (c & 1) ? b0 : b1;
-        tmem_wait_ld(cur);
-        if (c < 3) tmem_ld32_async(tS + 32 * (c + 1), nxt);
-        const float2 cc = c < 2 ? make_float2(c0, c0) : make_float2(c1, c1);
-        float y[32];
+    for (int c = 0; c < 8; c++) {  // 16-key chunks
+      uint32_t pk[4];
+      const float2 cc = c < 4 ? make_float2(c0, c0) : make_float2(c1, c1);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 x = __ffma2_rn(
-              __fadd2_rn(make_float2(__uint_as_float(cur[e]), __uint_as_float(cur[e + 1])), nb2), cc, nm2);
-          y[e] = x.x;
-          y[e + 1] = x.y;
+      for (int q4 = 0; q4 < 4; q4++) {
+        const int j = c * 16 + q4 * 4;
+        float y[4];
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          const float2 sf = __fadd2_rn(make_float2(__uint_as_float(sv[j + e] + 0x4B400000u),
+                                                   __uint_as_float(sv[j + e + 1] + 0x4B400000u)), nb2);
+          const float2 x = __ffma2_rn(sf, cc, nm2);
+          y[e] = x.x; y[e + 1] = x.y;
         }
         if (!full) {
 #pragma unroll
-          for (int e = 0; e < 32; e++) y[e] = (32 * c + e < nvis) ? y[e] : -INFINITY;
+          for (int e = 0; e < 4; e++) y[e] = (j + e < nvis) ? y[e] : -INFINITY;
         }
 #pragma unroll
-        for (int e = 0; e < 32; e++) y[e] = ex2_approx(y[e]);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          acc[0] = __fadd2_rn(acc[0], make_float2(y[e], y[e + 1]));
-          acc[1] = __fadd2_rn(acc[1], make_float2(y[e + 2], y[e + 3]));
-        }
-#pragma unroll
-        for (int h = 0; h < 2; h++) {  // two 16-key chunks of the P row
-          uint32_t pk[4];
-#pragma unroll
-          for (int q4 = 0; q4 < 4; q4++) {
-            const int e = h * 16 + q4 * 4;
-            pk[q4] = __byte_perm(cvt_e4m3x2(y[e], y[e + 1]), cvt_e4m3x2(y[e + 2], y[e + 3]), 0x5410);
-          }
-          const int chunk = 2 * c + h;
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
+        for (int e = 0; e < 4; e++) y[e] = ex2_approx(y[e]);
+        acc[q4 & 1] = __fadd2_rn(acc[q4 & 1], make_float2(y[0], y[1]));
+        acc[q4 & 1] = __fadd2_rn(acc[q4 & 1], make_float2(y[2], y[3]));
+        pk[q4] = __byte_perm(cvt_e4m3x2(y[0], y[1]), cvt_e4m3x2(y[2], y[3]), 0x5410);
       }
-    }
-    seed_scores(tS);  // S seed for the next tile
-    fence_proxy_async_smem();
-    release_scores(&s.s_free[X], lane);
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&s.turn[X ^ 1]);   // the other warpgroup's turn
-      mbar_arrive(&s.p_full[X]);
+      *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
     const float2 a2 = __fadd2_rn(acc[0], acc[1]);
-    l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(a2.x, a2.y));
+    const float rs = __fadd_rn(a2.x, a2.y);
+    fence_proxy_async_smem();
+
+    // rescale the O row when the running max moved (never before the first P V)
+    if (it > 0 && __any_sync(kFull, alpha != 1.0f)) {
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+#pragma unroll
+        for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), alpha));
+        tmem_st32(tO + c, o);
+      }
+    }
+    l = __fadd_rn(__fmul_rn(l, alpha), rs);
     m = m_new;
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.p_full);
   }
-  s.fin_m[X][r] = m;
-  s.fin_l[X][r] = l;
-  warp_arrive(&s.fin_ready[X], lane);
-}
 
-// ------------------------------------------------------------------ correction + epilogue
-
-template <int D>
-__device__ __forceinline__ void rescale_row(uint32_t tO, float alpha) {
-  // 32-column pieces keep the register footprint small
+  if (!ok || nk == 0) return;
+  if (!warp_wait(&s.o_ready, (nk - 1) & 1, w, kSiteSmEpi)) return;
+  tc_fence_after();
+  const float inv = __frcp_rn(l);  // l is in units of 2^8 p
+  const float* vsc = p.v_scale + static_cast<size_t>(bh) * D;
+  const size_t orow = (static_cast<size_t>(bh) * p.Nq + (valid ? i : 0)) * D;
 #pragma unroll 1
   for (int c = 0; c < D; c += 32) {
     uint32_t o[32];
     tmem_ld32(tO + c, o);
+    if (!valid) continue;
+    float f[32];
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
-                                  make_float2(alpha, alpha));
-      o[e] = __float_as_uint(v.x);
-      o[e + 1] = __float_as_uint(v.y);
+    for (int e = 0; e < 32; e++) f[e] = __uint_as_float(o[e]) * (__ldg(vsc + c + e) * inv);
+    uint32_t b[16];
+#pragma unroll
+    for (int e = 0; e < 16; e++) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+      b[e] = *reinterpret_cast<uint32_t*>(&h);
     }
-    tmem_st32(tO + c, o);
+    uint4* dst = reinterpret_cast<uint4*>(p.o + orow + c);
+#pragma unroll
+    for (int e = 0; e < 4; e++) dst[e] = make_uint4(b[4 * e], b[4 * e + 1], b[4 * e + 2], b[4 * e + 3]);
+    if (p.o_f32) {
+      float4* d32 = reinterpret_cast<float4*>(p.o_f32 + orow + c);
+#pragma unroll
+      for (int e = 0; e < 8; e++) d32[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+    }
   }
+  if (valid && p.lse)
+    p.lse[static_cast<size_t>(bh) * p.Nq + i] = (m + log2f(l) - 8.0f) * 0.69314718055994531f;
 }
 
+// Score dump (debug): copy the int32 S tile from TMEM to global memory.
 template <int D>
-__device__ __forceinline__ void correction_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem,
-                                                int bh, int q0, int nk, const WaitCtx& w) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int quad = warp & 3;
-  const int r = quad * 32 + lane;
-  const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-  for (int it = 0; it < nk; it++) {
-    const int pb = it & 1;
-    for (int x = 0; x < NQT; x++) {
-      if (!warp_wait(&s.alpha_full[x][pb], (it >> 1) & 1, w, kSiteCorrAlpha)) return;
-      const float alpha = s.alpha[x][pb][r];
-      if (it > 0) {
-        // P V of the previous tile must have completed before O is rescaled
-        if (!warp_wait(&s.o_done[x], (it - 1) & 1, w, kSiteCorrO)) return;
-        tc_fence_after();
-        if (__any_sync(kFull, alpha != 1.0f))
-          rescale_row<D>(tmem + lane_off + 2 * BN + x * BN, alpha);
-      }
-      tc_fence_before();
-      warp_arrive(&s.corr_done[x], lane);
-    }
-  }
-  // epilogue: O_X * v_scale / l -> bf16 (and fp32 O, lse)
-  const float* vsc = p.v_scale + static_cast<size_t>(bh) * D;
-  for (int x = 0; x < NQT; x++) {
-    if (!warp_wait(&s.o_done[x], (nk - 1) & 1, w, kSiteEpiO)) return;
-    if (!warp_wait(&s.fin_ready[x], 0, w, kSiteEpiFin)) return;
-    tc_fence_after();
-    const int i = q0 + x * BM + r;
-    const bool valid = i < p.Nq;
-    const float l = s.fin_l[x][r], m = s.fin_m[x][r];
-    const float inv = __frcp_rn(l);  // l is in units of 2^8 p
-    const size_t orow = (static_cast<size_t>(bh) * p.Nq + (valid ? i : 0)) * D;
-    const uint32_t tO = tmem + lane_off + 2 * BN + x * BN;
-#pragma unroll 1
-    for (int c = 0; c < D; c += 32) {
-      uint32_t o[32];
-      tmem_ld32(tO + c, o);
-      if (!valid) continue;
-#pragma unroll
-      for (int e = 0; e < 32; e++)
-        o[e] = __float_as_uint(__uint_as_float(o[e]) * (__ldg(vsc + c + e) * inv));
-      if (p.o_f32) {
-        float4* d32 = reinterpret_cast<float4*>(p.o_f32 + orow + c);
-#pragma unroll
-        for (int e = 0; e < 8; e++)
-          d32[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                               __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
-      }
-#pragma unroll
-      for (int e = 0; e < 16; e++) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1]));
-        o[e] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      uint4* dst = reinterpret_cast<uint4*>(p.o + orow + c);
-#pragma unroll
-      for (int e = 0; e < 4; e++) dst[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-    }
-    if (valid && p.lse)
-      p.lse[static_cast<size_t>(bh) * p.Nq + i] = (m + log2f(l) - 8.0f) * 0.69314718055994531f;
-  }
-}
-
-// Score dump (debug): copy the int32 S tile of query tile A from TMEM to
-// global memory (the accumulator seed removed).
-template <int D>
-__device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem,
+__device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
                                           const WaitCtx& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
-  const uint32_t tS = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-  seed_scores(tS);
-  release_scores(&s.s_free[0], lane);
-  if (!warp_wait(&s.s_full[0], 0, w, kSiteSmS)) return;
+  if (!warp_wait(&s.s_full, 0, w, kSiteSmS)) return;
   tc_fence_after();
+  const uint32_t tS = tmem_S + (static_cast<uint32_t>(quad * 32) << 16);
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     uint32_t v[32];
     tmem_ld32(tS + c, v);
-#pragma unroll
-    for (int e = 0; e < 32; e++) v[e] -= kBiasBits;
     uint4* dst = reinterpret_cast<uint4*>(p.dbg_out + static_cast<size_t>(r) * BN + c);
 #pragma unroll
     for (int e = 0; e < 8; e++) dst[e] = make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
   }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&s.s_free);
 }
 
-// ------------------------------------------------------------------ kernel
-
 template <int D, bool DUMP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& s = *reinterpret_cast<Smem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = DUMP ? p.dbg_qt : static_cast<int>(blockIdx.x);
   const int bh = DUMP ? p.dbg_bh : static_cast<int>(blockIdx.y);
-  // first query row of the CTA (DUMP: the requested 128-row tile)
-  const int q0 = DUMP ? p.dbg_qt * BM : static_cast<int>(blockIdx.x) * NQT * BM;
 
   // KV tiles this CTA visits: those holding a key visible to its last valid
   // row (the masks' limits grow with the row index).
@@ -541,31 +369,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     kt0 = p.dbg_kt;
     nk = 1;
   } else {
-    const int last = min(p.Nq - 1, q0 + NQT * BM - 1);
+    const int last = min(p.Nq - 1, qt * BM + BM - 1);
     nk = (row_limit(last, p) + BN - 1) / BN;
   }
 
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
-    for (int i = 0; i < NK; i++) {
+    for (int i = 0; i < NS; i++) {
       mbar_init(&s.k_full[i], 1);
       mbar_init(&s.k_empty[i], 1);
-    }
-    for (int i = 0; i < NV; i++) {
       mbar_init(&s.v_full[i], 1);
       mbar_init(&s.v_empty[i], 1);
     }
-    for (int x = 0; x < NQT; x++) {
-      mbar_init(&s.s_full[x], 1);
-      mbar_init(&s.s_free[x], 4);
-      mbar_init(&s.p_full[x], 4);
-      mbar_init(&s.p_free[x], 1);
-      for (int b = 0; b < 2; b++) mbar_init(&s.alpha_full[x][b], 4);
-      mbar_init(&s.corr_done[x], 4);
-      mbar_init(&s.o_done[x], 1);
-      mbar_init(&s.turn[x], 4);
-      mbar_init(&s.fin_ready[x], 4);
-    }
+    mbar_init(&s.s_full, 1);
+    mbar_init(&s.s_free, 4);
+    mbar_init(&s.p_full, 4);
+    mbar_init(&s.o_ready, 1);
     mbar_init(&s.drain, 1);
     s.abort = 0;
     fence_mbar_init();
@@ -577,29 +396,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = s.tmem_base;  // S_A, S_B at columns 0, 128; O_A, O_B at 256, 384
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t tmem_S = tmem;        // columns [0, 128): int32 scores
+  const uint32_t tmem_O = tmem + 128;  // columns [128, 128 + D): fp32 output
   const WaitCtx w{p.budget, p.status, &s.abort};
 
-  const int wg = warp >> 2;
-  if (wg == 0) {
-    regs_dec<kRegsRoles>();
-    if (warp == 0) {
-      if (lane == 0) producer<D, DUMP>(s, maps, bh, q0, kt0, nk, true, w);
-    } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, DUMP>(s, tmem, nk, w);
-    } else if (warp == 2 && !DUMP) {
-      if (lane == 0) producer<D, DUMP>(s, maps, bh, q0, kt0, nk, false, w);
-    }
-  } else if (wg <= NQT) {
-    regs_inc<kRegsSoftmax>();
-    if (DUMP) {
-      if (wg == 1) dump_rows<D>(s, p, tmem, w);
-    } else {
-      softmax_rows<D>(s, p, tmem, wg - 1, bh, q0, nk, w);
-    }
+  if (warp == 0) {
+    if (lane == 0) producer<D, DUMP>(s, maps, bh, qt, kt0, nk, w);
+  } else if (warp == 1) {
+    if (lane == 0) mma_issuer<D, DUMP>(s, tmem_S, tmem_O, nk, w);
   } else {
-    regs_dec<kRegsCorr>();
-    if (!DUMP) correction_rows<D>(s, p, tmem, bh, q0, nk, w);
+    if (DUMP) dump_rows<D>(s, p, tmem_S, w);
+    else softmax_rows<D>(s, p, tmem_S, tmem_O, bh, qt, nk, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -610,22 +418,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// One-time per-device setup: dynamic shared memory size, and a check that
-// the compiled kernels were built with exactly kLaunchRegs registers per
-// thread.  The warpgroups' setmaxnreg shares add up to that launch
-// allocation; a different allocation could leave an increase waiting, so
-// such a build is refused here instead of launched.
-template <int D, bool DUMP>
-cudaError_t prepare_one() {
-  cudaError_t e = cudaFuncSetAttribute(k_attn<D, DUMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem_bytes_for(D)));
-  if (e != cudaSuccess) return e;
-  cudaFuncAttributes attr;
-  e = cudaFuncGetAttributes(&attr, k_attn<D, DUMP>);
-  if (e != cudaSuccess) return e;
-  return attr.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidDeviceFunction;
-}
-
 }  // namespace
 
 size_t attn_smem_bytes(int D) { return smem_bytes_for(D); }
@@ -633,17 +425,23 @@ size_t attn_smem_bytes(int D) { return smem_bytes_for(D); }
 cudaError_t attn_prepare(int D) {
   cudaError_t e;
   if (D == 128) {
-    e = prepare_one<128, false>();
-    if (e == cudaSuccess) e = prepare_one<128, true>();
+    e = cudaFuncSetAttribute(k_attn<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for(128)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_attn<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes_for(128)));
   } else {
-    e = prepare_one<64, false>();
-    if (e == cudaSuccess) e = prepare_one<64, true>();
+    e = cudaFuncSetAttribute(k_attn<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for(64)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_attn<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_bytes_for(64)));
   }
   return e;
 }
 
 cudaError_t launch_attn(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
-  dim3 grid((p.Nq + NQT * BM - 1) / (NQT * BM), p.BH);
+  dim3 grid((p.Nq + BM - 1) / BM, p.BH);
   if (p.D == 128)
     k_attn<128, false><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
   else
