@@ -49,8 +49,6 @@ def lib():
         L.orc_quant_head.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P]
         L.orc_qk_int32.restype = None
         L.orc_qk_int32.argtypes = [P, P, i32, i64, i64, i64, i64, P]
-        L.orc_exp2_poly.restype = ctypes.c_float
-        L.orc_exp2_poly.argtypes = [ctypes.c_float]
         L.orc_row_limit.restype = i64
         L.orc_row_limit.argtypes = [i64, i64, i64, i32, i64]
         L.orc_attn_rows.restype = i32
@@ -132,15 +130,6 @@ def qk_int32(q8, k8, i0, ni, j0, nj):
     out = np.empty((ni, nj), np.int32)
     lib().orc_qk_int32(_p(q8), _p(k8), q8.shape[1], i0, ni, j0, nj, _p(out))
     return out
-
-
-POLY_FROM = 12   # keys with index mod 16 >= POLY_FROM use the software exp2
-
-
-def exp2_poly(x):
-    L = lib()
-    return np.array([L.orc_exp2_poly(float(v)) for v in np.asarray(x, np.float32).ravel()],
-                    np.float32).reshape(np.shape(x))
 
 
 def row_limit(i, nq, nkv, mask, mb):

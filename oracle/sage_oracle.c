@@ -309,37 +309,6 @@ typedef struct {
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
 
-/* Software base-2 exponential used for a fixed share of the keys (those
- * with key index mod 16 >= 12): Cody-Waite range reduction x = n + f with
- * n = round(x) obtained by adding and subtracting 1.5 * 2^23, f = x - n in
- * [-1/2, 1/2], a degree-3 polynomial for 2^f (coefficients fitted here for
- * minimum maximum relative error with the constant term fixed to 1; maximum
- * relative error 1.02e-4), and n added to the exponent field.  Arguments are
- * clamped at -125 so that the exponent never underflows (2^-125 is far below
- * the smallest nonzero e4m3 code of P). */
-#define ORC_EXP2_C1 0x1.62f5f8p-1f
-#define ORC_EXP2_C2 0x1.f00bb8p-3f
-#define ORC_EXP2_C3 0x1.c2a0e8p-5f
-
-float orc_exp2_poly(float x)
-{
-    float xc = x > -125.0f ? x : -125.0f;
-    float j = xc + 12582912.0f;
-    float n = j - 12582912.0f;
-    float f = xc - n;
-    float p = fmaf(fmaf(fmaf(ORC_EXP2_C3, f, ORC_EXP2_C2), f, ORC_EXP2_C1), f, 1.0f);
-    uint32_t pb, jb, yb;
-    float y;
-    memcpy(&pb, &p, sizeof pb);
-    memcpy(&jb, &j, sizeof jb);
-    yb = pb + (jb << 23);
-    memcpy(&y, &yb, sizeof y);
-    return y;
-}
-
-/* Keys whose index mod 16 is at least this use orc_exp2_poly. */
-#define ORC_POLY_FROM 12
-
 /* Width, in units of y = p*2^8, of the set of e4m3 codes that y*(1 +- eps)
  * can round to; zero when the uncertainty interval does not straddle a
  * rounding boundary. */
@@ -368,9 +337,7 @@ static double e4m3_flip_gap(double y, double eps)
  *   S_ij  = sum_d q8 k8 (exact integer)
  *   t_ij  = fp32(fp32(S_ij) * c_ij)             (for the max)
  *   P is quantized with the fixed scale 2^8, folded into the exponent:
- *   y_ij  = exp2(fmaf(fp32(S_ij), c_ij, fp32(8 - m_k)))   (~ 256 p_ij), where
- *           exp2 is fp32(exp2) in fp64 for keys with j mod 16 < 12 (the
- *           device's hardware exp2) and orc_exp2_poly for the others
+ *   y_ij  = fp32(exp2(fmaf(fp32(S_ij), c_ij, fp32(8 - m_k))))   (~ 256 p_ij)
  *   l is accumulated in fp32 from y (before quantization),
  *   w_ij  = e4m3(y_ij), V_j = e4m3 code values,
  *   O     = O_acc * vs[d] / l;  lse = (m + log2(l) - 8) * ln 2.
@@ -453,13 +420,10 @@ static void attend_row(const attn_job *J, long r)
                     acc[d] += p * J->vd[j * D + d];
             } else {
                 float x = fmaf((float)S[jj], c[jj], nm8);
-                const int poly = (int)(j % 16) >= ORC_POLY_FROM;
-                float y = poly ? orc_exp2_poly(x) : exp2_f32(x);
+                float y = exp2_f32(x);
                 rowsum_f += y;
                 double w = orc_e4m3_decode(orc_e4m3_encode(y));
-                /* the polynomial is reproduced exactly; only the hardware
-                 * exp2 leaves a rounding uncertainty */
-                double gap = (sl && !poly) ? e4m3_flip_gap((double)y, J->eps) : 0.0;
+                double gap = sl ? e4m3_flip_gap((double)y, J->eps) : 0.0;
                 for (int d = 0; d < D; d++) {
                     double vv = orc_e4m3_decode(J->v8[j * D + d]);
                     acc[d] += w * vv;

@@ -192,35 +192,3 @@ def test_invalid_arguments_raise():
     qh = oracle.quant_head(q, k, v)
     with pytest.raises(ValueError):
         oracle.attn_rows(qh, np.arange(3), oracle.MASK_CAUSAL, 0)
-
-
-def test_software_exp2_accuracy_and_special_points():
-    # relative error bound of the fitted polynomial, exact powers of two at
-    # integers, monotone clamp below -125
-    x = np.concatenate([np.linspace(-40, 8, 200001), np.arange(-30, 9)]).astype(np.float32)
-    y = oracle.exp2_poly(x).astype(np.float64)
-    rel = np.abs(y / np.exp2(x.astype(np.float64)) - 1)
-    assert rel.max() < 1.1e-4
-    ints = np.arange(-30, 9).astype(np.float32)
-    assert np.array_equal(oracle.exp2_poly(ints), np.exp2(ints.astype(np.float64)).astype(np.float32))
-    tail = oracle.exp2_poly(np.array([-125.0, -126.0, -1e4, -np.inf], np.float32))
-    assert np.all(tail == np.float32(2.0 ** -125))
-
-
-def test_quant_recipe_splits_hardware_and_software_exp2():
-    # keys with index mod 16 >= 12 use the software exp2, which both sides
-    # compute identically: when only those keys carry nonzero values, no output
-    # can depend on a hardware-exp2 rounding, so the slack is exactly zero even
-    # for a large exp2 uncertainty; keys 0..3 (hardware exp2) do produce slack
-    nq, nkv, D = 64, 64, 64
-    q, k, v = _bits(nq, nkv, D, 16)
-    only_sw = v.copy()
-    only_sw[:12] = 0
-    only_sw[16:] = 0
-    only_hw = v.copy()
-    only_hw[4:] = 0
-    rows = np.arange(nq)
-    _, s_sw, _ = oracle.attn_rows(oracle.quant_head(q, k, only_sw), rows, eps=1e-2)
-    _, s_hw, _ = oracle.attn_rows(oracle.quant_head(q, k, only_hw), rows, eps=1e-2)
-    assert not s_sw.any()
-    assert s_hw.any()
