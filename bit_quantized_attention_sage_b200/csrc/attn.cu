@@ -12,20 +12,25 @@
 // KV tiles of 128 keys.  Warp roles (192 threads, two CTAs per SM):
 //   warp 0      TMA producer: the Q tile once, then K and V^T tiles through
 //               a two-stage shared-memory ring (128-byte swizzle).
+//               The e4m3 P tile is double-buffered: the softmax of tile k
+//               writes P(k) while P V of tile k-1 may still read P(k-1).
 //   warp 1      allocates 256 TMEM columns (S: 128 x 128 int32, O: 128 x D
 //               fp32) and one elected thread issues every tcgen05.mma:
 //               S = Q K^T (kind::i8) for tile k+1 while the softmax warps
 //               work on tile k, then O (+)= P V^T (kind::f8f6f4).
 //   warps 2-5   softmax: thread t of the warpgroup owns query row t (TMEM
-//               lane t).  Per tile: load the int32 score row from TMEM, take
-//               the masked max in the integer domain per 64-key scale group,
-//               update the running max, y = exp2(fma(S, c, 8 - m)) (P scale
-//               2^8 folded into the exponent; S converted exactly without
-//               the conversion unit as as_float(S + 0x4B400000) - 1.5*2^23)
-//               with packed fp32x2 arithmetic, row sum, e4m3(y) into the
-//               swizzled shared-memory P tile, and rescale the O row in TMEM
-//               when the max moved.  Epilogue: O * v_scale / l -> bf16 (and
-//               optional fp32 O, lse).
+//               lane t).  The S accumulator columns are seeded with the bit
+//               pattern 0x4B400000 before each Q K^T, so the int32 result
+//               0x4B400000 + S reads as the fp32 value 1.5*2^23 + S exactly
+//               (no conversion unit, no integer add).  Per tile: load the
+//               score row from TMEM and re-seed it, take the masked max per
+//               64-key scale group with a tree of 3-input maxima, update the
+//               running max, y = exp2(fma(S, c, 8 - m)) (P scale 2^8 folded
+//               into the exponent) with packed fp32x2 arithmetic, row sum,
+//               e4m3(y) into the swizzled shared-memory P buffer of the
+//               tile's parity, then (once P V of the previous tile has
+//               completed) rescale the O row in TMEM when the max moved.
+//               Epilogue: O * v_scale / l -> bf16 (and optional fp32 O, lse).
 // Every wait is bounded (see WaitCtx); on a timeout the CTA drains its
 // in-flight copies and MMAs, frees TMEM and returns.
 #include "attn.cuh"
@@ -44,11 +49,16 @@ constexpr int NS = 2;              // K/V pipeline stages
 constexpr int kThreads = 192;      // 6 warps
 constexpr int kTmemCols = 256;
 constexpr uint32_t kFull = 0xffffffffu;
+// The S accumulator is seeded with the bit pattern of 1.5 * 2^23; for
+// |S| < 2^22 the int32 sum 0x4B400000 + S reads as the fp32 value
+// 1.5 * 2^23 + S exactly (|S| <= 128 * 128 * D < 2^22 for D <= 128).
+constexpr uint32_t kBiasBits = 0x4B400000u;
+constexpr float kBias = 12582912.0f;
 
 // wait-site codes for the status word (kernel 1 = attention)
 enum : int {
   kSiteProdKEmpty = 0x10101, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaSFree,
-  kSiteMmaV, kSiteMmaP, kSiteSmS, kSiteSmO, kSiteSmEpi, kSiteDrain
+  kSiteMmaV, kSiteMmaP, kSiteSmS, kSiteSmO, kSiteSmEpi, kSiteDrain, kSiteSmemAlign
 };
 
 template <int D>
@@ -56,7 +66,7 @@ struct alignas(1024) Smem {
   uint8_t q[BM * D];         // int8 Q tile [128 rows][D]
   uint8_t k[NS][BN * D];     // int8 K tiles [128 keys][D]
   uint8_t v[NS][D * BN];     // e4m3 V^T tiles [D][128 keys]
-  uint8_t p[BM * BN];        // e4m3 P tile [128 rows][128 keys], 128-byte swizzle
+  uint8_t p[2][BM * BN];     // e4m3 P tiles [parity][128 rows][128 keys], 128-byte swizzle
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS];
   uint64_t v_full[NS], v_empty[NS];
@@ -65,9 +75,13 @@ struct alignas(1024) Smem {
   int abort;
 };
 
+// Exactly the struct: two D = 128 CTAs fill the SM's 228 KB (2 x (113 KB +
+// 1 KB reserved)), so there is no room for alignment slack.  The dynamic
+// shared-memory window is 1024-byte aligned (the kernel checks this).
 __host__ __device__ inline size_t smem_bytes_for(int D) {
-  return (D == 128 ? sizeof(Smem<128>) : sizeof(Smem<64>)) + 1024;  // + alignment slack
+  return D == 128 ? sizeof(Smem<128>) : sizeof(Smem<64>);
 }
+static_assert(sizeof(Smem<128>) <= 115712, "two CTAs per SM must fit in 228 KB");
 
 // A wait taken by all 32 threads of a warp that reports success only if it
 // succeeded for every lane, so that the warp never splits before the
@@ -138,20 +152,22 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t
   constexpr uint32_t idesc_qk = idesc_i8_s32(BM, BN);
   constexpr uint32_t idesc_pv = idesc_e4m3_f32(BM, D);
   const uint32_t q_addr = smem_u32(s.q);
-  const uint32_t p_addr = smem_u32(s.p);
+  const uint32_t p_addr0 = smem_u32(s.p[0]);
   bool ok = mbar_wait(&s.q_full, 0, w, kSiteMmaQ);
   for (int it = 0; ok && it <= nk; it++) {
     if (it < nk) {  // S = Q K^T for tile it
       const int st = it % NS;
       const uint32_t ph = (it / NS) & 1;
       if (!mbar_wait(&s.k_full[st], ph, w, kSiteMmaK)) break;
-      if (it > 0 && !mbar_wait(&s.s_free, (it - 1) & 1, w, kSiteMmaSFree)) break;
+      // the softmax warps have read S of the previous tile and re-seeded it
+      // (score dumps are not seeded and hold one tile only)
+      if (!DUMP && !mbar_wait(&s.s_free, it & 1, w, kSiteMmaSFree)) break;
       tc_fence_after();
       const uint32_t k_addr = smem_u32(s.k[st]);
 #pragma unroll
       for (int kk = 0; kk < D / 32; kk++)
         mma_i8_ss(tmem_S, smem_desc_kmajor(q_addr + kk * 32, D),
-                  smem_desc_kmajor(k_addr + kk * 32, D), idesc_qk, kk > 0);
+                  smem_desc_kmajor(k_addr + kk * 32, D), idesc_qk, DUMP ? kk > 0 : 1);
       mma_commit(&s.k_empty[st]);
       mma_commit(&s.s_full);
     }
@@ -163,6 +179,7 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t
       if (!mbar_wait(&s.p_full, j & 1, w, kSiteMmaP)) break;
       tc_fence_after();
       const uint32_t v_addr = smem_u32(s.v[st]);
+      const uint32_t p_addr = p_addr0 + static_cast<uint32_t>(j & 1) * (BM * BN);
 #pragma unroll
       for (int kk = 0; kk < BN / 32; kk++)
         mma_f8_ss(tmem_O, smem_desc_kmajor(p_addr + kk * 32, BN),
@@ -174,6 +191,35 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t
   // Drain: all MMAs issued by this thread complete before TMEM is freed.
   mma_commit(&s.drain);
   drain_wait(&s.drain, 0, w);
+}
+
+// O row (this thread's TMEM lane) *= alpha: one TMEM round trip, packed
+// fp32x2 multiplies.
+template <int D>
+__device__ __forceinline__ void rescale_row(uint32_t tO, float alpha) {
+  const float2 al2 = make_float2(alpha, alpha);
+  if constexpr (D == 128) {
+    uint32_t o[128];
+    tmem_ld128(tO, o);
+#pragma unroll
+    for (int e = 0; e < 128; e += 2) {
+      const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
+      o[e] = __float_as_uint(v.x);
+      o[e + 1] = __float_as_uint(v.y);
+    }
+    tmem_st128_nowait(tO, o);
+  } else {
+    uint32_t o[64];
+    tmem_ld64(tO, o);
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+      const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
+      o[e] = __float_as_uint(v.x);
+      o[e + 1] = __float_as_uint(v.y);
+    }
+    tmem_st64_nowait(tO, o);
+  }
+  tmem_wait_st();
 }
 
 // Softmax / correction / epilogue for one query row per thread.
@@ -192,24 +238,24 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   const float sqC = valid ? __fmul_rn(__ldg(p.q_scale + static_cast<size_t>(bh) * p.nq_blocks + i / 64), p.c0)
                           : 0.0f;
   const float* ksc = p.k_scale + static_cast<size_t>(bh) * p.nkv_blocks;
-  uint8_t* prow = s.p + r * BN;
+  uint8_t* prow0 = s.p[0] + r * BN;
 
   float m = -INFINITY, l = 0.0f;
   bool ok = true;
+  // seed the S row for the first tile (the MMA issuer waits for it)
+  tmem_fill128_nowait(tS, kBiasBits);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&s.s_free);
   for (int it = 0; it < nk; it++) {
     const int j0 = it * BN;
     if (!warp_wait(&s.s_full, it & 1, w, kSiteSmS)) { ok = false; break; }
     tc_fence_after();
-    uint32_t sv[128];
-    {
-      uint32_t (&h0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&sv[0]);
-      uint32_t (&h1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&sv[64]);
-      tmem_ld64(tS, h0);
-      tmem_ld64(tS + 64, h1);
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&s.s_free);
+    uint32_t sv[128];  // 0x4B400000 + S: the fp32 value 1.5 * 2^23 + S
+    tmem_ld128(tS, sv);
+    const bool more = it + 1 < nk;
+    if (more) tmem_fill128_x8_nowait(tS, kBiasBits);  // seed for the next tile
 
     // scale of each 64-key group of the tile (blocks past the end read as 0)
     const int g0 = 2 * it, g1 = 2 * it + 1;
@@ -218,35 +264,51 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
     const bool full = __all_sync(kFull, nvis == BN);
 
-    // masked max per group in the integer domain: for c >= 0,
-    // max_j fp32(S_j * c) = fp32(max_j S_j * c)
-    int mx0 = INT_MIN, mx1 = INT_MIN;
-    if (full) {
+    // masked keys read as 0.0f, below every seeded score (> 2^23)
+    if (!full) {
 #pragma unroll
-      for (int j = 0; j < 64; j++) mx0 = max(mx0, static_cast<int>(sv[j]));
-#pragma unroll
-      for (int j = 64; j < 128; j++) mx1 = max(mx1, static_cast<int>(sv[j]));
-    } else {
-#pragma unroll
-      for (int j = 0; j < 64; j++) if (j < nvis) mx0 = max(mx0, static_cast<int>(sv[j]));
-#pragma unroll
-      for (int j = 64; j < 128; j++) if (j < nvis) mx1 = max(mx1, static_cast<int>(sv[j]));
+      for (int j = 0; j < BN; j++) sv[j] = j < nvis ? sv[j] : 0u;
     }
-    const float t0 = mx0 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mx0), c0);
-    const float t1 = mx1 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mx1), c1);
+    // masked max per 64-key group on the seeded values, a tree of 3-input
+    // maxima (monotone in S; for c >= 0, max_j fp32(S_j c) = fp32(max_j S_j c))
+    float mg[2];
+#pragma unroll
+    for (int g = 0; g < 2; g++) {
+      float t[8];
+#pragma unroll
+      for (int a = 0; a < 8; a++) {
+        const int j = g * 64 + a * 8;
+        t[a] = fmax3(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1]), __uint_as_float(sv[j + 2]));
+      }
+#pragma unroll
+      for (int a = 0; a < 8; a++) {
+        const int j = g * 64 + a * 8;
+        t[a] = fmax3(t[a], __uint_as_float(sv[j + 3]), __uint_as_float(sv[j + 4]));
+        t[a] = fmax3(t[a], __uint_as_float(sv[j + 5]), __uint_as_float(sv[j + 6]));
+        t[a] = fmaxf(t[a], __uint_as_float(sv[j + 7]));
+      }
+      mg[g] = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
+    }
+    const float t0 = mg[0] < 8388608.0f ? -INFINITY : __fmul_rn(__fsub_rn(mg[0], kBias), c0);
+    const float t1 = mg[1] < 8388608.0f ? -INFINITY : __fmul_rn(__fsub_rn(mg[1], kBias), c1);
     const float m_new = fmaxf(m, fmaxf(t0, t1));
     const float alpha = (m == -INFINITY) ? 0.0f
                         : (m == m_new)   ? 1.0f
                                          : ex2_approx(__fsub_rn(m, m_new));
     const float nm8 = __fsub_rn(8.0f, m_new);  // P scale 2^8 folded into the exponent
 
-    // the P tile is free once P V of the previous tile has completed
-    if (it > 0 && !warp_wait(&s.o_ready, (it - 1) & 1, w, kSiteSmO)) { ok = false; break; }
-    tc_fence_after();
+    // the seed has landed; the MMA issuer may now write S of the next tile
+    if (more) tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (more && lane == 0) mbar_arrive(&s.s_free);
 
+    // P buffer it & 1 was last read by P V of tile it - 2, which completed
+    // before this thread's previous iteration passed its o_ready wait
+    uint8_t* prow = prow0 + (it & 1) * (BM * BN);
     float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
     const float2 nm2 = make_float2(nm8, nm8);
-    const float2 nb2 = make_float2(-12582912.0f, -12582912.0f);
+    const float2 nb2 = make_float2(-kBias, -kBias);
 #pragma unroll
     for (int c = 0; c < 8; c++) {  // 16-key chunks
       uint32_t pk[4];
@@ -257,8 +319,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
         float y[4];
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
-          const float2 sf = __fadd2_rn(make_float2(__uint_as_float(sv[j + e] + 0x4B400000u),
-                                                   __uint_as_float(sv[j + e + 1] + 0x4B400000u)), nb2);
+          const float2 sf = __fadd2_rn(make_float2(__uint_as_float(sv[j + e]), __uint_as_float(sv[j + e + 1])), nb2);
           const float2 x = __ffma2_rn(sf, cc, nm2);
           y[e] = x.x; y[e + 1] = x.y;
         }
@@ -278,17 +339,11 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     const float rs = __fadd_rn(a2.x, a2.y);
     fence_proxy_async_smem();
 
+    // O holds the sum through tile it - 1 once that tile's P V has completed;
     // rescale the O row when the running max moved (never before the first P V)
-    if (it > 0 && __any_sync(kFull, alpha != 1.0f)) {
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + c, o);
-#pragma unroll
-        for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), alpha));
-        tmem_st32(tO + c, o);
-      }
-    }
+    if (it > 0 && !warp_wait(&s.o_ready, (it - 1) & 1, w, kSiteSmO)) { ok = false; break; }
+    tc_fence_after();
+    if (it > 0 && __any_sync(kFull, alpha != 1.0f)) rescale_row<D>(tO, alpha);
     l = __fadd_rn(__fmul_rn(l, alpha), rs);
     m = m_new;
     tc_fence_before();
@@ -355,9 +410,15 @@ __device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint3
 template <int D, bool DUMP>
 __global__ void __launch_bounds__(kThreads, 2)
     k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem<D>& s = *reinterpret_cast<Smem<D>*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 128-byte swizzled TMA tiles and the MMA descriptors need 1024-byte
+  // aligned tiles; refuse (before any barrier, copy or TMEM use) otherwise.
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0 && atomicCAS(p.status, 0, 3 /* SAGE_ERR_CUDA */) == 0)
+      atomicExch(p.status + 1, kSiteSmemAlign);
+    return;
+  }
+  Smem<D>& s = *reinterpret_cast<Smem<D>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = DUMP ? p.dbg_qt : static_cast<int>(blockIdx.x);
   const int bh = DUMP ? p.dbg_bh : static_cast<int>(blockIdx.y);
