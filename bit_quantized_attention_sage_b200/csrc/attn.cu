@@ -54,6 +54,7 @@ constexpr uint32_t kFull = 0xffffffffu;
 // 1.5 * 2^23 + S exactly (|S| <= 128 * 128 * D < 2^22 for D <= 128).
 constexpr uint32_t kBiasBits = 0x4B400000u;
 constexpr float kBias = 12582912.0f;
+constexpr uint32_t kNegInfBits = 0xFF800000u;
 
 // wait-site codes for the status word (kernel 1 = attention)
 enum : int {
@@ -193,6 +194,11 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t
   drain_wait(&s.drain, 0, w);
 }
 
+// Scale of K block g of a head; blocks past the end read as 0.
+__device__ __forceinline__ float k_block_scale(const float* ksc, int g, int nblocks) {
+  return g < nblocks ? __ldg(ksc + g) : 0.0f;
+}
+
 // O row (this thread's TMEM lane) *= alpha: one TMEM round trip, packed
 // fp32x2 multiplies.
 template <int D>
@@ -240,6 +246,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   const float* ksc = p.k_scale + static_cast<size_t>(bh) * p.nkv_blocks;
   uint8_t* prow0 = s.p[0] + r * BN;
 
+  float ks0 = k_block_scale(ksc, 0, p.nkv_blocks), ks1 = k_block_scale(ksc, 1, p.nkv_blocks);
   float m = -INFINITY, l = 0.0f;
   bool ok = true;
   // seed the S row for the first tile (the MMA issuer waits for it)
@@ -257,17 +264,19 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     const bool more = it + 1 < nk;
     if (more) tmem_fill128_x8_nowait(tS, kBiasBits);  // seed for the next tile
 
-    // scale of each 64-key group of the tile (blocks past the end read as 0)
-    const int g0 = 2 * it, g1 = 2 * it + 1;
-    const float c0 = __fmul_rn(sqC, g0 < p.nkv_blocks ? __ldg(ksc + g0) : 0.0f);
-    const float c1 = __fmul_rn(sqC, g1 < p.nkv_blocks ? __ldg(ksc + g1) : 0.0f);
+    // scale of each 64-key group of the tile; the next tile's K scales are
+    // loaded now so that their latency is hidden behind this tile
+    const float c0 = __fmul_rn(sqC, ks0), c1 = __fmul_rn(sqC, ks1);
+    ks0 = k_block_scale(ksc, 2 * it + 2, p.nkv_blocks);
+    ks1 = k_block_scale(ksc, 2 * it + 3, p.nkv_blocks);
     const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
     const bool full = __all_sync(kFull, nvis == BN);
 
-    // masked keys read as 0.0f, below every seeded score (> 2^23)
+    // masked keys read as -inf: below every seeded score (> 2^23) in the
+    // max, and exp2 of their argument is exactly 0 (see ce0, ce1, nm8)
     if (!full) {
 #pragma unroll
-      for (int j = 0; j < BN; j++) sv[j] = j < nvis ? sv[j] : 0u;
+      for (int j = 0; j < BN; j++) sv[j] = j < nvis ? sv[j] : kNegInfBits;
     }
     // masked max per 64-key group on the seeded values, a tree of 3-input
     // maxima (monotone in S; for c >= 0, max_j fp32(S_j c) = fp32(max_j S_j c))
@@ -295,7 +304,14 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     const float alpha = (m == -INFINITY) ? 0.0f
                         : (m == m_new)   ? 1.0f
                                          : ex2_approx(__fsub_rn(m, m_new));
-    const float nm8 = __fsub_rn(8.0f, m_new);  // P scale 2^8 folded into the exponent
+    // P scale 2^8 folded into the exponent; a row with no visible key so far
+    // (m_new = -inf) keeps every argument at -inf
+    const float nm8 = m_new == -INFINITY ? 0.0f : __fsub_rn(8.0f, m_new);
+    // exp arguments fma(S, c, nm8) with c replaced by FLT_MIN where c = 0:
+    // identical for visible keys (c = 0 gives nm8 either way: |S| FLT_MIN is
+    // far below half an ulp of nm8) and -inf for masked keys (-inf * c must
+    // not be -inf * 0 = NaN)
+    const float ce0 = c0 > 0.0f ? c0 : FLT_MIN, ce1 = c1 > 0.0f ? c1 : FLT_MIN;
 
     // the seed has landed; the MMA issuer may now write S of the next tile
     if (more) tmem_wait_st();
@@ -312,7 +328,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
 #pragma unroll
     for (int c = 0; c < 8; c++) {  // 16-key chunks
       uint32_t pk[4];
-      const float2 cc = c < 4 ? make_float2(c0, c0) : make_float2(c1, c1);
+      const float2 cc = c < 4 ? make_float2(ce0, ce0) : make_float2(ce1, ce1);
 #pragma unroll
       for (int q4 = 0; q4 < 4; q4++) {
         const int j = c * 16 + q4 * 4;
@@ -322,10 +338,6 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
           const float2 sf = __fadd2_rn(make_float2(__uint_as_float(sv[j + e]), __uint_as_float(sv[j + e + 1])), nb2);
           const float2 x = __ffma2_rn(sf, cc, nm2);
           y[e] = x.x; y[e + 1] = x.y;
-        }
-        if (!full) {
-#pragma unroll
-          for (int e = 0; e < 4; e++) y[e] = (j + e < nvis) ? y[e] : -INFINITY;
         }
 #pragma unroll
         for (int e = 0; e < 4; e++) y[e] = ex2_approx(y[e]);

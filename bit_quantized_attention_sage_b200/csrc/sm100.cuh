@@ -100,6 +100,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Same contract as mbar_wait, but the thread polls (try_wait without a
+// suspend hint) instead of being suspended: for the single-thread roles
+// whose reaction time is on the critical path (the MMA issuer).
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                               int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*w.abort) return false;
+    if (clock64() - t0 > w.budget) {
+      record_timeout(w.status, site);
+      *w.abort = 1;
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
