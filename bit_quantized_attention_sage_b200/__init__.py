@@ -134,7 +134,7 @@ class QuantizedQKV:
         if name == "k_i8":
             return t.view(torch.int8).view(s.B, s.H, nkp, s.D)
         if name == "v_f8":
-            return t.view(s.B, s.H, s.D, nkp)
+            return t.view(s.B, s.H, nkp, s.D)
         if name == "q_scale":
             return t.view(torch.float32).view(s.B, s.H, nqp // 64)
         if name == "k_scale":

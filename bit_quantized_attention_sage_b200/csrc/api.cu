@@ -127,8 +127,8 @@ bool make_maps(const sage_qkv_quant* q, const sage_shape* s, AttnMaps* m) {
                       swqk) &&
          encode_u8_3d(&m->k, q->k_i8, D, pad64(s->Nkv), bh, static_cast<uint32_t>(D), kAttnBN,
                       swqk) &&
-         encode_u8_3d(&m->v, q->v_f8, pad64(s->Nkv), D, bh, kAttnBN, static_cast<uint32_t>(D),
-                      CU_TENSOR_MAP_SWIZZLE_128B);
+         encode_u8_3d(&m->v, q->v_f8, D, pad64(s->Nkv), bh, static_cast<uint32_t>(D), kAttnBN,
+                      swqk);
 }
 
 AttnParams base_params(const sage_qkv_quant* q, const sage_shape* s, const DeviceState* d) {

@@ -10,14 +10,15 @@
 //
 // One CTA owns 128 query rows of one (batch, head) and streams the visible
 // KV tiles of 128 keys.  Warp roles (192 threads, two CTAs per SM):
-//   warp 0      TMA producer: the Q tile once, then K and V^T tiles through
-//               a two-stage shared-memory ring (128-byte swizzle).
+//   warp 0      TMA producer: the Q tile once, then K and V tiles through
+//               a two-stage shared-memory ring (128-byte swizzle; V tiles
+//               are [keys][D], used as MN-major operands).
 //               The e4m3 P tile is double-buffered: the softmax of tile k
 //               writes P(k) while P V of tile k-1 may still read P(k-1).
 //   warp 1      allocates 256 TMEM columns (S: 128 x 128 int32, O: 128 x D
 //               fp32) and one elected thread issues every tcgen05.mma:
 //               S = Q K^T (kind::i8) for tile k+1 while the softmax warps
-//               work on tile k, then O (+)= P V^T (kind::f8f6f4).
+//               work on tile k, then O (+)= P V (kind::f8f6f4).
 //   warps 2-5   softmax: thread t of the warpgroup owns query row t (TMEM
 //               lane t).  The S accumulator columns are seeded with the bit
 //               pattern 0x4B400000 before each Q K^T, so the int32 result
@@ -66,7 +67,7 @@ template <int D>
 struct alignas(1024) Smem {
   uint8_t q[BM * D];         // int8 Q tile [128 rows][D]
   uint8_t k[NS][BN * D];     // int8 K tiles [128 keys][D]
-  uint8_t v[NS][D * BN];     // e4m3 V^T tiles [D][128 keys]
+  uint8_t v[NS][BN * D];     // e4m3 V tiles [128 keys][D] (MN-major operand)
   uint8_t p[2][BM * BN];     // e4m3 P tiles [parity][128 rows][128 keys], 128-byte swizzle
   uint64_t q_full;
   uint64_t k_full[NS], k_empty[NS];
@@ -134,7 +135,7 @@ __device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int b
     if (DUMP) continue;
     if (it >= NS && !mbar_wait(&s.v_empty[st], ph ^ 1, w, kSiteProdVEmpty)) break;
     mbar_arrive_expect_tx(&s.v_full[st], D * BN);
-    tma_load_3d(s.v[st], &maps.v, &s.v_full[st], kt * BN, 0, bh);
+    tma_load_3d(s.v[st], &maps.v, &s.v_full[st], 0, kt * BN, bh);
     v_issued++;
   }
   // Drain: every issued load must have landed before the CTA may exit.  A
@@ -151,7 +152,8 @@ template <int D, bool DUMP>
 __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t tmem_O, int nk,
                                            const WaitCtx& w) {
   constexpr uint32_t idesc_qk = idesc_i8_s32(BM, BN);
-  constexpr uint32_t idesc_pv = idesc_e4m3_f32(BM, D);
+  // P V: B = V tile stored [keys][D], i.e. N-contiguous (MN-major)
+  constexpr uint32_t idesc_pv = idesc_e4m3_f32(BM, D) | kIdescBMajorMN;
   const uint32_t q_addr = smem_u32(s.q);
   const uint32_t p_addr0 = smem_u32(s.p[0]);
   bool ok = mbar_wait(&s.q_full, 0, w, kSiteMmaQ);
@@ -172,7 +174,7 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t
       mma_commit(&s.k_empty[st]);
       mma_commit(&s.s_full);
     }
-    if (!DUMP && it > 0) {  // O (+)= P V^T for tile it - 1
+    if (!DUMP && it > 0) {  // O (+)= P V for tile it - 1
       const int j = it - 1;
       const int st = j % NS;
       const uint32_t ph = (j / NS) & 1;
@@ -184,7 +186,7 @@ __device__ __forceinline__ void mma_issuer(Smem<D>& s, uint32_t tmem_S, uint32_t
 #pragma unroll
       for (int kk = 0; kk < BN / 32; kk++)
         mma_f8_ss(tmem_O, smem_desc_kmajor(p_addr + kk * 32, BN),
-                  smem_desc_kmajor(v_addr + kk * 32, BN), idesc_pv, (j > 0 || kk > 0));
+                  smem_desc_mnmajor(v_addr + kk * 32 * D, D), idesc_pv, (j > 0 || kk > 0));
       mma_commit(&s.v_empty[st]);
       mma_commit(&s.o_ready);
     }

@@ -34,7 +34,7 @@ struct AttnParams {
 struct AttnMaps {
   CUtensorMap q;  // int8 [BH][Nq_pad][D], box D x 128
   CUtensorMap k;  // int8 [BH][Nkv_pad][D], box D x 128
-  CUtensorMap v;  // e4m3 [BH][D][Nkv_pad], box 128 x D
+  CUtensorMap v;  // e4m3 [BH][Nkv_pad][D], box D x 128
 };
 
 size_t attn_smem_bytes(int D);

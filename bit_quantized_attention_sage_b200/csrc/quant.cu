@@ -15,8 +15,7 @@
 //   finalize one CTA per (head, 32 channels): ascending sum of the block
 //            sums -> k_mean; max of the block maxima -> v_scale, 448/absmax.
 //   pass2    one CTA per (head, 64-token block): K - mean block codes + scale;
-//            V codes written channel-major ([B,H,D,Nkv_pad]) through shared
-//            memory so that the attention kernel reads K-major V^T tiles.
+//            V codes, token-major like the K codes ([B,H,Nkv_pad,D]).
 // Memory traffic: 16-byte vectorised bf16 loads; every fp32 operation is an
 // explicit IEEE round-to-nearest intrinsic so the codes match a plain CPU
 // implementation bit for bit.
@@ -219,7 +218,6 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;
   __shared__ float red[kThreads / 32];
-  __shared__ __align__(16) uint8_t vt[D * kBlk];  // [d][token] e4m3 codes
 
   const int blk = blockIdx.x;
   const int bh = blockIdx.y;
@@ -227,6 +225,19 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   const int nkv_pad = nkb * kBlk;
   const int valid = min(kBlk, a.Nkv - blk * kBlk);
   const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
+
+  // The V loads are issued first, together with the K loads, so that the
+  // whole 64-token block of K and V is in flight at once.  Chunk c*256 + t
+  // (8 channels of one token) belongs to thread t, as for K.
+  uint4 vu[CH];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.v + base);
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      vu[c] = chunk / kChunksPerRow < valid ? __ldg(src + chunk) : make_uint4(0, 0, 0, 0);
+    }
+  }
 
   {  // K - mean, block codes and scale
     const uint4* src = reinterpret_cast<const uint4*>(a.k + base);
@@ -248,40 +259,33 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
                              red);
   }
 
-  {  // V codes, transposed through shared memory
-    // thread t owns token row t % 64 and channels [g*DG, g*DG + DG) with
-    // g = t / 64; a warp then stores 32 consecutive tokens of one channel per
-    // instruction (32 bytes, no bank conflict), and the rows are written out
-    // as 16-byte chunks.
-    constexpr int DG = D / (kThreads / kBlk);  // channels per thread: 32 (D=128) or 16
-    const int row = threadIdx.x % kBlk;
-    const int g = threadIdx.x / kBlk;
-    const uint4* src = reinterpret_cast<const uint4*>(a.v + base + static_cast<size_t>(row) * D + g * DG);
-    const float* inv = a.ws_vinv + static_cast<size_t>(bh) * D + g * DG;
+  {  // V codes, token-major like K: [BH][Nkv_pad][D] (the attention kernel
+     // reads V tiles as MN-major tensor-core operands, so no transpose)
+    const float* inv = a.ws_vinv + static_cast<size_t>(bh) * D;
+    uint8_t* dst = a.v_f8 + (static_cast<size_t>(bh) * nkv_pad + static_cast<size_t>(blk) * kBlk) * D;
 #pragma unroll
-    for (int c = 0; c < DG / 8; c++) {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (row < valid) u = __ldg(src + c);
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      const int col = (chunk % kChunksPerRow) * 8;
       float x[8];
-      unpack8(u, x);
+      unpack8(vu[c], x);
+      uint32_t w[2];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const int d = c * 8 + e;
-        const float i0 = __ldg(inv + d), i1 = __ldg(inv + d + 1);
-        uint32_t p = cvt_e4m3x2(__fmul_rn(x[e], i0), __fmul_rn(x[e + 1], i1));
-        if (i0 == 0.0f || row >= valid) p &= 0xFF00u;  // zero channel or padding token
-        if (i1 == 0.0f || row >= valid) p &= 0x00FFu;
-        vt[(g * DG + d) * kBlk + row] = static_cast<uint8_t>(p & 0xFF);
-        vt[(g * DG + d + 1) * kBlk + row] = static_cast<uint8_t>(p >> 8);
+      for (int h = 0; h < 2; h++) {
+        uint32_t b4 = 0;
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          const int d = col + h * 4 + e;
+          const float i0 = __ldg(inv + d), i1 = __ldg(inv + d + 1);
+          uint32_t pr = cvt_e4m3x2(__fmul_rn(x[h * 4 + e], i0), __fmul_rn(x[h * 4 + e + 1], i1));
+          if (i0 == 0.0f) pr &= 0xFF00u;  // zero channel
+          if (i1 == 0.0f) pr &= 0x00FFu;
+          b4 |= pr << (8 * e);
+        }
+        w[h] = row < valid ? b4 : 0u;  // padding tokens are 0
       }
-    }
-    __syncthreads();
-    // D rows of 64 bytes: 4 x 16-byte chunks per channel
-    uint8_t* dst = a.v_f8 + static_cast<size_t>(bh) * D * nkv_pad + static_cast<size_t>(blk) * kBlk;
-    for (int chunk = threadIdx.x; chunk < D * (kBlk / 16); chunk += kThreads) {
-      const int d = chunk / (kBlk / 16), part = chunk % (kBlk / 16);
-      *reinterpret_cast<uint4*>(dst + static_cast<size_t>(d) * nkv_pad + part * 16) =
-          reinterpret_cast<const uint4*>(vt)[chunk];
+      *reinterpret_cast<uint2*>(dst + static_cast<size_t>(row) * D + col) = make_uint2(w[0], w[1]);
     }
   }
 }

@@ -218,6 +218,11 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
          (uint32_t(M >> 4) << 24);
 }
 
+// Instruction-descriptor bit 16: operand B is MN-major (N contiguous in
+// shared memory) instead of K-major.  Valid for 8-bit (e4m3, e5m2, int8),
+// 16-bit and tf32 operands.
+constexpr uint32_t kIdescBMajorMN = 1u << 16;
+
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
 // with 128-byte (layout 2) or 64-byte (layout 4) swizzling: start address
 // >> 4 in bits 0-13, leading byte offset (unused for swizzled K-major, 16 B)
@@ -225,6 +230,19 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
 // 32-45, descriptor version 1 in 46-47, swizzle mode in 61-63.  The tile base
 // must be aligned to the swizzle atom (8 rows x row bytes).
 __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, uint32_t row_bytes) {
+  const uint64_t layout = (row_bytes == 128) ? 2ull : 4ull;
+  const uint64_t sbo = (8ull * row_bytes) >> 4;
+  return (uint64_t((saddr >> 4) & 0x3FFFu)) | (1ull << 16) | (sbo << 32) | (1ull << 46) |
+         (layout << 61);
+}
+
+// Shared-memory matrix descriptor for an MN-major 8-bit operand tile written
+// by TMA with 128-byte (N = 128 bytes per K row, layout 2) or 64-byte (N = 64
+// bytes, layout 4) swizzling: the swizzle atom spans the whole N extent, so
+// the leading byte offset (stride between atoms along N) is unused (16 B),
+// and the stride byte offset is the distance between groups of 8 K rows.
+// `saddr` is the first K row of the slice and must be atom aligned (8 rows).
+__device__ __forceinline__ uint64_t smem_desc_mnmajor(uint32_t saddr, uint32_t row_bytes) {
   const uint64_t layout = (row_bytes == 128) ? 2ull : 4ull;
   const uint64_t sbo = (8ull * row_bytes) >> 4;
   return (uint64_t((saddr >> 4) & 0x3FFFu)) | (1ull << 16) | (sbo << 32) | (1ull << 46) |

@@ -84,8 +84,8 @@ typedef struct {
  *   k_i8    int8  [B, H, Nkv_pad, D]  codes of K - k_mean; rows >= Nkv are 0
  *   k_scale f32   [B, H, Nkv_pad/64]  per-block K scale
  *   k_mean  f32   [B, H, D]           per-channel mean of K over all Nkv tokens
- *   v_f8    e4m3  [B, H, D, Nkv_pad]  V codes, CHANNEL-major (transposed):
- *                                     byte ((b*H+h)*D + d)*Nkv_pad + n;
+ *   v_f8    e4m3  [B, H, Nkv_pad, D]  V codes, token-major like k_i8:
+ *                                     byte ((b*H+h)*Nkv_pad + n)*D + d;
  *                                     tokens n >= Nkv are 0
  *   v_scale f32   [B, H, D]           per-channel V scale (absmax/448)
  * Dequantization: q = q_i8 * q_scale[n/64]; k = k_i8 * k_scale[n/64] + k_mean;

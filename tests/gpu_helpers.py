@@ -44,9 +44,9 @@ def check_quant_head(qkv, b, h, ref):
     for name, key in (("q_scale", "qs"), ("k_scale", "ks"), ("k_mean", "mu"), ("v_scale", "vs")):
         got = qkv.view(name)[b, h].cpu().numpy()
         assert np.array_equal(f32_bits(got), f32_bits(ref[key])), name + " differs"
-    v8t = qkv.view("v_f8")[b, h].cpu().numpy()  # [D, Nkv_pad]
-    assert np.array_equal(v8t[:, :s.Nkv].T, ref["v8"]), "v_f8 differs"
-    assert not v8t[:, s.Nkv:].any(), "v_f8 padding not zero"
+    v8 = qkv.view("v_f8")[b, h].cpu().numpy()  # [Nkv_pad, D]
+    assert np.array_equal(v8[:s.Nkv], ref["v8"]), "v_f8 differs"
+    assert not v8[s.Nkv:].any(), "v_f8 padding not zero"
 
 
 def bf16_half_ulp(x):
