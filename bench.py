@@ -48,6 +48,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the 72-point sweep (N x D x mask x K outlier magnitude) and report "
+                         "TOPS and accuracy against fp64 attention per point, one JSON line each")
+    ap.add_argument("--sweep-filter", default="",
+                    help="only sweep points whose name contains this string")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="approximate CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -368,6 +373,67 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ sweep
+
+def fp64_rows(w, q, k, v, rows):
+    """Textbook softmax attention in fp64 (torch, on the GPU) for the given
+    query rows of head (0, 0): the full-precision accuracy reference."""
+    import torch
+    rows = torch.as_tensor(rows, device=q.device, dtype=torch.int64)
+    qd = q[0, 0, rows].double()
+    kd, vd = k[0, 0].double(), v[0, 0].double()
+    s = (qd @ kd.T) / float(np.sqrt(w.D))
+    g = rows + (w.Nkv - w.Nq)
+    if w.mask == 1:
+        lim = g + 1
+    elif w.mask == 2:
+        lim = (g // w.mask_block + 1) * w.mask_block
+    else:
+        lim = torch.full_like(g, w.Nkv)
+    keys = torch.arange(w.Nkv, device=q.device)
+    s = s.masked_fill(keys[None, :] >= lim[:, None], float("-inf"))
+    return torch.softmax(s, dim=1) @ vd
+
+
+def run_sweep(args):
+    """One JSON line per sweep point: step and attention TOPS (CUDA events,
+    inputs resident) and the accuracy of 64 sampled rows of head 0 against
+    fp64 attention (cosine similarity and mean relative L1)."""
+    import torch
+    import bit_quantized_attention_sage_b200 as sage
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    sage.lib()
+    pk = peaks()
+    for w in synth.sweep():
+        if args.sweep_filter and args.sweep_filter not in w.name:
+            continue
+        runner = Runner(w, 0, device)
+        t = time_steps(runner, args.steps, args.warmup, 1, per_kernel=True)
+        o32 = torch.empty((w.B, w.H, w.Nq, w.D), dtype=torch.float32, device=device)
+        sage.attn_fwd(runner.qkv, w.mask, w.mask_block, out=runner.o, o_f32=o32)
+        if sage.sync_status() != 0:
+            raise RuntimeError("device status error in sweep point " + w.name)
+        rows = np.sort(np.random.default_rng(w.seed).choice(w.Nq, size=min(64, w.Nq),
+                                                            replace=False))
+        ref = fp64_rows(w, runner.q, runner.k, runner.v, rows)
+        got = o32[0, 0, torch.as_tensor(rows, device=device)].double()
+        cos = float(torch.nn.functional.cosine_similarity(got.flatten(), ref.flatten(), dim=0))
+        rel = float(((got - ref).abs().sum(1) / ref.abs().sum(1).clamp_min(1e-30)).mean())
+        ops = w.ops()
+        print(json.dumps({
+            "sweep_point": w.name, "N": w.Nq, "D": w.D, "H": w.H,
+            "mask": ["none", "causal", "block_causal"][w.mask], "mask_block": w.mask_block,
+            "outlier_mag": w.outlier_mag, "step_ms": round(t["ms"], 4),
+            "attn_ms": round(t["attn_ms"], 4), "quant_ms": round(t["quant_ms"], 4),
+            "TOPS": round(ops / (t["ms"] / 1e3) / 1e12, 2),
+            "attn_TOPS": round(ops / (t["attn_ms"] / 1e3) / 1e12, 2),
+            "attn_frac_of_peak": round(ops / (t["attn_ms"] / 1e3) / 1e12 / pk["i8_sustained"], 4),
+            "cos_vs_fp64": round(cos, 6), "relL1_vs_fp64": round(rel, 5)}), flush=True)
+        del runner, o32
+        torch.cuda.empty_cache()
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args):
@@ -403,6 +469,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

@@ -102,3 +102,23 @@ def test_full_size_sampled(w):
     # the recipe's own accuracy against fp64 (reported; outliers x20 cost cos ~0.995)
     print("%s: cos %.5f relL1 %.4f" % (w.name, cos, rel))
     assert cos > 0.99 and rel < 0.12
+
+
+SWEEP = [w for w in synth.sweep() if w.Nq in (4096, 16384)] + [
+    w for w in synth.sweep() if w.name in ("sweep_n131072_d64_bc_mag20", "sweep_n131072_d128_nc_mag0")]
+
+
+@pytest.mark.parametrize("w", SWEEP, ids=lambda w: w.name)
+def test_sweep_sampled(w):
+    """Sweep points (N x D x mask x K outlier magnitude, H = 16): the sampled
+    head's quantized tensors bit-exact, 32 sampled rows against the oracle."""
+    q, k, v = synth.full(w)
+    qkv, o, o32, lse = run(q, k, v, w.mask, w.mask_block)
+    rng = np.random.default_rng(w.seed)
+    bh = int(rng.integers(w.B * w.H))
+    b, h = divmod(bh, w.H)
+    ref = oracle.quant_head(q[b, h], k[b, h], v[b, h])
+    check_quant_head(qkv, b, h, ref)
+    rows = _sample_rows(w, rng, 32)
+    check_rows(ref, rows, rows_of(o, b, h, rows), rows_of(o32, b, h, rows),
+               rows_of(lse, b, h, rows), w.mask, w.mask_block)
