@@ -20,6 +20,7 @@ from . import build as _build
 MASK_NONE, MASK_CAUSAL, MASK_BLOCK_CAUSAL = 0, 1, 2
 BLK = 64          # Q/K quantization block (tokens)
 TKV = 128         # KV tile width of the online softmax (the device kernel's)
+BQ = 128          # query rows per block of a block-sparse mask (one query tile)
 
 # Relative uncertainty of the device's exp2 result plus one fp32 rounding of
 # the oracle's own exp2.  The device uses the hardware ex2.approx.ftz.f32; its
@@ -57,6 +58,12 @@ def lib():
         L.orc_attn_rows_identity.restype = i32
         L.orc_attn_rows_identity.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
                                              P, i64, P, P, i32]
+        L.orc_attn_rows_bs.restype = i32
+        L.orc_attn_rows_bs.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
+                                       P, i64, i64, P, i64, P, P, P, i32]
+        L.orc_attn_rows_identity_bs.restype = i32
+        L.orc_attn_rows_identity_bs.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
+                                                P, i64, i64, P, i64, P, P, i32]
         L.orc_attn_fp64_rows.restype = i32
         L.orc_attn_fp64_rows.argtypes = [P, P, P, i64, i64, i32, i32, i64, P, i64, P, i32]
         _lib = L
@@ -138,10 +145,22 @@ def row_limit(i, nq, nkv, mask, mb):
 
 # ---------------------------------------------------------------- attention
 
+def _block_mask(block_mask, nkv, tkv):
+    """(pointer, bq, n_kt) of an optional block mask [n_qt, n_kt] of one head."""
+    if block_mask is None:
+        return None, 0, 0, None
+    bm = np.ascontiguousarray(block_mask, np.uint8)
+    if bm.ndim != 2 or bm.shape[1] < -(-nkv // tkv):
+        raise ValueError("block mask must be [n_qtiles, ceil(Nkv / tkv)]")
+    return _p(bm), BQ, bm.shape[1], bm
+
+
 def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
-              threads=None):
+              threads=None, block_mask=None):
     """Same-quantization attention of one quantized head on the given rows.
 
+    block_mask: optional uint8 [ceil(Nq / 128), ceil(Nkv / tkv)] of this head;
+    query row i visits KV tile t only if block_mask[i // 128, t] != 0.
     Returns (o [n, D] float64 of the fp32 recipe, slack [n, D] or None, lse [n]).
     """
     rows = np.ascontiguousarray(rows, np.int64)
@@ -155,16 +174,18 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
     qs = np.ascontiguousarray(qh["qs"])
     ks = np.ascontiguousarray(qh["ks"])
     vs = np.ascontiguousarray(qh["vs"])
-    rc = lib().orc_attn_rows(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
-                             qh["nq"], qh["nkv"], D, mask, mb, tkv, eps,
-                             _p(rows), n, _p(o), _p(slack) if slack is not None else None,
-                             _p(lse), _threads(threads))
+    bptr, bq, n_kt, _keep = _block_mask(block_mask, qh["nkv"], tkv)
+    rc = lib().orc_attn_rows_bs(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
+                                qh["nq"], qh["nkv"], D, mask, mb, tkv, eps, bptr, bq, n_kt,
+                                _p(rows), n, _p(o), _p(slack) if slack is not None else None,
+                                _p(lse), _threads(threads))
     if rc:
         raise ValueError("orc_attn_rows: invalid arguments")
     return o, slack, lse
 
 
-def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=None):
+def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=None,
+                       block_mask=None):
     """The oracle's tiled loop with identity quantizers, fp64 throughout."""
     q = np.ascontiguousarray(q, np.float64)
     k = np.ascontiguousarray(k, np.float64)
@@ -173,9 +194,10 @@ def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=Non
     n, D = rows.size, q.shape[1]
     o = np.empty((n, D), np.float64)
     lse = np.empty(n, np.float64)
-    rc = lib().orc_attn_rows_identity(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
-                                      mask, mb, tkv, _p(rows), n, _p(o), _p(lse),
-                                      _threads(threads))
+    bptr, bq, n_kt, _keep = _block_mask(block_mask, k.shape[0], tkv)
+    rc = lib().orc_attn_rows_identity_bs(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
+                                         mask, mb, tkv, bptr, bq, n_kt, _p(rows), n, _p(o),
+                                         _p(lse), _threads(threads))
     if rc:
         raise ValueError("orc_attn_rows_identity: invalid arguments")
     return o, lse

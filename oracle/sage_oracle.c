@@ -33,6 +33,11 @@
  *   orc_attn_rows (quant)    : closed forms (Q = 0, single visible key) and
  *                              the error bound against fp64 attention.
  *   orc_attn_fp64_rows       : textbook softmax attention (torch) to 1e-12.
+ *   orc_attn_rows_bs / _identity_bs (block mask): identity mode against
+ *                              textbook softmax attention under the combined
+ *                              row and block mask to 1e-12; an all-ones mask
+ *                              reproduces the dense result bit for bit; rows
+ *                              that see no key give O = 0, lse = -inf.
  */
 #include <math.h>
 #include <pthread.h>
@@ -305,6 +310,10 @@ typedef struct {
     double *o;     /* [nrows, D] */
     double *slack; /* [nrows, D] or NULL */
     double *lse;   /* [nrows] natural-log log-sum-exp, or NULL */
+    /* block-sparse skipping (NULL: dense): KV tile t (keys t*tkv ..) is
+     * visited by query row i only if bmask[(i / bq) * n_kt + t] != 0 */
+    const uint8_t *bmask;
+    long bq, n_kt;
 } attn_job;
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
@@ -369,6 +378,8 @@ static void attend_row(const attn_job *J, long r)
         o[d] = 0.0;
 
     for (long j0 = 0; j0 < lim; j0 += tkv) {
+        if (J->bmask && !J->bmask[(i / J->bq) * J->n_kt + j0 / tkv])
+            continue; /* tile switched off by the block mask */
         long j1 = j0 + tkv < lim ? j0 + tkv : lim; /* visible keys of this tile */
         long nj = j1 - j0;
         /* scores */
@@ -442,8 +453,17 @@ static void attend_row(const attn_job *J, long r)
         else
             lf = lf * (float)alpha + rowsum_f;
     }
-    /* output */
-    if (J->identity) {
+    /* output; a row that sees no key at all (possible only with a block
+     * mask) has no softmax: O = 0 and lse = -inf by definition */
+    if ((J->identity && l == 0.0) || (!J->identity && lf == 0.0f)) {
+        for (int d = 0; d < D; d++) {
+            o[d] = 0.0;
+            if (sl)
+                sl[d] = 0.0;
+        }
+        if (J->lse)
+            J->lse[r] = -INFINITY;
+    } else if (J->identity) {
         for (int d = 0; d < D; d++)
             o[d] = o[d] / l;
         if (J->lse)
@@ -515,12 +535,15 @@ static void attend_row_cb(const void *job, long r) { attend_row((const attn_job 
  * o, slack: [nrows, D] doubles; lse: [nrows] or NULL; slack may be NULL.
  * eps: relative uncertainty of the device exp2 (plus one fp32 rounding) used
  * to mark e4m3 rounding decisions of p*256 that may go either way. */
-int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
-                  const uint8_t *v8, const float *vs, long nq, long nkv, int D,
-                  int mask, long mb, long tkv, double eps,
-                  const long *rows, long nrows, double *o, double *slack, double *lse,
-                  int nthreads)
+int orc_attn_rows_bs(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
+                     const uint8_t *v8, const float *vs, long nq, long nkv, int D,
+                     int mask, long mb, long tkv, double eps,
+                     const uint8_t *bmask, long bq, long n_kt,
+                     const long *rows, long nrows, double *o, double *slack, double *lse,
+                     int nthreads)
 {
+    if (bmask && (bq <= 0 || n_kt < (nkv + tkv - 1) / tkv))
+        return 1;
     if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0)
         return 1;
     if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
@@ -547,6 +570,9 @@ int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const flo
     J.o = o;
     J.slack = slack;
     J.lse = lse;
+    J.bmask = bmask;
+    J.bq = bq;
+    J.n_kt = n_kt;
     if (slack)
         memset(slack, 0, sizeof(double) * (size_t)(nrows * D));
     for_rows(&J, attend_row_cb, nrows, nthreads);
@@ -555,11 +581,14 @@ int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const flo
 
 /* The same tiled online-softmax loop with the quantizers replaced by
  * identity and all arithmetic in fp64 (q, k, v: [n, D] doubles). */
-int orc_attn_rows_identity(const double *q, const double *k, const double *v,
-                           long nq, long nkv, int D, int mask, long mb, long tkv,
-                           const long *rows, long nrows, double *o, double *lse,
-                           int nthreads)
+int orc_attn_rows_identity_bs(const double *q, const double *k, const double *v,
+                              long nq, long nkv, int D, int mask, long mb, long tkv,
+                              const uint8_t *bmask, long bq, long n_kt,
+                              const long *rows, long nrows, double *o, double *lse,
+                              int nthreads)
 {
+    if (bmask && (bq <= 0 || n_kt < (nkv + tkv - 1) / tkv))
+        return 1;
     if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0)
         return 1;
     if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
@@ -581,8 +610,31 @@ int orc_attn_rows_identity(const double *q, const double *k, const double *v,
     J.nrows = nrows;
     J.o = o;
     J.lse = lse;
+    J.bmask = bmask;
+    J.bq = bq;
+    J.n_kt = n_kt;
     for_rows(&J, attend_row_cb, nrows, nthreads);
     return 0;
+}
+
+/* Dense forms (no block mask). */
+int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
+                  const uint8_t *v8, const float *vs, long nq, long nkv, int D,
+                  int mask, long mb, long tkv, double eps,
+                  const long *rows, long nrows, double *o, double *slack, double *lse,
+                  int nthreads)
+{
+    return orc_attn_rows_bs(q8, qs, k8, ks, v8, vs, nq, nkv, D, mask, mb, tkv, eps, NULL, 0, 0,
+                            rows, nrows, o, slack, lse, nthreads);
+}
+
+int orc_attn_rows_identity(const double *q, const double *k, const double *v,
+                           long nq, long nkv, int D, int mask, long mb, long tkv,
+                           const long *rows, long nrows, double *o, double *lse,
+                           int nthreads)
+{
+    return orc_attn_rows_identity_bs(q, k, v, nq, nkv, D, mask, mb, tkv, NULL, 0, 0, rows, nrows,
+                                     o, lse, nthreads);
 }
 
 /* ------------------------------------------------------------------ */
