@@ -67,6 +67,8 @@ def lib():
         L.sage_quant_qk_noalloc.argtypes = [P, P, P, P, P, P]
         L.sage_attn_fwd.restype = I
         L.sage_attn_fwd.argtypes = [P, P, I, I, P, P, P, P]
+        L.sage_attn_fwd_block_sparse.restype = I
+        L.sage_attn_fwd_block_sparse.argtypes = [P, P, I, I, P, P, P, P, P]
         L.sage_debug_qk_int32.restype = I
         L.sage_debug_qk_int32.argtypes = [P, P, P, I, P, P]
         L.sage_debug_timeout_probe.restype = I
@@ -183,17 +185,37 @@ def quant_qk_noalloc(q, k, v, out, stream=None):
     return out
 
 
-def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, stream=None):
-    """sage_attn_fwd on a QuantizedQKV; returns the bf16 output tensor."""
+def block_mask_shape(B, H, Nq, Nkv):
+    """Shape of a block mask: one byte per 128-query x 128-key tile."""
+    return (B, H, -(-Nq // 128), -(-Nkv // 128))
+
+
+def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, stream=None,
+             block_mask=None):
+    """sage_attn_fwd on a QuantizedQKV; returns the bf16 output tensor.
+
+    block_mask: optional contiguous uint8 CUDA tensor of block_mask_shape();
+    tiles whose byte is 0 are skipped (sage_attn_fwd_block_sparse)."""
     import torch
     s = qkv.shape
     dev = qkv.bufs["q_i8"].device
     if out is None:
         out = torch.empty((s.B, s.H, s.Nq, s.D), dtype=torch.bfloat16, device=dev)
     st = qkv.struct()
-    _check(lib().sage_attn_fwd(ctypes.byref(st), ctypes.byref(s), int(mask), int(mask_block),
-                               _ptr(out), _ptr(o_f32), _ptr(lse), _stream(stream)),
-           "sage_attn_fwd")
+    if block_mask is None:
+        _check(lib().sage_attn_fwd(ctypes.byref(st), ctypes.byref(s), int(mask), int(mask_block),
+                                   _ptr(out), _ptr(o_f32), _ptr(lse), _stream(stream)),
+               "sage_attn_fwd")
+        return out
+    if (block_mask.dtype != torch.uint8 or not block_mask.is_cuda
+            or not block_mask.is_contiguous()
+            or tuple(block_mask.shape) != block_mask_shape(s.B, s.H, s.Nq, s.Nkv)):
+        raise ValueError("block_mask must be a contiguous uint8 CUDA tensor of shape %s"
+                         % (block_mask_shape(s.B, s.H, s.Nq, s.Nkv),))
+    _check(lib().sage_attn_fwd_block_sparse(ctypes.byref(st), ctypes.byref(s), int(mask),
+                                            int(mask_block), _ptr(block_mask), _ptr(out),
+                                            _ptr(o_f32), _ptr(lse), _stream(stream)),
+           "sage_attn_fwd_block_sparse")
     return out
 
 

@@ -233,9 +233,10 @@ SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, co
                                                                            : SAGE_ERR_CUDA;
 }
 
-SAGE_EXPORT sage_status sage_attn_fwd(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
-                                      int mask_block, void* o_bf16, float* o_f32, float* lse,
-                                      void* stream) {
+namespace {
+sage_status attn_common(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
+                        int mask_block, const uint8_t* block_mask, void* o_bf16, float* o_f32,
+                        float* lse, void* stream) {
   if (!shape_ok(shape) || !qkv_ok(qkv) || !aligned16(o_bf16)) return SAGE_ERR_INVALID_ARG;
   if (o_f32 && !aligned16(o_f32)) return SAGE_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SAGE_ERR_INVALID_ARG;
@@ -252,8 +253,28 @@ SAGE_EXPORT sage_status sage_attn_fwd(const sage_qkv_quant* qkv, const sage_shap
   p.o = static_cast<__nv_bfloat16*>(o_bf16);
   p.o_f32 = o_f32;
   p.lse = lse;
+  p.bmask = block_mask;
+  p.n_qt = (shape->Nq + kAttnBM - 1) / kAttnBM;
+  p.n_kt = (shape->Nkv + kAttnBN - 1) / kAttnBN;
   return launch_attn(maps, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
                                                                                 : SAGE_ERR_CUDA;
+}
+}  // namespace
+
+SAGE_EXPORT sage_status sage_attn_fwd(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
+                                      int mask_block, void* o_bf16, float* o_f32, float* lse,
+                                      void* stream) {
+  return attn_common(qkv, shape, mask, mask_block, nullptr, o_bf16, o_f32, lse, stream);
+}
+
+SAGE_EXPORT sage_status sage_attn_fwd_block_sparse(const sage_qkv_quant* qkv,
+                                                   const sage_shape* shape, int mask,
+                                                   int mask_block, const uint8_t* block_mask,
+                                                   void* o_bf16, float* o_f32, float* lse,
+                                                   void* stream) {
+  if (!block_mask || !shape_ok(shape)) return SAGE_ERR_INVALID_ARG;
+  if ((shape->Nkv + kAttnBN - 1) / kAttnBN > kAttnMaxKvTiles) return SAGE_ERR_UNSUPPORTED;
+  return attn_common(qkv, shape, mask, mask_block, block_mask, o_bf16, o_f32, lse, stream);
 }
 
 SAGE_EXPORT sage_status sage_debug_qk_int32(const sage_qkv_quant* qkv, const sage_shape* shape,

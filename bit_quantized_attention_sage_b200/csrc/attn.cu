@@ -49,6 +49,7 @@ constexpr int BN = kAttnBN;
 constexpr int NS = 2;              // K/V pipeline stages
 constexpr int kThreads = 192;      // 6 warps
 constexpr int kTmemCols = 256;
+constexpr int kMaxTileWords = kAttnMaxKvTiles / 32;  // block-sparse tile bitmap
 constexpr uint32_t kFull = 0xffffffffu;
 // The S accumulator is seeded with the bit pattern of 1.5 * 2^23; for
 // |S| < 2^22 the int32 sum 0x4B400000 + S reads as the fp32 value
@@ -75,6 +76,8 @@ struct alignas(1024) Smem {
   uint64_t s_full, s_free, p_full, o_ready, drain;
   uint32_t tmem_base;
   int abort;
+  // block-sparse mode: bit t set = KV tile t is visited by this CTA
+  uint32_t tile_bits[kMaxTileWords];
 };
 
 // Exactly the struct: two D = 128 CTAs fill the SM's 228 KB (2 x (113 KB +
@@ -115,7 +118,29 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
   }
 }
 
-template <int D, bool DUMP>
+// The KV tiles a CTA visits, in ascending order: kt0, kt0 + 1, ... (dense) or
+// the set bits of the CTA's tile bitmap (block-sparse).  next() must be
+// called at most as many times as there are tiles.
+template <bool SPARSE>
+struct TileSeq {
+  const uint32_t* bits;
+  int w;
+  uint32_t cur;
+  __device__ __forceinline__ TileSeq(const uint32_t* b, int kt0)
+      : bits(b), w(SPARSE ? 0 : kt0), cur(SPARSE ? b[0] : 0u) {}
+  __device__ __forceinline__ int next() {
+    if constexpr (!SPARSE) {
+      return w++;
+    } else {
+      while (cur == 0u) cur = bits[++w];
+      const int t = w * 32 + __ffs(static_cast<int>(cur)) - 1;
+      cur &= cur - 1u;
+      return t;
+    }
+  }
+};
+
+template <int D, bool DUMP, bool SPARSE>
 __device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int bh, int qt,
                                          int kt0, int nk, const WaitCtx& w) {
   tma_prefetch_desc(&maps.q);
@@ -124,10 +149,11 @@ __device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int b
   mbar_arrive_expect_tx(&s.q_full, BM * D);
   tma_load_3d(s.q, &maps.q, &s.q_full, 0, qt * BM, bh);
   int k_issued = 0, v_issued = 0;
+  TileSeq<SPARSE> seq(s.tile_bits, kt0);
   for (int it = 0; it < nk; it++) {
     const int st = it % NS;
     const uint32_t ph = (it / NS) & 1;
-    const int kt = kt0 + it;
+    const int kt = seq.next();
     if (it >= NS && !mbar_wait(&s.k_empty[st], ph ^ 1, w, kSiteProdKEmpty)) break;
     mbar_arrive_expect_tx(&s.k_full[st], BN * D);
     tma_load_3d(s.k[st], &maps.k, &s.k_full[st], 0, kt * BN, bh);
@@ -231,7 +257,7 @@ __device__ __forceinline__ void rescale_row(uint32_t tO, float alpha) {
 }
 
 // Softmax / correction / epilogue for one query row per thread.
-template <int D>
+template <int D, bool SPARSE>
 __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
                                              uint32_t tmem_O, int bh, int qt, int nk,
                                              const WaitCtx& w) {
@@ -248,7 +274,10 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   const float* ksc = p.k_scale + static_cast<size_t>(bh) * p.nkv_blocks;
   uint8_t* prow0 = s.p[0] + r * BN;
 
-  float ks0 = k_block_scale(ksc, 0, p.nkv_blocks), ks1 = k_block_scale(ksc, 1, p.nkv_blocks);
+  TileSeq<SPARSE> seq(s.tile_bits, 0);
+  int kt = (SPARSE && nk > 0) ? seq.next() : 0;  // KV tile of this iteration (sparse)
+  float ks0 = k_block_scale(ksc, 2 * kt, p.nkv_blocks);
+  float ks1 = k_block_scale(ksc, 2 * kt + 1, p.nkv_blocks);
   float m = -INFINITY, l = 0.0f;
   bool ok = true;
   // seed the S row for the first tile (the MMA issuer waits for it)
@@ -258,7 +287,8 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   __syncwarp();
   if (lane == 0) mbar_arrive(&s.s_free);
   for (int it = 0; it < nk; it++) {
-    const int j0 = it * BN;
+    if constexpr (!SPARSE) kt = it;
+    const int j0 = kt * BN;
     if (!warp_wait(&s.s_full, it & 1, w, kSiteSmS)) { ok = false; break; }
     tc_fence_after();
     uint32_t sv[128];  // 0x4B400000 + S: the fp32 value 1.5 * 2^23 + S
@@ -269,8 +299,9 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     // scale of each 64-key group of the tile; the next tile's K scales are
     // loaded now so that their latency is hidden behind this tile
     const float c0 = __fmul_rn(sqC, ks0), c1 = __fmul_rn(sqC, ks1);
-    ks0 = k_block_scale(ksc, 2 * it + 2, p.nkv_blocks);
-    ks1 = k_block_scale(ksc, 2 * it + 3, p.nkv_blocks);
+    const int kt_next = (SPARSE && more) ? seq.next() : kt + 1;
+    ks0 = k_block_scale(ksc, 2 * kt_next, p.nkv_blocks);
+    ks1 = k_block_scale(ksc, 2 * kt_next + 1, p.nkv_blocks);
     const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
     const bool full = __all_sync(kFull, nvis == BN);
 
@@ -360,17 +391,35 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     if (it > 0 && __any_sync(kFull, alpha != 1.0f)) rescale_row<D>(tO, alpha);
     l = __fadd_rn(__fmul_rn(l, alpha), rs);
     m = m_new;
+    kt = kt_next;
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.p_full);
   }
 
-  if (!ok || nk == 0) return;
-  if (!warp_wait(&s.o_ready, (nk - 1) & 1, w, kSiteSmEpi)) return;
-  tc_fence_after();
-  const float inv = __frcp_rn(l);  // l is in units of 2^8 p
+  if (!ok) return;
   const float* vsc = p.v_scale + static_cast<size_t>(bh) * D;
   const size_t orow = (static_cast<size_t>(bh) * p.Nq + (valid ? i : 0)) * D;
+  if (nk == 0) {  // block-sparse: no tile at all for this CTA; O = 0, lse = -inf
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(p.o + orow);
+#pragma unroll 1
+      for (int e = 0; e < D / 8; e++) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      if (p.o_f32) {
+        float4* d32 = reinterpret_cast<float4*>(p.o_f32 + orow);
+#pragma unroll 1
+        for (int e = 0; e < D / 4; e++) d32[e] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+      if (p.lse) p.lse[static_cast<size_t>(bh) * p.Nq + i] = -INFINITY;
+    }
+    return;
+  }
+  if (!warp_wait(&s.o_ready, (nk - 1) & 1, w, kSiteSmEpi)) return;
+  tc_fence_after();
+  // a row that saw no key (possible only with a block mask) has l = 0:
+  // O = 0 (its O_acc row is 0) and lse = -inf
+  const bool seen = l > 0.0f;
+  const float inv = seen ? __frcp_rn(l) : 0.0f;  // l is in units of 2^8 p
 #pragma unroll 1
   for (int c = 0; c < D; c += 32) {
     uint32_t o[32];
@@ -395,7 +444,8 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     }
   }
   if (valid && p.lse)
-    p.lse[static_cast<size_t>(bh) * p.Nq + i] = (m + log2f(l) - 8.0f) * 0.69314718055994531f;
+    p.lse[static_cast<size_t>(bh) * p.Nq + i] =
+        seen ? (m + log2f(l) - 8.0f) * 0.69314718055994531f : -INFINITY;
 }
 
 // Score dump (debug): copy the int32 S tile from TMEM to global memory.
@@ -421,7 +471,7 @@ __device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint3
   if (lane == 0) mbar_arrive(&s.s_free);
 }
 
-template <int D, bool DUMP>
+template <int D, bool DUMP, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 2)
     k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -447,6 +497,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int last = min(p.Nq - 1, qt * BM + BM - 1);
     nk = (row_limit(last, p) + BN - 1) / BN;
   }
+  if constexpr (SPARSE) {
+    // bitmap of the tiles below nk that the block mask switches on (one
+    // ballot per 32 tiles); nk becomes their count after the barrier below
+    const uint8_t* row = p.bmask + (static_cast<size_t>(bh) * p.n_qt + qt) * p.n_kt;
+    const int nwords = (nk + 31) / 32;
+    for (int wd = warp; wd < nwords; wd += kThreads / 32) {
+      const int t = wd * 32 + lane;
+      const uint32_t b = __ballot_sync(kFull, t < nk && row[t] != 0);
+      if (lane == 0) s.tile_bits[wd] = b;
+    }
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
@@ -471,18 +532,24 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if constexpr (SPARSE) {
+    const int nwords = (nk + 31) / 32;
+    int cnt = 0;
+    for (int wd = 0; wd < nwords; wd++) cnt += __popc(s.tile_bits[wd]);
+    nk = cnt;
+  }
   const uint32_t tmem = s.tmem_base;
   const uint32_t tmem_S = tmem;        // columns [0, 128): int32 scores
   const uint32_t tmem_O = tmem + 128;  // columns [128, 128 + D): fp32 output
   const WaitCtx w{p.budget, p.status, &s.abort};
 
   if (warp == 0) {
-    if (lane == 0) producer<D, DUMP>(s, maps, bh, qt, kt0, nk, w);
+    if (lane == 0) producer<D, DUMP, SPARSE>(s, maps, bh, qt, kt0, nk, w);
   } else if (warp == 1) {
     if (lane == 0) mma_issuer<D, DUMP>(s, tmem_S, tmem_O, nk, w);
   } else {
     if (DUMP) dump_rows<D>(s, p, tmem_S, w);
-    else softmax_rows<D>(s, p, tmem_S, tmem_O, bh, qt, nk, w);
+    else softmax_rows<D, SPARSE>(s, p, tmem_S, tmem_O, bh, qt, nk, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -497,38 +564,46 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 size_t attn_smem_bytes(int D) { return smem_bytes_for(D); }
 
+namespace {
+template <int D, bool DUMP, bool SPARSE>
+cudaError_t prepare_one() {
+  return cudaFuncSetAttribute(k_attn<D, DUMP, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(smem_bytes_for(D)));
+}
+}  // namespace
+
 cudaError_t attn_prepare(int D) {
   cudaError_t e;
   if (D == 128) {
-    e = cudaFuncSetAttribute(k_attn<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes_for(128)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_attn<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes_for(128)));
+    e = prepare_one<128, false, false>();
+    if (e == cudaSuccess) e = prepare_one<128, true, false>();
+    if (e == cudaSuccess) e = prepare_one<128, false, true>();
   } else {
-    e = cudaFuncSetAttribute(k_attn<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes_for(64)));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_attn<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_bytes_for(64)));
+    e = prepare_one<64, false, false>();
+    if (e == cudaSuccess) e = prepare_one<64, true, false>();
+    if (e == cudaSuccess) e = prepare_one<64, false, true>();
   }
   return e;
 }
 
 cudaError_t launch_attn(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
   dim3 grid((p.Nq + BM - 1) / BM, p.BH);
-  if (p.D == 128)
-    k_attn<128, false><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
-  else
-    k_attn<64, false><<<grid, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+  const bool sparse = p.bmask != nullptr;
+  if (p.D == 128) {
+    if (sparse) k_attn<128, false, true><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
+    else k_attn<128, false, false><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
+  } else {
+    if (sparse) k_attn<64, false, true><<<grid, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+    else k_attn<64, false, false><<<grid, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_dump(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
   if (p.D == 128)
-    k_attn<128, true><<<1, kThreads, smem_bytes_for(128), stream>>>(maps, p);
+    k_attn<128, true, false><<<1, kThreads, smem_bytes_for(128), stream>>>(maps, p);
   else
-    k_attn<64, true><<<1, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+    k_attn<64, true, false><<<1, kThreads, smem_bytes_for(64), stream>>>(maps, p);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,8 @@ namespace sage {
 
 constexpr int kAttnBM = 128;  // query rows per CTA (tcgen05 M)
 constexpr int kAttnBN = 128;  // keys per KV tile
+// block-sparse mode: at most this many KV tiles (786432 keys) per head
+constexpr int kAttnMaxKvTiles = 6144;
 
 struct AttnParams {
   int BH, Nq, Nkv, D;
@@ -26,6 +28,10 @@ struct AttnParams {
   float c0;                   // fp32(log2(e) / sqrt(D))
   long long budget;           // per-wait budget, SM cycles
   int* status;                // device status word pair
+  // block-sparse mode (null: dense): uint8 [BH][n_qt][n_kt], tile (qt, kt)
+  // visited only if non-zero
+  const uint8_t* bmask;
+  int n_qt, n_kt;
   // score-dump mode (debug): a single tile (bh, qt, kt), int32 [128, 128]
   int dbg_bh, dbg_qt, dbg_kt;
   int32_t* dbg_out;

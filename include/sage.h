@@ -191,6 +191,26 @@ sage_status sage_quant_qk_noalloc(const void *q_bf16, const void *k_bf16, const 
 sage_status sage_attn_fwd(const sage_qkv_quant *qkv, const sage_shape *shape, int mask,
                           int mask_block, void *o_bf16, float *o_f32, float *lse, void *stream);
 
+/* sage_attn_fwd with block-sparse skipping: tiles of 128 query rows x 128
+ * keys that `block_mask` switches off are not computed (neither Q K^T nor
+ * P V nor the softmax visits them).  This is the skipping that the sparse
+ * layers stacked on quantized attention rely on (TurboDiffusion notes,
+ * hybrid-attention bullet: SageAttention combined with sparse-linear
+ * attention); how the mask is predicted is not given by the pages and is
+ * the caller's business.
+ *   block_mask  device uint8 [B, H, ceil(Nq/128), ceil(Nkv/128)], row-major;
+ *               key j is visible to query i iff `mask` allows it AND
+ *               block_mask[b][h][i/128][j/128] != 0.  Read only.
+ * The tile order of the online softmax is unchanged (ascending over the
+ * visited tiles), so an all-ones mask gives exactly sage_attn_fwd's result.
+ * A query row that sees no key at all gets O = 0 (bf16 and f32) and
+ * lse = -inf.
+ * Errors: as sage_attn_fwd, plus SAGE_ERR_INVALID_ARG for a NULL block_mask
+ * and SAGE_ERR_UNSUPPORTED for more than 6144 KV tiles (786432 keys). */
+sage_status sage_attn_fwd_block_sparse(const sage_qkv_quant *qkv, const sage_shape *shape,
+                                       int mask, int mask_block, const uint8_t *block_mask,
+                                       void *o_bf16, float *o_f32, float *lse, void *stream);
+
 /* Debug: run the attention kernel's load + INT8 MMA path on selected tiles
  * and copy the int32 score tile it leaves in tensor memory to `out`.
  *   tiles  host int array of n_tiles triples (bh, qt, kt): head index b*H+h,

@@ -17,14 +17,17 @@ def to_dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def run(q, k, v, mask=0, mb=0):
-    """Quantize + attend on the GPU.  Returns (qkv, o_bf16, o_f32, lse) on device."""
+def run(q, k, v, mask=0, mb=0, block_mask=None):
+    """Quantize + attend on the GPU (block-sparse when `block_mask`, a numpy
+    uint8 [B, H, n_qt, n_kt], is given).  Returns (qkv, o_bf16, o_f32, lse)."""
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     B, H, Nq, D = q.shape
     qkv = sage.quant_qk(qd, kd, vd)
     o_f32 = torch.empty((B, H, Nq, D), dtype=torch.float32, device="cuda")
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
-    o = sage.attn_fwd(qkv, mask, mb, o_f32=o_f32, lse=lse)
+    bm = None if block_mask is None else torch.from_numpy(
+        np.ascontiguousarray(block_mask, np.uint8)).cuda()
+    o = sage.attn_fwd(qkv, mask, mb, o_f32=o_f32, lse=lse, block_mask=bm)
     st = sage.sync_status()
     assert st == 0, "device status %d" % st
     return qkv, o, o_f32, lse
@@ -55,9 +58,10 @@ def bf16_half_ulp(x):
     return 0.5 * 2.0 ** (e - 7)
 
 
-def check_rows(ref_head, rows, o_bf16_rows, o_f32_rows, lse_rows, mask, mb):
-    """O and lse of the given rows against the oracle (same quantized inputs)."""
-    o_ref, slack, lse_ref = oracle.attn_rows(ref_head, rows, mask, mb)
+def check_rows(ref_head, rows, o_bf16_rows, o_f32_rows, lse_rows, mask, mb, block_mask=None):
+    """O and lse of the given rows against the oracle (same quantized inputs;
+    `block_mask`: this head's [n_qt, n_kt] tile mask, if any)."""
+    o_ref, slack, lse_ref = oracle.attn_rows(ref_head, rows, mask, mb, block_mask=block_mask)
     tol = O_ATOL + slack
     err32 = np.abs(o_f32_rows.astype(np.float64) - o_ref)
     bad = err32 > tol
@@ -66,7 +70,10 @@ def check_rows(ref_head, rows, o_bf16_rows, o_f32_rows, lse_rows, mask, mb):
     errb = np.abs(o_bf16_rows.astype(np.float64) - o_ref)
     tolb = tol + bf16_half_ulp(o_ref)
     assert not (errb > tolb).any(), "bf16 O out of tolerance"
-    assert np.abs(lse_rows.astype(np.float64) - lse_ref).max() <= LSE_ATOL
+    empty = np.isneginf(lse_ref)  # rows that see no key (block masks only)
+    assert np.all(np.isneginf(lse_rows[empty])), "lse of rows without keys is not -inf"
+    assert np.abs(lse_rows[~empty].astype(np.float64) - lse_ref[~empty]).max(initial=0.0) \
+        <= LSE_ATOL
     return o_ref, slack
 
 
