@@ -51,6 +51,10 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="time the 72-point sweep (N x D x mask x K outlier magnitude) and report "
                          "TOPS and accuracy against fp64 attention per point, one JSON line each")
+    ap.add_argument("--block-density", type=float, default=None,
+                    help="time sage_attn_fwd_block_sparse on the workload with a seeded random "
+                         "128x128 tile mask of this density (one JSON line; TOPS over the "
+                         "visible pairs of the enabled tiles)")
     ap.add_argument("--sweep-filter", default="",
                     help="only sweep points whose name contains this string")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -476,6 +480,70 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+# ------------------------------------------------------------------ block-sparse
+
+def block_sparse_pairs(w, bm):
+    """Visible (query, key) pairs of one head under the row mask and the
+    tile mask bm [n_qt, n_kt] (the algorithmic work of the sparse call)."""
+    g = np.arange(w.Nq, dtype=np.int64) + (w.Nkv - w.Nq)
+    if w.mask == 1:
+        lim = g + 1
+    elif w.mask == 2:
+        lim = (g // w.mask_block + 1) * w.mask_block
+    else:
+        lim = np.full(w.Nq, w.Nkv, np.int64)
+    lim = np.minimum(lim, w.Nkv)
+    total = 0
+    starts = np.arange(bm.shape[1], dtype=np.int64) * 128
+    for qt in range(bm.shape[0]):
+        li = lim[qt * 128:(qt + 1) * 128]
+        on = starts[bm[qt] != 0]
+        total += int(np.clip(li[:, None] - on[None, :], 0, 128).sum())
+    return total
+
+
+def run_block_sparse(args):
+    import torch
+    import bit_quantized_attention_sage_b200 as sage
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    sage.lib()
+    w = synth.WORKLOADS[args.workload]
+    runner = Runner(w, 0, device)
+    rng = np.random.default_rng(7)
+    shape = sage.block_mask_shape(w.B, w.H, w.Nq, w.Nkv)
+    bm_h = (rng.random(shape) < args.block_density).astype(np.uint8)
+    bm = torch.from_numpy(bm_h).to(device)
+    pairs = sum(block_sparse_pairs(w, bm_h[b, h]) for b in range(w.B) for h in range(w.H))
+    sage.quant_qk(runner.q, runner.k, runner.v, out=runner.qkv, workspace=runner.ws)
+
+    def timed(block_mask):
+        for _ in range(args.warmup):
+            sage.attn_fwd(runner.qkv, w.mask, w.mask_block, out=runner.o, block_mask=block_mask)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            sage.attn_fwd(runner.qkv, w.mask, w.mask_block, out=runner.o, block_mask=block_mask)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    t_sparse, t_dense = timed(bm), timed(None)
+    if sage.sync_status() != 0:
+        raise RuntimeError("device status error in the block-sparse run")
+    ops = 4 * w.D * pairs
+    print(json.dumps({
+        "block_sparse": w.name, "density": args.block_density,
+        "enabled_tile_fraction": round(float(bm_h.mean()), 4),
+        "visible_pair_fraction": round(pairs / (w.B * w.H * w.visible_pairs()), 4),
+        "attn_ms": round(t_sparse, 4), "dense_attn_ms": round(t_dense, 4),
+        "speedup_vs_dense": round(t_dense / t_sparse, 3),
+        "TOPS": round(ops / (t_sparse / 1e3) / 1e12, 2),
+        "attn_frac_of_peak": round(ops / (t_sparse / 1e3) / 1e12 / peaks()["i8_sustained"], 4)}),
+        flush=True)
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args):
@@ -513,6 +581,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.block_density is not None:
+        run_block_sparse(args)
     else:
         run_ours(args)
 
