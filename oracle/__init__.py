@@ -64,6 +64,12 @@ def lib():
         L.orc_attn_rows_identity_bs.restype = i32
         L.orc_attn_rows_identity_bs.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
                                                 P, i64, i64, P, i64, P, P, i32]
+        L.orc_w8a8_quant_act.restype = i32
+        L.orc_w8a8_quant_act.argtypes = [P, i64, i64, P, P]
+        L.orc_w8a8_quant_weight.restype = i32
+        L.orc_w8a8_quant_weight.argtypes = [P, i64, i64, P, P]
+        L.orc_w8a8_gemm_rows.restype = i32
+        L.orc_w8a8_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, i32]
         L.orc_attn_fp64_rows.restype = i32
         L.orc_attn_fp64_rows.argtypes = [P, P, P, i64, i64, i32, i32, i64, P, i64, P, i32]
         _lib = L
@@ -234,3 +240,47 @@ def accuracy(o, ref):
 def c0(D):
     """fp32(log2(e)/sqrt(D)) as the recipe defines it (for tests)."""
     return np.float32(math.log2(math.e) / math.sqrt(D))
+
+
+# ---------------------------------------------------------------- W8A8 linear layer
+
+W8A8_G = 128  # channels per quantization group along K
+
+
+def w8a8_quant_act(x):
+    """X [M, K] bf16 bits -> (xq [M, K] int8, sx [M, K/128] f32): one scale
+    per token and 128-channel group."""
+    x = np.ascontiguousarray(x, np.uint16)
+    M, K = x.shape
+    xq = np.empty((M, K), np.int8)
+    sx = np.empty((M, K // W8A8_G), np.float32)
+    if lib().orc_w8a8_quant_act(_p(x), M, K, _p(xq), _p(sx)):
+        raise ValueError("orc_w8a8_quant_act: K must be a multiple of 128")
+    return xq, sx
+
+
+def w8a8_quant_weight(w):
+    """W [N, K] bf16 bits -> (wq [N, K] int8, sw [N/128, K/128] f32): one
+    scale per 128 x 128 block."""
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    wq = np.empty((N, K), np.int8)
+    sw = np.empty((N // W8A8_G, K // W8A8_G), np.float32)
+    if lib().orc_w8a8_quant_weight(_p(w), N, K, _p(wq), _p(sw)):
+        raise ValueError("orc_w8a8_quant_weight: N and K must be multiples of 128")
+    return wq, sw
+
+
+def w8a8_gemm_rows(xq, sx, wq, sw, rows, threads=None):
+    """Rows of Y = X W^T from the quantized operands (fp32, before the bf16
+    rounding), promoting each 128-channel group's exact integer dot product
+    into an fp32 running sum with one fma, in ascending group order."""
+    xq, sx, wq, sw = (np.ascontiguousarray(a) for a in (xq, sx, wq, sw))
+    rows = np.ascontiguousarray(rows, np.int64)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = np.empty((rows.size, N), np.float32)
+    if lib().orc_w8a8_gemm_rows(_p(xq), _p(sx), _p(wq), _p(sw), M, N, K, _p(rows), rows.size,
+                                _p(y), _threads(threads)):
+        raise ValueError("orc_w8a8_gemm_rows: invalid arguments")
+    return y

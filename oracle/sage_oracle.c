@@ -38,6 +38,12 @@
  *                              row and block mask to 1e-12; an all-ones mask
  *                              reproduces the dense result bit for bit; rows
  *                              that see no key give O = 0, lse = -inf.
+ *   orc_w8a8_quant_act / _weight : quantizer invariants (max code 127, half-
+ *                              step reconstruction, zero groups, RNE ties,
+ *                              block shapes).
+ *   orc_w8a8_gemm_rows       : exact integer product on unit scales (numpy
+ *                              int64), fp64 blockwise definition within the
+ *                              fp32 accumulation bound.
  */
 #include <math.h>
 #include <pthread.h>
@@ -700,5 +706,135 @@ int orc_attn_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         return 1;
     fp64_job J = {q, k, v, nq, nkv, D, mask, mb, rows, o};
     for_rows(&J, fp64_row, nrows, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-block W8A8 linear layer (Y = X W^T with INT8 operands)          */
+/* ------------------------------------------------------------------ */
+/* The pages quantize the linear layers to 8-bit weights and activations
+ * per block, on INT8 tensor cores, because per-tensor and per-channel
+ * scales are stretched by outliers (Vidu S1 digest, "Infra"; TurboDiffusion
+ * notes, W8A8 bullet).  Readings taken here: blocks are 128 channels wide
+ * along the reduction dimension K; an activation block is one token x 128
+ * channels, a weight block 128 output channels x 128 channels; both are
+ * symmetric absmax/127 with round-half-to-even, as the attention quantizer.
+ * Each 128-channel group is reduced exactly in integers and promoted into an
+ * fp32 running sum, group by group in ascending order:
+ *   y = fmaf((float)P_g, fp32(sx[m,g] * sw[n/128,g]), y),
+ * and Y is y rounded to bf16 (round-half-to-even). */
+
+#define ORC_W8A8_G 128
+
+static void quant_group_i8(const float *x, long n, int8_t *q, float *scale)
+{
+    float a = 0.0f;
+    for (long i = 0; i < n; i++) {
+        float t = fabsf(x[i]);
+        if (t > a)
+            a = t;
+    }
+    if (a == 0.0f) {
+        *scale = 0.0f;
+        memset(q, 0, (size_t)n);
+        return;
+    }
+    *scale = a / 127.0f;
+    float inv = 127.0f / a;
+    for (long i = 0; i < n; i++) {
+        float t = nearbyintf(x[i] * inv);
+        if (t > 127.0f)
+            t = 127.0f;
+        if (t < -127.0f)
+            t = -127.0f;
+        q[i] = (int8_t)t;
+    }
+}
+
+/* X [M, K] bf16 bits, K a multiple of 128 -> xq [M, K] int8, sx [M, K/128]. */
+int orc_w8a8_quant_act(const uint16_t *x, long M, long K, int8_t *xq, float *sx)
+{
+    if (M <= 0 || K <= 0 || K % ORC_W8A8_G)
+        return 1;
+    const long G = K / ORC_W8A8_G;
+    float buf[ORC_W8A8_G];
+    for (long m = 0; m < M; m++)
+        for (long g = 0; g < G; g++) {
+            for (int c = 0; c < ORC_W8A8_G; c++)
+                buf[c] = bf16_to_f32(x[m * K + g * ORC_W8A8_G + c]);
+            quant_group_i8(buf, ORC_W8A8_G, xq + m * K + g * ORC_W8A8_G, sx + m * G + g);
+        }
+    return 0;
+}
+
+/* W [N, K] bf16 bits, N and K multiples of 128 -> wq [N, K] int8,
+ * sw [N/128, K/128] (one scale per 128 x 128 block). */
+int orc_w8a8_quant_weight(const uint16_t *w, long N, long K, int8_t *wq, float *sw)
+{
+    if (N <= 0 || K <= 0 || N % ORC_W8A8_G || K % ORC_W8A8_G)
+        return 1;
+    const long G = K / ORC_W8A8_G, NB = N / ORC_W8A8_G;
+    float *blk = (float *)malloc(sizeof(float) * ORC_W8A8_G * ORC_W8A8_G);
+    int8_t *qb = (int8_t *)malloc(ORC_W8A8_G * ORC_W8A8_G);
+    if (!blk || !qb) {
+        free(blk);
+        free(qb);
+        return 1;
+    }
+    for (long nb = 0; nb < NB; nb++)
+        for (long g = 0; g < G; g++) {
+            for (int r = 0; r < ORC_W8A8_G; r++)
+                for (int c = 0; c < ORC_W8A8_G; c++)
+                    blk[r * ORC_W8A8_G + c] =
+                        bf16_to_f32(w[(nb * ORC_W8A8_G + r) * K + g * ORC_W8A8_G + c]);
+            quant_group_i8(blk, (long)ORC_W8A8_G * ORC_W8A8_G, qb, sw + nb * G + g);
+            for (int r = 0; r < ORC_W8A8_G; r++)
+                memcpy(wq + (nb * ORC_W8A8_G + r) * K + g * ORC_W8A8_G, qb + r * ORC_W8A8_G,
+                       ORC_W8A8_G);
+        }
+    free(blk);
+    free(qb);
+    return 0;
+}
+
+typedef struct {
+    const int8_t *xq, *wq;
+    const float *sx, *sw;
+    long N, K;
+    const long *rows;
+    float *y;
+} w8a8_job;
+
+static void w8a8_row(const void *job, long r)
+{
+    const w8a8_job *J = (const w8a8_job *)job;
+    const long m = J->rows[r], K = J->K, G = K / ORC_W8A8_G;
+    for (long n = 0; n < J->N; n++) {
+        float y = 0.0f;
+        for (long g = 0; g < G; g++) {
+            int64_t p = 0;
+            for (int c = 0; c < ORC_W8A8_G; c++)
+                p += (int64_t)J->xq[m * K + g * ORC_W8A8_G + c] *
+                     (int64_t)J->wq[n * K + g * ORC_W8A8_G + c];
+            const float s = J->sx[m * G + g] * J->sw[(n / ORC_W8A8_G) * G + g];
+            y = fmaf((float)p, s, y);
+        }
+        J->y[r * J->N + n] = y;
+    }
+}
+
+/* Rows `rows` of Y = (dequantized X)(dequantized W)^T by the promotion rule
+ * above: y [nrows, N] fp32 (round to bf16 for the layer's output). */
+int orc_w8a8_gemm_rows(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                       long M, long N, long K, const long *rows, long nrows, float *y,
+                       int nthreads)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || K % ORC_W8A8_G || N % ORC_W8A8_G)
+        return 1;
+    for (long r = 0; r < nrows; r++)
+        if (rows[r] < 0 || rows[r] >= M)
+            return 1;
+    w8a8_job J = {xq, wq, sx, sw, N, K, rows, y};
+    for_rows(&J, w8a8_row, nrows, nthreads);
     return 0;
 }
