@@ -77,6 +77,13 @@ def lib():
         L.sage_debug_e4m3.argtypes = [P, P, SZ, P]
         L.sage_debug_exp2.restype = I
         L.sage_debug_exp2.argtypes = [P, P, SZ, P]
+        LL = ctypes.c_longlong
+        L.sage_w8a8_quant_act.restype = I
+        L.sage_w8a8_quant_act.argtypes = [P, LL, LL, P, P, P]
+        L.sage_w8a8_quant_weight.restype = I
+        L.sage_w8a8_quant_weight.argtypes = [P, LL, LL, P, P, P]
+        L.sage_w8a8_gemm.restype = I
+        L.sage_w8a8_gemm.argtypes = [P, P, P, P, LL, LL, LL, P, P, P]
         L.sage_sync_status.restype = I
         L.sage_sync_status.argtypes = [P]
         _lib = L
@@ -273,3 +280,55 @@ def timeout_probe(budget_cycles, stream=None):
 def sync_status(stream=None):
     """Synchronize the stream and return (and clear) the device status code."""
     return int(lib().sage_sync_status(_stream(stream)))
+
+
+# ---------------------------------------------------------------- W8A8 linear layer
+
+W8A8_GROUP = 128
+
+
+def w8a8_quant_act(x, xq=None, sx=None, stream=None):
+    """X bf16 [M, K] (CUDA, contiguous) -> (xq int8 [M, K], sx f32 [M, K/128])."""
+    import torch
+    M, K = x.shape
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    sx = torch.empty((M, K // W8A8_GROUP), dtype=torch.float32, device=x.device) if sx is None else sx
+    _check(lib().sage_w8a8_quant_act(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)),
+           "sage_w8a8_quant_act")
+    return xq, sx
+
+
+def w8a8_quant_weight(w, stream=None):
+    """W bf16 [N, K] (CUDA, contiguous) -> (wq int8 [N, K], sw f32 [N/128, K/128])."""
+    import torch
+    N, K = w.shape
+    if w.dtype != torch.bfloat16 or not w.is_cuda or not w.is_contiguous():
+        raise ValueError("w must be a contiguous bf16 CUDA tensor")
+    wq = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    sw = torch.empty((N // W8A8_GROUP, K // W8A8_GROUP), dtype=torch.float32, device=w.device)
+    _check(lib().sage_w8a8_quant_weight(_ptr(w), N, K, _ptr(wq), _ptr(sw), _stream(stream)),
+           "sage_w8a8_quant_weight")
+    return wq, sw
+
+
+def w8a8_gemm(xq, sx, wq, sw, out=None, y_f32=None, stream=None):
+    """Y bf16 [M, N] = dequant(X) dequant(W)^T from the quantized operands."""
+    import torch
+    M, K = xq.shape
+    N = wq.shape[0]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    _check(lib().sage_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(out),
+                                _ptr(y_f32), _stream(stream)), "sage_w8a8_gemm")
+    return out
+
+
+def linear_w8a8(x, wq, sw, stream=None):
+    """A W8A8 linear layer on bf16 activations [..., K] with pre-quantized
+    weights (from w8a8_quant_weight): quantize X per token and 128-channel
+    group, then the INT8 GEMM; returns bf16 [..., N]."""
+    lead = x.shape[:-1]
+    x2 = x.reshape(-1, x.shape[-1])
+    xq, sx = w8a8_quant_act(x2.contiguous(), stream=stream)
+    return w8a8_gemm(xq, sx, wq, sw, stream=stream).reshape(*lead, wq.shape[0])

@@ -13,6 +13,7 @@
 #include "attn.cuh"
 #include "quant.cuh"
 #include "sage.h"
+#include "w8a8.cuh"
 #include "sm100.cuh"
 
 #define SAGE_EXPORT extern "C" __attribute__((visibility("default")))
@@ -64,6 +65,7 @@ DeviceState* device_state() {
     d.status = static_cast<int*>(p);
     if (d.init_err == cudaSuccess) d.init_err = attn_prepare(128);
     if (d.init_err == cudaSuccess) d.init_err = attn_prepare(64);
+    if (d.init_err == cudaSuccess) d.init_err = w8a8_prepare();
   });
   if (d.init_err != cudaSuccess) return nullptr;
   return &d;
@@ -180,6 +182,69 @@ __global__ void k_exp2(const float* x, float* y, size_t n) {
 using namespace sage;
 
 SAGE_EXPORT int sage_abi_version(void) { return SAGE_ABI_VERSION; }
+
+// ---------------------------------------------------------------- W8A8 linear layer
+
+namespace {
+bool w8a8_dims_ok(long long M, long long N, long long K) {
+  return M >= 1 && N >= kW8a8BN && K >= kW8a8Group && N % kW8a8BN == 0 && K % kW8a8Group == 0 &&
+         M <= (1ll << 31) - 1 && N <= (1 << 24) && K <= (1 << 24) &&
+         (M + kW8a8BM - 1) / kW8a8BM <= 65535;
+}
+}  // namespace
+
+SAGE_EXPORT sage_status sage_w8a8_quant_act(const void* x_bf16, long long M, long long K,
+                                            int8_t* xq, float* sx, void* stream) {
+  if (!w8a8_dims_ok(M, kW8a8BN, K) || !aligned16(x_bf16) || !aligned16(xq) || !sx ||
+      (reinterpret_cast<uintptr_t>(sx) & 3u))
+    return SAGE_ERR_INVALID_ARG;
+  if (!device_state()) return SAGE_ERR_CUDA;
+  return launch_w8a8_quant_act(static_cast<const uint16_t*>(x_bf16), static_cast<int>(M),
+                               static_cast<int>(K), xq, sx,
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SAGE_OK
+             : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_w8a8_quant_weight(const void* w_bf16, long long N, long long K,
+                                               int8_t* wq, float* sw, void* stream) {
+  if (!w8a8_dims_ok(1, N, K) || !aligned16(w_bf16) || !aligned16(wq) || !sw ||
+      (reinterpret_cast<uintptr_t>(sw) & 3u))
+    return SAGE_ERR_INVALID_ARG;
+  if (!device_state()) return SAGE_ERR_CUDA;
+  return launch_w8a8_quant_weight(static_cast<const uint16_t*>(w_bf16), static_cast<int>(N),
+                                  static_cast<int>(K), wq, sw,
+                                  static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SAGE_OK
+             : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq,
+                                       const float* sw, long long M, long long N, long long K,
+                                       void* y_bf16, float* y_f32, void* stream) {
+  if (!w8a8_dims_ok(M, N, K) || !aligned16(xq) || !aligned16(wq) || !aligned16(y_bf16) || !sx ||
+      !sw || (y_f32 && !aligned16(y_f32)))
+    return SAGE_ERR_INVALID_ARG;
+  DeviceState* d = device_state();
+  if (!d) return SAGE_ERR_CUDA;
+  W8a8Maps maps;
+  if (!encode_u8_3d(&maps.x, xq, K, M, 1, kW8a8Group, kW8a8BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_u8_3d(&maps.w, wq, K, N, 1, kW8a8Group, kW8a8BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SAGE_ERR_CUDA;
+  W8a8Params p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.sx = sx;
+  p.sw = sw;
+  p.y = static_cast<uint16_t*>(y_bf16);
+  p.y_f32 = y_f32;
+  p.budget = kWaitBudget;
+  p.status = d->status;
+  return launch_w8a8_gemm(maps, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SAGE_OK
+             : SAGE_ERR_CUDA;
+}
 
 SAGE_EXPORT const char* sage_status_string(sage_status st) {
   switch (st) {

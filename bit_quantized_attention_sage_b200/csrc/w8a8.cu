@@ -1,0 +1,389 @@
+// w8a8.cu -- per-block W8A8 linear layer on sm_100a: Y = X W^T with INT8
+// activations and weights (the 8-bit block-wise linear-layer quantization of
+// the "Vidu S1" digest, section "Infra", and the TurboDiffusion notes' W8A8
+// bullet: per-block scales because per-tensor and per-channel scales are
+// stretched by outliers; the products run on INT8 tensor cores).
+//
+// Quantization (symmetric absmax/127, round-half-to-even, like the attention
+// quantizer): one activation scale per token and 128-channel group, one
+// weight scale per 128 x 128 block.
+//
+// GEMM: one CTA per 128 x 128 output tile (one weight block wide), 320
+// threads, one CTA per SM:
+//   warp 0      TMA producer: the X and W tiles of each 128-channel group
+//               through a 4-stage shared-memory ring (128-byte swizzle).
+//   warp 1      allocates 512 TMEM columns: four int32 accumulators of
+//               128 x 128, two steps of two groups in flight; one elected thread
+//               issues tcgen05.mma kind::i8 (four K = 32 steps per group)
+//               onto an accumulator seeded with the bit pattern 0x4B400000,
+//               so that the group's exact integer product P reads back as
+//               the fp32 value 1.5 * 2^23 + P.
+//   warps 2-9   promotion: column part c (0-1) of lane quadrant q owns
+//               output rows 32 q .. 32 q + 31 and columns 64 c .. 64 c + 63
+//               (two warps per SM sub-partition).  Per group:
+//               load the 64 scores, re-seed them, release the accumulator,
+//               then y = fma(P, sx * sw, y) in fp32 registers (packed
+//               fp32x2), in ascending group order.  At the end: y -> bf16
+//               (and optional fp32) rows.
+// Every wait is bounded; on a timeout the CTA drains what it issued, frees
+// TMEM and returns.
+#include "w8a8.cuh"
+#include "sm100.cuh"
+
+#include <cuda_bf16.h>
+
+namespace sage {
+
+namespace {
+
+constexpr int G = kW8a8Group;
+constexpr int BM = kW8a8BM;
+constexpr int BN = kW8a8BN;
+constexpr int GPS = 2;           // 128-channel groups per pipeline step
+constexpr int NS = 3;            // shared-memory stages (one step each)
+constexpr int NACC = 4;          // TMEM accumulators (NACC / GPS steps in flight)
+constexpr int NPAIR = NACC / GPS;
+constexpr int kPromWarps = 8;    // two per lane quadrant, 64 columns each
+constexpr int kPromCols = BN / (kPromWarps / 4);
+constexpr int kThreads = 64 + 32 * kPromWarps;  // producer, MMA, promotion
+constexpr int kTmemCols = 512;
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr uint32_t kBiasBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr float kBias = 12582912.0f;
+
+enum : int {
+  kSiteProdEmpty = 0x20101, kSiteMmaFull, kSiteMmaAccFree, kSitePromFull, kSiteDrain,
+  kSiteSmemAlign
+};
+
+// ---------------------------------------------------------------- quantizers
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t q_i8x4(float a, float b, float c, float d, float inv) {
+  auto q1 = [inv](float x) {
+    int q = __float2int_rn(__fmul_rn(x, inv));
+    q = q > 127 ? 127 : (q < -127 ? -127 : q);
+    return static_cast<uint32_t>(static_cast<uint8_t>(static_cast<int8_t>(q)));
+  };
+  return q1(a) | (q1(b) << 8) | (q1(c) << 16) | (q1(d) << 24);
+}
+
+// One (token, 128-channel group) per 16 consecutive threads, 8 channels each.
+__global__ void __launch_bounds__(256) k_w8a8_quant_act(const uint16_t* __restrict__ x, int M,
+                                                         int K, int8_t* __restrict__ xq,
+                                                         float* __restrict__ sx) {
+  const int ngroups = K / G;
+  const long long gid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  const int sub = threadIdx.x & 15;
+  const bool live = gid < static_cast<long long>(M) * ngroups;
+  const long long m = live ? gid / ngroups : 0;
+  const int g = live ? static_cast<int>(gid % ngroups) : 0;
+  const size_t off = static_cast<size_t>(m) * K + static_cast<size_t>(g) * G + sub * 8;
+  uint4 u = make_uint4(0, 0, 0, 0);
+  if (live) u = __ldg(reinterpret_cast<const uint4*>(x + off));
+  const float v[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                      bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+  float a = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; e++) a = fmaxf(a, fabsf(v[e]));
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+  if (!live) return;
+  const float inv = a == 0.0f ? 0.0f : __fdiv_rn(127.0f, a);
+  if (sub == 0) sx[static_cast<size_t>(m) * ngroups + g] = a == 0.0f ? 0.0f : __fdiv_rn(a, 127.0f);
+  *reinterpret_cast<uint2*>(xq + off) =
+      make_uint2(q_i8x4(v[0], v[1], v[2], v[3], inv), q_i8x4(v[4], v[5], v[6], v[7], inv));
+}
+
+// One 128 x 128 weight block per CTA (256 threads, 8 chunks of 8 each).
+__global__ void __launch_bounds__(256) k_w8a8_quant_weight(const uint16_t* __restrict__ w, int N,
+                                                            int K, int8_t* __restrict__ wq,
+                                                            float* __restrict__ sw) {
+  __shared__ float red[8];
+  const int ngroups = K / G;
+  const int g = blockIdx.x, nb = blockIdx.y;
+  constexpr int kChunks = G * G / 8 / 256;  // 8 chunks of 8 channels per thread
+  float v[kChunks][8];
+  float a = 0.0f;
+#pragma unroll
+  for (int c = 0; c < kChunks; c++) {
+    const int chunk = c * 256 + threadIdx.x;
+    const int r = chunk / (G / 8), col = (chunk % (G / 8)) * 8;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(
+        w + static_cast<size_t>(nb * BN + r) * K + static_cast<size_t>(g) * G + col));
+    v[c][0] = bf16_lo(u.x); v[c][1] = bf16_hi(u.x); v[c][2] = bf16_lo(u.y); v[c][3] = bf16_hi(u.y);
+    v[c][4] = bf16_lo(u.z); v[c][5] = bf16_hi(u.z); v[c][6] = bf16_lo(u.w); v[c][7] = bf16_hi(u.w);
+#pragma unroll
+    for (int e = 0; e < 8; e++) a = fmaxf(a, fabsf(v[c][e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; i++) a = fmaxf(a, red[i]);
+  const float inv = a == 0.0f ? 0.0f : __fdiv_rn(127.0f, a);
+  if (threadIdx.x == 0) sw[static_cast<size_t>(nb) * ngroups + g] = a == 0.0f ? 0.0f : __fdiv_rn(a, 127.0f);
+#pragma unroll
+  for (int c = 0; c < kChunks; c++) {
+    const int chunk = c * 256 + threadIdx.x;
+    const int r = chunk / (G / 8), col = (chunk % (G / 8)) * 8;
+    *reinterpret_cast<uint2*>(wq + static_cast<size_t>(nb * BN + r) * K +
+                              static_cast<size_t>(g) * G + col) =
+        make_uint2(q_i8x4(v[c][0], v[c][1], v[c][2], v[c][3], inv),
+                   q_i8x4(v[c][4], v[c][5], v[c][6], v[c][7], inv));
+  }
+}
+
+// ---------------------------------------------------------------- GEMM
+
+struct alignas(1024) GemmSmem {
+  uint8_t x[NS][GPS][BM * G];  // int8 X tiles [group][128 rows][128 channels]
+  uint8_t w[NS][GPS][BN * G];  // int8 W tiles [group][128 out channels][128 channels]
+  uint64_t full[NS], empty[NS];
+  uint64_t acc_full[NPAIR], acc_free[NPAIR];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(GemmSmem) <= 227 * 1024, "shared memory of one CTA");
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                          int site) {
+  return __all_sync(kFull, mbar_wait(bar, parity, w, site));
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > w.budget) {
+      record_timeout(w.status, kSiteDrain);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void gemm_producer(GemmSmem& s, const W8a8Maps& maps, int m0, int n0,
+                                              int ngroups, const WaitCtx& w) {
+  tma_prefetch_desc(&maps.x);
+  tma_prefetch_desc(&maps.w);
+  const int nsteps = (ngroups + GPS - 1) / GPS;
+  int issued = 0;
+  for (int j = 0; j < nsteps; j++) {
+    const int st = j % NS;
+    if (j >= NS && !mbar_wait(&s.empty[st], ((j / NS) & 1) ^ 1, w, kSiteProdEmpty)) break;
+    const int ng = min(GPS, ngroups - j * GPS);  // groups of this step
+    mbar_arrive_expect_tx(&s.full[st], ng * (BM + BN) * G);
+    for (int q = 0; q < ng; q++) {
+      const int g = j * GPS + q;
+      tma_load_3d(s.x[st][q], &maps.x, &s.full[st], g * G, m0, 0);
+      tma_load_3d(s.w[st][q], &maps.w, &s.full[st], g * G, n0, 0);
+    }
+    issued++;
+  }
+  // every issued load must land before the CTA exits (only the last NS can
+  // still be in flight)
+  for (int j = (issued > NS ? issued - NS : 0); j < issued; j++)
+    drain_wait(&s.full[j % NS], (j / NS) & 1, w);
+}
+
+__device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups, const WaitCtx& w) {
+  constexpr uint32_t idesc = idesc_i8_s32(BM, BN);
+  const int nsteps = (ngroups + GPS - 1) / GPS;
+  for (int j = 0; j < nsteps; j++) {
+    const int st = j % NS, pr = j % NPAIR;
+    if (!mbar_wait(&s.full[st], (j / NS) & 1, w, kSiteMmaFull)) break;
+    // the promotion warps have read this accumulator pair's previous step
+    // and re-seeded it (the first use waits for the initial seed)
+    if (!mbar_wait(&s.acc_free[pr], (j / NPAIR) & 1, w, kSiteMmaAccFree)) break;
+    tc_fence_after();
+    const int ng = min(GPS, ngroups - j * GPS);
+    for (int q = 0; q < ng; q++) {
+      const uint32_t xa = smem_u32(s.x[st][q]), wa = smem_u32(s.w[st][q]);
+      const uint32_t acc = tmem + (pr * GPS + q) * BN;
+#pragma unroll
+      for (int kk = 0; kk < G / 32; kk++)
+        mma_i8_ss(acc, smem_desc_kmajor(xa + kk * 32, G), smem_desc_kmajor(wa + kk * 32, G), idesc,
+                  1);
+    }
+    mma_commit(&s.empty[st]);
+    mma_commit(&s.acc_full[pr]);
+  }
+  mma_commit(&s.drain);
+  drain_wait(&s.drain, 0, w);
+}
+
+// A promotion warp's kPromCols accumulator columns: load / re-seed.
+template <int C>
+__device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&v)[C]) {
+  if constexpr (C == 64) tmem_ld64(taddr, v);
+  else tmem_ld32(taddr, v);
+}
+__device__ __forceinline__ void fill_cols(uint32_t taddr) {
+  if constexpr (kPromCols == 64) tmem_fill64_x8_nowait(taddr, kBiasBits);
+  else tmem_fill32_x8_nowait(taddr, kBiasBits);
+}
+
+// Promotion warps: rows 32 q + lane, columns kPromCols * c .. + kPromCols - 1
+// of the tile (q = lane quadrant, c = column part).
+__device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, uint32_t tmem,
+                                             int m0, int n0, int ngroups, const WaitCtx& w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3, part = (warp - 2) >> 2;
+  const int r = quad * 32 + lane;
+  const int m = m0 + r;
+  const bool valid = m < p.M;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16) + part * kPromCols;
+  const float* sxr = p.sx + static_cast<size_t>(valid ? m : 0) * ngroups;
+  const float* swr = p.sw + static_cast<size_t>(n0 / BN) * ngroups;
+
+  // seed this warp's columns of every accumulator, then release them
+#pragma unroll 1
+  for (int b = 0; b < NACC; b++) fill_cols(tl + b * BN);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0)
+    for (int pr = 0; pr < NPAIR; pr++) mbar_arrive(&s.acc_free[pr]);
+
+  float2 y[kPromCols / 2];
+#pragma unroll
+  for (int e = 0; e < kPromCols / 2; e++) y[e] = make_float2(0.0f, 0.0f);
+  const float2 nb2 = make_float2(-kBias, -kBias);
+  float sxn = valid ? __ldg(sxr) : 0.0f, swn = __ldg(swr);
+  const int nsteps = (ngroups + GPS - 1) / GPS;
+  bool ok = true;
+  for (int j = 0; j < nsteps; j++) {
+    const int pr = j % NPAIR;
+    if (!warp_wait(&s.acc_full[pr], (j / NPAIR) & 1, w, kSitePromFull)) { ok = false; break; }
+    tc_fence_after();
+    // re-seed for the step that reuses these accumulators; the stores drain
+    // while the promotion runs
+    const bool reuse = j + NPAIR < nsteps;
+    const int ng = min(GPS, ngroups - j * GPS);
+    for (int q = 0; q < ng; q++) {
+      const int g = j * GPS + q;
+      const uint32_t acc = tl + (pr * GPS + q) * BN;
+      const float sc = __fmul_rn(sxn, swn);  // fp32(sx[m, g] * sw[n / 128, g])
+      if (g + 1 < ngroups) {
+        sxn = valid ? __ldg(sxr + g + 1) : 0.0f;
+        swn = __ldg(swr + g + 1);
+      }
+      uint32_t v[kPromCols];  // 0x4B400000 + P
+      load_cols(acc, v);
+      if (reuse) fill_cols(acc);
+      const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+      for (int e = 0; e < kPromCols / 2; e++) {
+        const float2 pf = __fadd2_rn(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), nb2);
+        y[e] = __ffma2_rn(pf, sc2, y[e]);
+      }
+    }
+    if (reuse) tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (reuse && lane == 0) mbar_arrive(&s.acc_free[pr]);
+  }
+  if (!ok || !valid) return;
+  const size_t orow = static_cast<size_t>(m) * p.N + n0 + part * kPromCols;
+  uint32_t packed[kPromCols / 2];
+#pragma unroll
+  for (int e = 0; e < kPromCols / 2; e++) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(y[e].x, y[e].y);
+    packed[e] = *reinterpret_cast<uint32_t*>(&h2);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(p.y + orow);
+#pragma unroll
+  for (int e = 0; e < kPromCols / 8; e++)
+    dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+  if (p.y_f32) {
+    float4* d32 = reinterpret_cast<float4*>(p.y_f32 + orow);
+#pragma unroll
+    for (int e = 0; e < kPromCols / 4; e++)
+      d32[e] = make_float4(y[2 * e].x, y[2 * e].y, y[2 * e + 1].x, y[2 * e + 1].y);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_w8a8_gemm(const __grid_constant__ W8a8Maps maps, const W8a8Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0 && atomicCAS(p.status, 0, 3 /* SAGE_ERR_CUDA */) == 0)
+      atomicExch(p.status + 1, kSiteSmemAlign);
+    return;
+  }
+  GemmSmem& s = *reinterpret_cast<GemmSmem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // column tiles run fastest, so that the CTAs in flight share their X rows
+  // (read once from HBM, then from L2) and sweep all of W (L2-resident)
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int ngroups = p.K / G;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; i++) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < NPAIR; i++) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_free[i], kPromWarps);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const WaitCtx w{p.budget, p.status, &s.abort};
+  if (warp == 0) {
+    if (lane == 0) gemm_producer(s, maps, m0, n0, ngroups, w);
+  } else if (warp == 1) {
+    if (lane == 0) gemm_mma(s, tmem, ngroups, w);
+  } else {
+    gemm_promote(s, p, tmem, m0, n0, ngroups, w);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t w8a8_prepare() {
+  return cudaFuncSetAttribute(k_w8a8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(sizeof(GemmSmem)));
+}
+
+cudaError_t launch_w8a8_quant_act(const uint16_t* x, int M, int K, int8_t* xq, float* sx,
+                                  cudaStream_t stream) {
+  const long long threads = static_cast<long long>(M) * (K / G) * 16;
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  k_w8a8_quant_act<<<blocks, 256, 0, stream>>>(x, M, K, xq, sx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w8a8_quant_weight(const uint16_t* w, int N, int K, int8_t* wq, float* sw,
+                                     cudaStream_t stream) {
+  k_w8a8_quant_weight<<<dim3(K / G, N / BN), 256, 0, stream>>>(w, N, K, wq, sw);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w8a8_gemm(const W8a8Maps& maps, const W8a8Params& p, cudaStream_t stream) {
+  dim3 grid(p.N / BN, (p.M + BM - 1) / BM);
+  k_w8a8_gemm<<<grid, kThreads, sizeof(GemmSmem), stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+}  // namespace sage

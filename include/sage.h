@@ -243,6 +243,44 @@ sage_status sage_debug_exp2(const float *x, float *y, size_t n, void *stream);
  * SAGE_ERR_CUDA if the synchronization failed, else SAGE_OK. */
 sage_status sage_sync_status(void *stream);
 
+/* ------------------------------------------------------------------------
+ * Per-block W8A8 linear layer: Y = X W^T with INT8 activations and weights
+ * (Vidu S1 digest, section "Infra": per-block W8A8 for the linear layers,
+ * because per-tensor and per-channel scales are stretched by outliers;
+ * TurboDiffusion notes, W8A8 bullet: 8-bit block-wise quantization on INT8
+ * tensor cores).  Blocks are 128 channels wide along the reduction dim K:
+ * one activation scale per token and 128-channel group, one weight scale per
+ * 128 x 128 block; symmetric absmax/127, codes round-half-to-even, an
+ * all-zero block gets scale 0.  Requirements: K and N multiples of 128,
+ * 1 <= M <= 65535 * 128; all pointers device pointers, caller-allocated,
+ * 16-byte aligned (scale arrays 4-byte aligned).  Asynchronous on `stream`;
+ * errors as for the attention calls.
+ * ---------------------------------------------------------------------- */
+
+/* X bf16 [M, K] -> xq int8 [M, K], sx f32 [M, K/128]:
+ *   a = max |x| over (m, channels 128g .. 128g+127), sx = a/127,
+ *   xq = clamp(rne(x * fp32(127/a)), -127, 127). */
+sage_status sage_w8a8_quant_act(const void *x_bf16, long long M, long long K, int8_t *xq,
+                                float *sx, void *stream);
+
+/* W bf16 [N, K] -> wq int8 [N, K], sw f32 [N/128, K/128], one scale per
+ * 128 x 128 block, same rule as above. */
+sage_status sage_w8a8_quant_weight(const void *w_bf16, long long N, long long K, int8_t *wq,
+                                   float *sw, void *stream);
+
+/* Y = dequant(X) dequant(W)^T on the INT8 tensor cores: for each output
+ * element, each 128-channel group's integer product P_g = sum xq*wq is exact
+ * (int32) and is promoted into an fp32 running sum in ascending group order,
+ *   y = fmaf((float)P_g, fp32(sx[m][g] * sw[n/128][g]), y),
+ * and Y = bf16(y) (round-half-to-even).
+ *   y_bf16  device bf16 [M, N] (required)
+ *   y_f32   device f32 [M, N] (y before rounding) or NULL
+ * One kernel launch (one 128 x 128 output tile per CTA, column tiles
+ * fastest). */
+sage_status sage_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                           long long M, long long N, long long K, void *y_bf16, float *y_f32,
+                           void *stream);
+
 /* Static description of a status code (never NULL). */
 const char *sage_status_string(sage_status status);
 

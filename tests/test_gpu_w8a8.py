@@ -1,0 +1,74 @@
+"""GPU parity of the per-block W8A8 linear layer against the oracle: the
+quantized activations, weights and their scales bit for bit, and the GEMM's
+fp32 output bit for bit (same exact group products, same fp32 promotion
+order), its bf16 output equal to the oracle's value rounded to bf16.  Small
+shapes compare every row (ragged M, one and several groups, zero groups);
+DiT-sized shapes compare sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_attention_sage_b200 as sage
+import oracle
+from bit_quantized_attention_sage_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def bits(shape, seed, outliers=0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(shape).astype(np.float32)
+    if outliers:
+        x[:, rng.choice(shape[1], outliers, replace=False)] *= 30.0
+    return synth.f32_to_bf16_bits(x)
+
+
+def dev(b):
+    return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run(x, w):
+    xq, sx = sage.w8a8_quant_act(dev(x))
+    wq, sw = sage.w8a8_quant_weight(dev(w))
+    y32 = torch.empty((x.shape[0], w.shape[0]), dtype=torch.float32, device="cuda")
+    y = sage.w8a8_gemm(xq, sx, wq, sw, y_f32=y32)
+    assert sage.sync_status() == 0
+    return xq, sx, wq, sw, y, y32
+
+
+def check(x, w, rows=None):
+    xq, sx, wq, sw, y, y32 = run(x, w)
+    rxq, rsx = oracle.w8a8_quant_act(x)
+    rwq, rsw = oracle.w8a8_quant_weight(w)
+    np.testing.assert_array_equal(xq.cpu().numpy(), rxq)
+    np.testing.assert_array_equal(sx.cpu().numpy().view(np.int32), rsx.view(np.int32))
+    np.testing.assert_array_equal(wq.cpu().numpy(), rwq)
+    np.testing.assert_array_equal(sw.cpu().numpy().view(np.int32), rsw.view(np.int32))
+    rows = np.arange(x.shape[0]) if rows is None else rows
+    ry = oracle.w8a8_gemm_rows(rxq, rsx, rwq, rsw, rows)
+    got32 = y32.cpu().numpy()[rows]
+    np.testing.assert_array_equal(got32.view(np.int32), ry.view(np.int32))
+    gotb = y.view(torch.int16).cpu().numpy().view(np.uint16)[rows]
+    np.testing.assert_array_equal(gotb, synth.f32_to_bf16_bits(ry))
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(1, 128, 128, 1), (200, 256, 384, 2), (333, 384, 1536, 3),
+                                        (129, 128, 640, 4)])
+def test_small_all_rows(M, N, K, seed):
+    check(bits((M, K), seed, outliers=3), bits((N, K), seed + 100))
+
+
+def test_zero_groups():
+    x = bits((150, 384), 5)
+    x[:, 128:256] = 0      # a zero activation group in every row
+    x[7] = 0               # a zero row
+    w = bits((256, 384), 6)
+    w[128:, :128] = 0      # a zero weight block
+    check(x, w)
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 1536, 1536), (2040, 5120, 5120)])
+def test_dit_shapes_sampled(M, N, K):
+    rng = np.random.default_rng(M + N)
+    rows = np.sort(np.concatenate([[0, M - 1], rng.choice(M, 30, replace=False)]))
+    check(bits((M, K), 7, outliers=8), bits((N, K), 8), rows=np.unique(rows))
