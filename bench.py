@@ -55,6 +55,10 @@ def parse():
                     help="time sage_attn_fwd_block_sparse on the workload with a seeded random "
                          "128x128 tile mask of this density (one JSON line; TOPS over the "
                          "visible pairs of the enabled tiles)")
+    ap.add_argument("--w8a8", default=None, metavar="M,N,K",
+                    help="time the per-block W8A8 linear layer (activation quantization + INT8 "
+                         "GEMM) on Y[M,N] = X[M,K] W[N,K]^T, one JSON line; the bf16 cuBLAS "
+                         "matmul of the same shape is timed alongside as a library reference")
     ap.add_argument("--sweep-filter", default="",
                     help="only sweep points whose name contains this string")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -544,6 +548,52 @@ def run_block_sparse(args):
         flush=True)
 
 
+# ------------------------------------------------------------------ W8A8 linear layer
+
+def run_w8a8(args):
+    import torch
+    import bit_quantized_attention_sage_b200 as sage
+    torch.cuda.set_device(0)
+    sage.lib()
+    M, N, K = (int(v) for v in args.w8a8.split(","))
+    g = torch.Generator(device="cuda").manual_seed(11)
+    x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    w = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    wq, sw = sage.w8a8_quant_weight(w)
+    xq, sx = sage.w8a8_quant_act(x)
+    y = sage.w8a8_gemm(xq, sx, wq, sw)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    t_gemm = timed(lambda: sage.w8a8_gemm(xq, sx, wq, sw, out=y))
+    t_quant = timed(lambda: sage.w8a8_quant_act(x, xq, sx))
+    t_ref = timed(lambda: torch.matmul(x, w.T))
+    if sage.sync_status() != 0:
+        raise RuntimeError("device status error in the W8A8 run")
+    ops = 2 * M * N * K
+    pk = peaks()
+    print(json.dumps({
+        "w8a8_linear": "M%d_N%d_K%d" % (M, N, K), "gemm_ms": round(t_gemm, 4),
+        "act_quant_ms": round(t_quant, 4), "layer_ms": round(t_gemm + t_quant, 4),
+        "gemm_TOPS": round(ops / (t_gemm / 1e3) / 1e12, 1),
+        "layer_TOPS": round(ops / ((t_gemm + t_quant) / 1e3) / 1e12, 1),
+        "roofline": {"bound": "tensor", "peak": round(pk["i8_sustained"], 1), "unit": "TOPS",
+                     "frac": round(ops / (t_gemm / 1e3) / 1e12 / pk["i8_sustained"], 4),
+                     "peak_note": "8-bit dense = 2 x sustained cuBLAS bf16 (of %s)" % pk["source"]},
+        "cublas_bf16_ms": round(t_ref, 4),
+        "cublas_bf16_TFLOPS": round(ops / (t_ref / 1e3) / 1e12, 1)}), flush=True)
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args):
@@ -583,6 +633,8 @@ def main():
         run_sweep(args)
     elif args.block_density is not None:
         run_block_sparse(args)
+    elif args.w8a8:
+        run_w8a8(args)
     else:
         run_ours(args)
 
