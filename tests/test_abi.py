@@ -84,3 +84,23 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
     tiles = (ctypes.c_int * 3)(0, 5, 0)
     assert L.sage_debug_qk_int32(ctypes.byref(ok), ctypes.byref(s), tiles, 1,
                                  ctypes.c_void_p(4096), None) == 1
+
+
+def test_block_sparse_and_w8a8_arguments_are_rejected_before_any_launch(L):
+    s = sage.make_shape(1, 1, 64, 64, 128)
+    ok = sage._QKV(*([16 * 1024] * 7))
+    out = ctypes.c_void_p(4096)
+    # block-sparse: the mask pointer is required; more than 6144 KV tiles is unsupported
+    assert L.sage_attn_fwd_block_sparse(ctypes.byref(ok), ctypes.byref(s), 0, 0, None, out,
+                                        None, None, None) == 1
+    big = sage.make_shape(1, 1, 64, 6144 * 128 + 1, 128)
+    assert L.sage_attn_fwd_block_sparse(ctypes.byref(ok), ctypes.byref(big), 0, 0,
+                                        ctypes.c_void_p(4096), out, None, None, None) == 2
+    p = ctypes.c_void_p(4096)
+    # W8A8: K and N must be multiples of 128, M >= 1, pointers 16-byte aligned
+    assert L.sage_w8a8_quant_act(p, 4, 100, p, p, None) == 1
+    assert L.sage_w8a8_quant_act(p, 0, 128, p, p, None) == 1
+    assert L.sage_w8a8_quant_weight(p, 130, 128, p, p, None) == 1
+    assert L.sage_w8a8_gemm(p, p, p, p, 8, 128, 200, p, None, None) == 1
+    assert L.sage_w8a8_gemm(p, p, p, p, 8, 64, 128, p, None, None) == 1
+    assert L.sage_w8a8_gemm(ctypes.c_void_p(4100), p, p, p, 8, 128, 128, p, None, None) == 1
