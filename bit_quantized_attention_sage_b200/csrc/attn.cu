@@ -400,7 +400,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   if (!ok) return;
   const float* vsc = p.v_scale + static_cast<size_t>(bh) * D;
   const size_t orow = (static_cast<size_t>(bh) * p.Nq + (valid ? i : 0)) * D;
-  if (nk == 0) {  // block-sparse: no tile at all for this CTA; O = 0, lse = -inf
+  if (SPARSE && nk == 0) {  // no tile at all for this CTA; O = 0, lse = -inf
     if (valid) {
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow);
 #pragma unroll 1
@@ -418,7 +418,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   tc_fence_after();
   // a row that saw no key (possible only with a block mask) has l = 0:
   // O = 0 (its O_acc row is 0) and lse = -inf
-  const bool seen = l > 0.0f;
+  const bool seen = !SPARSE || l > 0.0f;
   const float inv = seen ? __frcp_rn(l) : 0.0f;  // l is in units of 2^8 p
 #pragma unroll 1
   for (int c = 0; c < D; c += 32) {
