@@ -198,6 +198,23 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// Same with f16 operands (kind::f16, both A and B f16) and an fp32
+// accumulator.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Shared-memory matrix descriptor with no swizzle and both byte offsets 0:
+// every 8-row group and both 8-element K halves of a K = 16 f16 operand read
+// the same 8 x 16-byte core matrix at saddr (a 128-byte broadcast tile).
+__device__ __forceinline__ uint64_t smem_desc_bcast(uint32_t saddr) {
+  return (uint64_t((saddr >> 4) & 0x3FFFu)) | (1ull << 46);
+}
 // Arrive once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

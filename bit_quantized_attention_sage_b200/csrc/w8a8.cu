@@ -8,23 +8,27 @@
 // quantizer): one activation scale per token and 128-channel group, one
 // weight scale per 128 x 128 block.
 //
-// GEMM: one CTA per 128 x 128 output tile (one weight block wide), 320
+// GEMM: one CTA per 128 x 128 output tile (one weight block wide), 352
 // threads, one CTA per SM:
-//   warp 0      TMA producer: the X and W tiles of each 128-channel group
-//               through a 4-stage shared-memory ring (128-byte swizzle).
-//   warp 1      allocates 512 TMEM columns: four int32 accumulators of
-//               128 x 128, two steps of two groups in flight; one elected thread
-//               issues tcgen05.mma kind::i8 (four K = 32 steps per group)
-//               onto an accumulator seeded with the bit pattern 0x4B400000,
-//               so that the group's exact integer product P reads back as
-//               the fp32 value 1.5 * 2^23 + P.
-//   warps 2-9   promotion: column part c (0-1) of lane quadrant q owns
+//   warp 0      TMA producer: the X and W tiles of two 128-channel groups per
+//               step through a 3-stage shared-memory ring (128-byte swizzle).
+//   warps 1-2   two MMA-issuing threads, alternating steps (warp 1 also
+//               allocates 512 TMEM columns: four int32 accumulators of
+//               128 x 128, one pair per step in flight).  Per group: one
+//               kind::f16 MMA of a broadcast 128-byte tile (rows
+//               [2048, 1024, 1024, 0, ...] read twice along K = 16: every
+//               product sum is 2 (2^22 + 2^20 + 2^20) = 1.5 * 2^23) writes the
+//               bit pattern 0x4B400000 into the accumulator; four
+//               tcgen05.mma kind::i8 (K = 32 steps) add the group's exact
+//               integer product P, so that it reads back as the fp32 value
+//               1.5 * 2^23 + P.
+//   warps 3-10  promotion: column part c (0-1) of lane quadrant q owns
 //               output rows 32 q .. 32 q + 31 and columns 64 c .. 64 c + 63
-//               (two warps per SM sub-partition).  Per group:
-//               load the 64 scores, re-seed them, release the accumulator,
-//               then y = fma(P, sx * sw, y) in fp32 registers (packed
-//               fp32x2), in ascending group order.  At the end: y -> bf16
-//               (and optional fp32) rows.
+//               (two warps per SM sub-partition).  Per step: load the pair's
+//               scores, release the pair as soon as both groups are in
+//               registers, and fold them into y = fma(P, sx * sw, y) in fp32
+//               registers (packed fp32x2), in ascending group order.  At the
+//               end: y -> bf16 (and optional fp32) rows.
 // Every wait is bounded; on a timeout the CTA drains what it issued, frees
 // TMEM and returns.
 #include "w8a8.cuh"
@@ -45,11 +49,12 @@ constexpr int NACC = 4;          // TMEM accumulators (NACC / GPS steps in fligh
 constexpr int NPAIR = NACC / GPS;
 constexpr int kPromWarps = 8;    // two per lane quadrant, 64 columns each
 constexpr int kPromCols = BN / (kPromWarps / 4);
-constexpr int kThreads = 64 + 32 * kPromWarps;  // producer, MMA, promotion
+constexpr int kIssuers = 2;      // MMA-issuing threads, alternating steps
+constexpr int kFirstProm = 1 + kIssuers;  // warp index of the first promotion warp
+constexpr int kThreads = 32 * (kFirstProm + kPromWarps);
 constexpr int kTmemCols = 512;
 constexpr uint32_t kFull = 0xffffffffu;
-constexpr uint32_t kBiasBits = 0x4B400000u;  // 1.5 * 2^23
-constexpr float kBias = 12582912.0f;
+constexpr float kBias = 12582912.0f;  // 1.5 * 2^23, the accumulator seed
 
 enum : int {
   kSiteProdEmpty = 0x20101, kSiteMmaFull, kSiteMmaAccFree, kSitePromFull, kSiteDrain,
@@ -143,6 +148,7 @@ __global__ void __launch_bounds__(256) k_w8a8_quant_weight(const uint16_t* __res
 struct alignas(1024) GemmSmem {
   uint8_t x[NS][GPS][BM * G];  // int8 X tiles [group][128 rows][128 channels]
   uint8_t w[NS][GPS][BN * G];  // int8 W tiles [group][128 out channels][128 channels]
+  uint8_t seed[128];           // f16 broadcast tile of the accumulator seed MMA
   uint64_t full[NS], empty[NS];
   uint64_t acc_full[NPAIR], acc_free[NPAIR];
   uint64_t drain;
@@ -190,10 +196,12 @@ __device__ __forceinline__ void gemm_producer(GemmSmem& s, const W8a8Maps& maps,
     drain_wait(&s.full[j % NS], (j / NS) & 1, w);
 }
 
-__device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups, const WaitCtx& w) {
+// One thread per issuer: steps who, who + kIssuers, ...
+__device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups, const WaitCtx& w,
+                                         int who) {
   constexpr uint32_t idesc = idesc_i8_s32(BM, BN);
   const int nsteps = (ngroups + GPS - 1) / GPS;
-  for (int j = 0; j < nsteps; j++) {
+  for (int j = who; j < nsteps; j += kIssuers) {
     const int st = j % NS, pr = j % NPAIR;
     if (!mbar_wait(&s.full[st], (j / NS) & 1, w, kSiteMmaFull)) break;
     // the promotion warps have read this accumulator pair's previous step
@@ -204,6 +212,10 @@ __device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups
     for (int q = 0; q < ng; q++) {
       const uint32_t xa = smem_u32(s.x[st][q]), wa = smem_u32(s.w[st][q]);
       const uint32_t acc = tmem + (pr * GPS + q) * BN;
+      // seed: D = A B with A = B = the broadcast tile, 1.5 * 2^23 in every cell
+      // (the f16 kind's instruction descriptor has the same fields as e4m3's)
+      mma_f16_ss(acc, smem_desc_bcast(smem_u32(s.seed)), smem_desc_bcast(smem_u32(s.seed)),
+                 idesc_e4m3_f32(BM, BN), 0);
 #pragma unroll
       for (int kk = 0; kk < G / 32; kk++)
         mma_i8_ss(acc, smem_desc_kmajor(xa + kk * 32, G), smem_desc_kmajor(wa + kk * 32, G), idesc,
@@ -216,15 +228,11 @@ __device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups
   drain_wait(&s.drain, 0, w);
 }
 
-// A promotion warp's kPromCols accumulator columns: load / re-seed.
+// A promotion warp's kPromCols accumulator columns.
 template <int C>
 __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&v)[C]) {
   if constexpr (C == 64) tmem_ld64(taddr, v);
   else tmem_ld32(taddr, v);
-}
-__device__ __forceinline__ void fill_cols(uint32_t taddr) {
-  if constexpr (kPromCols == 64) tmem_fill64_x8_nowait(taddr, kBiasBits);
-  else tmem_fill32_x8_nowait(taddr, kBiasBits);
 }
 
 // Promotion warps: rows 32 q + lane, columns kPromCols * c .. + kPromCols - 1
@@ -232,7 +240,7 @@ __device__ __forceinline__ void fill_cols(uint32_t taddr) {
 __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, uint32_t tmem,
                                              int m0, int n0, int ngroups, const WaitCtx& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int quad = warp & 3, part = (warp - 2) >> 2;
+  const int quad = warp & 3, part = (warp - kFirstProm) >> 2;
   const int r = quad * 32 + lane;
   const int m = m0 + r;
   const bool valid = m < p.M;
@@ -240,10 +248,8 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
   const float* sxr = p.sx + static_cast<size_t>(valid ? m : 0) * ngroups;
   const float* swr = p.sw + static_cast<size_t>(n0 / BN) * ngroups;
 
-  // seed this warp's columns of every accumulator, then release them
-#pragma unroll 1
-  for (int b = 0; b < NACC; b++) fill_cols(tl + b * BN);
-  tmem_wait_st();
+  // release every accumulator pair for its first step (the issuers seed
+  // the accumulators themselves)
   tc_fence_before();
   __syncwarp();
   if (lane == 0)
@@ -274,7 +280,11 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
       }
       uint32_t v[kPromCols];  // 0x4B400000 + P
       load_cols(acc, v);
-      if (reuse) fill_cols(acc);
+      if (q == ng - 1) {  // the pair is in registers: release it
+        tc_fence_before();
+        __syncwarp();
+        if (reuse && lane == 0) mbar_arrive(&s.acc_free[pr]);
+      }
       const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
       for (int e = 0; e < kPromCols / 2; e++) {
@@ -282,10 +292,6 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
         y[e] = __ffma2_rn(pf, sc2, y[e]);
       }
     }
-    if (reuse) tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (reuse && lane == 0) mbar_arrive(&s.acc_free[pr]);
   }
   if (!ok || !valid) return;
   const size_t orow = static_cast<size_t>(m) * p.N + n0 + part * kPromCols;
@@ -330,9 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.acc_full[i], 1);
       mbar_init(&s.acc_free[i], kPromWarps);
     }
-    mbar_init(&s.drain, 1);
+    mbar_init(&s.drain, kIssuers);
     s.abort = 0;
     fence_mbar_init();
+  }
+  if (threadIdx.x < 32) {  // seed tile: 8 rows of f16 [2048, 1024, 1024, 0, 0, 0, 0, 0]
+    const uint32_t wv = (threadIdx.x & 3) == 0 ? 0x64006800u : (threadIdx.x & 3) == 1 ? 0x6400u : 0u;
+    reinterpret_cast<uint32_t*>(s.seed)[threadIdx.x] = wv;
+    fence_proxy_async_smem();
   }
   if (warp == 1) {
     tmem_alloc(&s.tmem_base, kTmemCols);
@@ -345,8 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx w{p.budget, p.status, &s.abort};
   if (warp == 0) {
     if (lane == 0) gemm_producer(s, maps, m0, n0, ngroups, w);
-  } else if (warp == 1) {
-    if (lane == 0) gemm_mma(s, tmem, ngroups, w);
+  } else if (warp < kFirstProm) {
+    if (lane == 0) gemm_mma(s, tmem, ngroups, w, warp - 1);
   } else {
     gemm_promote(s, p, tmem, m0, n0, ngroups, w);
   }
