@@ -189,7 +189,7 @@ namespace {
 bool w8a8_dims_ok(long long M, long long N, long long K) {
   return M >= 1 && N >= kW8a8BN && K >= kW8a8Group && N % kW8a8BN == 0 && K % kW8a8Group == 0 &&
          M <= (1ll << 31) - 1 && N <= (1 << 24) && K <= (1 << 24) &&
-         (M + kW8a8BM - 1) / kW8a8BM <= 65535;
+         ((M + kW8a8BM - 1) / kW8a8BM) * (N / kW8a8BN) <= (1ll << 31) - 1;
 }
 }  // namespace
 

@@ -8,8 +8,8 @@
 // quantizer): one activation scale per token and 128-channel group, one
 // weight scale per 128 x 128 block.
 //
-// GEMM: one CTA per 128 x 128 output tile (one weight block wide), 352
-// threads, one CTA per SM:
+// GEMM: persistent, one CTA per SM looping over 128 x 128 output tiles (one
+// weight block wide), 352 threads:
 //   warp 0      TMA producer: the X and W tiles of two 128-channel groups per
 //               step through a 3-stage shared-memory ring (128-byte swizzle).
 //   warps 1-2   two MMA-issuing threads, alternating steps (warp 1 also
@@ -172,41 +172,74 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
   }
 }
 
-__device__ __forceinline__ void gemm_producer(GemmSmem& s, const W8a8Maps& maps, int m0, int n0,
-                                              int ngroups, const WaitCtx& w) {
+// The output tiles of one CTA: t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// (one CTA per SM, persistent).  Column tiles run fastest, so that the CTAs
+// in flight share their X rows (read once from HBM, then from L2) and sweep
+// all of W (L2-resident).  Pipeline steps are numbered across the CTA's
+// tiles (step J = tile i * nsteps + step j of the tile), so the stage ring
+// and the accumulator pairs run on from one tile into the next.
+struct TileSched {
+  int ntn, ntiles, nsteps;
+  __device__ __forceinline__ TileSched(const W8a8Params& p)
+      : ntn(p.N / BN), ntiles(((p.M + BM - 1) / BM) * (p.N / BN)),
+        nsteps((p.K / G + GPS - 1) / GPS) {}
+  __device__ __forceinline__ int count() const {
+    const int b = static_cast<int>(blockIdx.x), g = static_cast<int>(gridDim.x);
+    return b < ntiles ? (ntiles - 1 - b) / g + 1 : 0;
+  }
+  __device__ __forceinline__ int tile(int i) const {
+    return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+  }
+  __device__ __forceinline__ int m0(int i) const { return (tile(i) / ntn) * BM; }
+  __device__ __forceinline__ int n0(int i) const { return (tile(i) % ntn) * BN; }
+  __device__ __forceinline__ int total() const { return count() * nsteps; }
+};
+
+__device__ __forceinline__ void gemm_producer(GemmSmem& s, const W8a8Maps& maps,
+                                              const TileSched& ts, int ngroups, const WaitCtx& w) {
   tma_prefetch_desc(&maps.x);
   tma_prefetch_desc(&maps.w);
-  const int nsteps = (ngroups + GPS - 1) / GPS;
-  int issued = 0;
-  for (int j = 0; j < nsteps; j++) {
-    const int st = j % NS;
-    if (j >= NS && !mbar_wait(&s.empty[st], ((j / NS) & 1) ^ 1, w, kSiteProdEmpty)) break;
-    const int ng = min(GPS, ngroups - j * GPS);  // groups of this step
-    mbar_arrive_expect_tx(&s.full[st], ng * (BM + BN) * G);
-    for (int q = 0; q < ng; q++) {
-      const int g = j * GPS + q;
-      tma_load_3d(s.x[st][q], &maps.x, &s.full[st], g * G, m0, 0);
-      tma_load_3d(s.w[st][q], &maps.w, &s.full[st], g * G, n0, 0);
+  const int ntile = ts.count();
+  int J = 0;  // pipeline step of the CTA
+  for (int i = 0; i < ntile; i++) {
+    const int m0 = ts.m0(i), n0 = ts.n0(i);
+    bool ok = true;
+    for (int j = 0; j < ts.nsteps; j++, J++) {
+      const int st = J % NS;
+      if (J >= NS && !mbar_wait(&s.empty[st], ((J / NS) & 1) ^ 1, w, kSiteProdEmpty)) {
+        ok = false;
+        break;
+      }
+      const int ng = min(GPS, ngroups - j * GPS);  // groups of this step
+      mbar_arrive_expect_tx(&s.full[st], ng * (BM + BN) * G);
+      for (int q = 0; q < ng; q++) {
+        const int g = j * GPS + q;
+        tma_load_3d(s.x[st][q], &maps.x, &s.full[st], g * G, m0, 0);
+        tma_load_3d(s.w[st][q], &maps.w, &s.full[st], g * G, n0, 0);
+      }
     }
-    issued++;
+    if (!ok) break;
   }
   // every issued load must land before the CTA exits (only the last NS can
   // still be in flight)
-  for (int j = (issued > NS ? issued - NS : 0); j < issued; j++)
-    drain_wait(&s.full[j % NS], (j / NS) & 1, w);
+  for (int k = (J > NS ? J - NS : 0); k < J; k++) drain_wait(&s.full[k % NS], (k / NS) & 1, w);
 }
 
 // One thread per issuer: steps who, who + kIssuers, ...
-__device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups, const WaitCtx& w,
-                                         int who) {
+__device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, const TileSched& ts,
+                                         int ngroups, const WaitCtx& w, int who) {
   constexpr uint32_t idesc = idesc_i8_s32(BM, BN);
-  const int nsteps = (ngroups + GPS - 1) / GPS;
-  for (int j = who; j < nsteps; j += kIssuers) {
-    const int st = j % NS, pr = j % NPAIR;
-    if (!mbar_wait(&s.full[st], (j / NS) & 1, w, kSiteMmaFull)) break;
-    // the promotion warps have read this accumulator pair's previous step
-    // and re-seeded it (the first use waits for the initial seed)
-    if (!mbar_wait(&s.acc_free[pr], (j / NPAIR) & 1, w, kSiteMmaAccFree)) break;
+  const int total = ts.total();
+  const uint64_t seed = smem_desc_bcast(smem_u32(s.seed));
+  // step J = who, who + kIssuers, ...; j = J mod nsteps kept without divisions
+  int j = who;
+  while (j >= ts.nsteps) j -= ts.nsteps;
+  for (int J = who; J < total; J += kIssuers) {
+    const int st = J % NS, pr = J % NPAIR;
+    if (!mbar_wait(&s.full[st], (J / NS) & 1, w, kSiteMmaFull)) break;
+    // the promotion warps have loaded this accumulator pair's previous step
+    // (the first use waits for their initial release)
+    if (!mbar_wait(&s.acc_free[pr], (J / NPAIR) & 1, w, kSiteMmaAccFree)) break;
     tc_fence_after();
     const int ng = min(GPS, ngroups - j * GPS);
     for (int q = 0; q < ng; q++) {
@@ -214,8 +247,7 @@ __device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups
       const uint32_t acc = tmem + (pr * GPS + q) * BN;
       // seed: D = A B with A = B = the broadcast tile, 1.5 * 2^23 in every cell
       // (the f16 kind's instruction descriptor has the same fields as e4m3's)
-      mma_f16_ss(acc, smem_desc_bcast(smem_u32(s.seed)), smem_desc_bcast(smem_u32(s.seed)),
-                 idesc_e4m3_f32(BM, BN), 0);
+      mma_f16_ss(acc, seed, seed, idesc_e4m3_f32(BM, BN), 0);
 #pragma unroll
       for (int kk = 0; kk < G / 32; kk++)
         mma_i8_ss(acc, smem_desc_kmajor(xa + kk * 32, G), smem_desc_kmajor(wa + kk * 32, G), idesc,
@@ -223,6 +255,8 @@ __device__ __forceinline__ void gemm_mma(GemmSmem& s, uint32_t tmem, int ngroups
     }
     mma_commit(&s.empty[st]);
     mma_commit(&s.acc_full[pr]);
+    j += kIssuers;
+    while (j >= ts.nsteps) j -= ts.nsteps;
   }
   mma_commit(&s.drain);
   drain_wait(&s.drain, 0, w);
@@ -236,17 +270,15 @@ __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&v)[C]) {
 }
 
 // Promotion warps: rows 32 q + lane, columns kPromCols * c .. + kPromCols - 1
-// of the tile (q = lane quadrant, c = column part).
+// of each tile (q = lane quadrant, c = column part).
 __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, uint32_t tmem,
-                                             int m0, int n0, int ngroups, const WaitCtx& w) {
+                                             const TileSched& ts, int ngroups, const WaitCtx& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3, part = (warp - kFirstProm) >> 2;
   const int r = quad * 32 + lane;
-  const int m = m0 + r;
-  const bool valid = m < p.M;
   const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16) + part * kPromCols;
-  const float* sxr = p.sx + static_cast<size_t>(valid ? m : 0) * ngroups;
-  const float* swr = p.sw + static_cast<size_t>(n0 / BN) * ngroups;
+  const float2 nb2 = make_float2(-kBias, -kBias);
+  const int ntile = ts.count(), total = ts.total();
 
   // release every accumulator pair for its first step (the issuers seed
   // the accumulators themselves)
@@ -255,61 +287,64 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
   if (lane == 0)
     for (int pr = 0; pr < NPAIR; pr++) mbar_arrive(&s.acc_free[pr]);
 
-  float2 y[kPromCols / 2];
+  int J = 0;
+  for (int i = 0; i < ntile; i++) {
+    const int m = ts.m0(i) + r, n0 = ts.n0(i);
+    const bool valid = m < p.M;
+    const float* sxr = p.sx + static_cast<size_t>(valid ? m : 0) * ngroups;
+    const float* swr = p.sw + static_cast<size_t>(n0 / BN) * ngroups;
+    float2 y[kPromCols / 2];
 #pragma unroll
-  for (int e = 0; e < kPromCols / 2; e++) y[e] = make_float2(0.0f, 0.0f);
-  const float2 nb2 = make_float2(-kBias, -kBias);
-  float sxn = valid ? __ldg(sxr) : 0.0f, swn = __ldg(swr);
-  const int nsteps = (ngroups + GPS - 1) / GPS;
-  bool ok = true;
-  for (int j = 0; j < nsteps; j++) {
-    const int pr = j % NPAIR;
-    if (!warp_wait(&s.acc_full[pr], (j / NPAIR) & 1, w, kSitePromFull)) { ok = false; break; }
-    tc_fence_after();
-    // re-seed for the step that reuses these accumulators; the stores drain
-    // while the promotion runs
-    const bool reuse = j + NPAIR < nsteps;
-    const int ng = min(GPS, ngroups - j * GPS);
-    for (int q = 0; q < ng; q++) {
-      const int g = j * GPS + q;
-      const uint32_t acc = tl + (pr * GPS + q) * BN;
-      const float sc = __fmul_rn(sxn, swn);  // fp32(sx[m, g] * sw[n / 128, g])
-      if (g + 1 < ngroups) {
-        sxn = valid ? __ldg(sxr + g + 1) : 0.0f;
-        swn = __ldg(swr + g + 1);
-      }
-      uint32_t v[kPromCols];  // 0x4B400000 + P
-      load_cols(acc, v);
-      if (q == ng - 1) {  // the pair is in registers: release it
-        tc_fence_before();
-        __syncwarp();
-        if (reuse && lane == 0) mbar_arrive(&s.acc_free[pr]);
-      }
-      const float2 sc2 = make_float2(sc, sc);
+    for (int e = 0; e < kPromCols / 2; e++) y[e] = make_float2(0.0f, 0.0f);
+    float sxn = valid ? __ldg(sxr) : 0.0f, swn = __ldg(swr);
+    for (int j = 0; j < ts.nsteps; j++, J++) {
+      const int pr = J % NPAIR;
+      if (!warp_wait(&s.acc_full[pr], (J / NPAIR) & 1, w, kSitePromFull)) return;
+      tc_fence_after();
+      const bool reuse = J + NPAIR < total;  // a later step fills this pair again
+      const int ng = min(GPS, ngroups - j * GPS);
+      for (int q = 0; q < ng; q++) {
+        const int g = j * GPS + q;
+        const uint32_t acc = tl + (pr * GPS + q) * BN;
+        const float sc = __fmul_rn(sxn, swn);  // fp32(sx[m, g] * sw[n / 128, g])
+        if (g + 1 < ngroups) {
+          sxn = valid ? __ldg(sxr + g + 1) : 0.0f;
+          swn = __ldg(swr + g + 1);
+        }
+        uint32_t v[kPromCols];  // 0x4B400000 + P
+        load_cols(acc, v);
+        if (q == ng - 1) {  // the pair is in registers: release it
+          tc_fence_before();
+          __syncwarp();
+          if (reuse && lane == 0) mbar_arrive(&s.acc_free[pr]);
+        }
+        const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-      for (int e = 0; e < kPromCols / 2; e++) {
-        const float2 pf = __fadd2_rn(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), nb2);
-        y[e] = __ffma2_rn(pf, sc2, y[e]);
+        for (int e = 0; e < kPromCols / 2; e++) {
+          const float2 pf = __fadd2_rn(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), nb2);
+          y[e] = __ffma2_rn(pf, sc2, y[e]);
+        }
       }
     }
-  }
-  if (!ok || !valid) return;
-  const size_t orow = static_cast<size_t>(m) * p.N + n0 + part * kPromCols;
-  uint32_t packed[kPromCols / 2];
+    // epilogue of this tile (the issuers already run the next tile's steps)
+    if (!valid) continue;
+    const size_t orow = static_cast<size_t>(m) * p.N + n0 + part * kPromCols;
+    uint32_t packed[kPromCols / 2];
 #pragma unroll
-  for (int e = 0; e < kPromCols / 2; e++) {
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(y[e].x, y[e].y);
-    packed[e] = *reinterpret_cast<uint32_t*>(&h2);
-  }
-  uint4* dst = reinterpret_cast<uint4*>(p.y + orow);
+    for (int e = 0; e < kPromCols / 2; e++) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(y[e].x, y[e].y);
+      packed[e] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.y + orow);
 #pragma unroll
-  for (int e = 0; e < kPromCols / 8; e++)
-    dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-  if (p.y_f32) {
-    float4* d32 = reinterpret_cast<float4*>(p.y_f32 + orow);
+    for (int e = 0; e < kPromCols / 8; e++)
+      dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+    if (p.y_f32) {
+      float4* d32 = reinterpret_cast<float4*>(p.y_f32 + orow);
 #pragma unroll
-    for (int e = 0; e < kPromCols / 4; e++)
-      d32[e] = make_float4(y[2 * e].x, y[2 * e].y, y[2 * e + 1].x, y[2 * e + 1].y);
+      for (int e = 0; e < kPromCols / 4; e++)
+        d32[e] = make_float4(y[2 * e].x, y[2 * e].y, y[2 * e + 1].x, y[2 * e + 1].y);
+    }
   }
 }
 
@@ -323,10 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   GemmSmem& s = *reinterpret_cast<GemmSmem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // column tiles run fastest, so that the CTAs in flight share their X rows
-  // (read once from HBM, then from L2) and sweep all of W (L2-resident)
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
   const int ngroups = p.K / G;
+  const TileSched ts(p);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; i++) {
       mbar_init(&s.full[i], 1);
@@ -355,11 +388,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{p.budget, p.status, &s.abort};
   if (warp == 0) {
-    if (lane == 0) gemm_producer(s, maps, m0, n0, ngroups, w);
+    if (lane == 0) gemm_producer(s, maps, ts, ngroups, w);
   } else if (warp < kFirstProm) {
-    if (lane == 0) gemm_mma(s, tmem, ngroups, w, warp - 1);
+    if (lane == 0) gemm_mma(s, tmem, ts, ngroups, w, warp - 1);
   } else {
-    gemm_promote(s, p, tmem, m0, n0, ngroups, w);
+    gemm_promote(s, p, tmem, ts, ngroups, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -392,7 +425,21 @@ cudaError_t launch_w8a8_quant_weight(const uint16_t* w, int N, int K, int8_t* wq
 }
 
 cudaError_t launch_w8a8_gemm(const W8a8Maps& maps, const W8a8Params& p, cudaStream_t stream) {
-  dim3 grid(p.N / BN, (p.M + BM - 1) / BM);
+  // one CTA per SM (the CTAs loop over the output tiles)
+  static int sms[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (sms[dev] == 0) {
+    e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const long long ntiles = static_cast<long long>((p.M + BM - 1) / BM) * (p.N / BN);
+  const int grid = static_cast<int>(ntiles < sms[dev] ? ntiles : sms[dev]);
+  // the pipeline step counters of one CTA are ints
+  const long long steps = (ntiles + grid - 1) / grid * ((p.K / G + GPS - 1) / GPS);
+  if (steps > (1ll << 31) - 1) return cudaErrorInvalidValue;
   k_w8a8_gemm<<<grid, kThreads, sizeof(GemmSmem), stream>>>(maps, p);
   return cudaGetLastError();
 }
