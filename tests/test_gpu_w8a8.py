@@ -2,8 +2,8 @@
 quantized activations, weights and their scales bit for bit, and the GEMM's
 fp32 output bit for bit (same exact group products, same fp32 promotion
 order), its bf16 output equal to the oracle's value rounded to bf16.  Small
-shapes compare every row (ragged M, one and several groups, zero groups);
-DiT-sized shapes compare sampled rows."""
+shapes compare every row (ragged M, one and several groups, zero groups,
+more tiles than SMs); DiT-sized shapes compare sampled rows."""
 import numpy as np
 import pytest
 import torch
@@ -56,6 +56,13 @@ def check(x, w, rows=None):
                                         (129, 128, 640, 4)])
 def test_small_all_rows(M, N, K, seed):
     check(bits((M, K), seed, outliers=3), bits((N, K), seed + 100))
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(2100, 1280, 256, 9), (1900, 1408, 640, 10)])
+def test_many_tiles_per_cta_all_rows(M, N, K, seed):
+    # more output tiles than SMs: each persistent CTA computes several tiles,
+    # with the pipeline steps (odd counts here) running on across them
+    check(bits((M, K), seed, outliers=2), bits((N, K), seed + 100))
 
 
 def test_zero_groups():
