@@ -48,6 +48,8 @@ def lib():
         L.orc_e4m3_encode_n.argtypes = [P, i64, P]
         L.orc_quant_head.restype = i32
         L.orc_quant_head.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P]
+        L.orc_quant_head_rope.restype = i32
+        L.orc_quant_head_rope.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P]
         L.orc_qk_int32.restype = None
         L.orc_qk_int32.argtypes = [P, P, i32, i64, i64, i64, i64, P]
         L.orc_row_limit.restype = i64
@@ -101,8 +103,12 @@ def e4m3_decode(codes):
 
 # ---------------------------------------------------------------- quantization
 
-def quant_head(q, k, v):
+def quant_head(q, k, v, rope=None):
     """Quantize one head.  q [nq, D], k/v [nkv, D] as uint16 bf16 bits.
+
+    rope: None, or (q_cos, q_sin, k_cos, k_sin), float32 [nq, D/2] and
+    [nkv, D/2]: Q and K are first rotated pairwise by those angles
+    (``orc_quant_head_rope``).
 
     Returns a dict: q8 [nq_pad, D] int8, qs [nq_blk] f32, k8 [nkv_pad, D] int8,
     ks [nkv_blk] f32, mu [D] f32, v8 [nkv, D] uint8 e4m3 codes, vs [D] f32.
@@ -117,19 +123,27 @@ def quant_head(q, k, v):
                k8=np.empty((nkb * BLK, D), np.int8), ks=np.empty(nkb, np.float32),
                mu=np.empty(D, np.float32), v8=np.empty((nkv, D), np.uint8),
                vs=np.empty(D, np.float32))
-    rc = lib().orc_quant_head(_p(q), _p(k), _p(v), nq, nkv, D,
-                              _p(out["q8"]), _p(out["qs"]), _p(out["k8"]), _p(out["ks"]),
-                              _p(out["mu"]), _p(out["v8"]), _p(out["vs"]))
+    outs = [_p(out[key]) for key in ("q8", "qs", "k8", "ks", "mu", "v8", "vs")]
+    if rope is None:
+        rc = lib().orc_quant_head(_p(q), _p(k), _p(v), nq, nkv, D, *outs)
+    else:
+        tabs = [np.ascontiguousarray(t, np.float32) for t in rope]
+        for t, n in zip(tabs, (nq, nq, nkv, nkv)):
+            if t.shape != (n, D // 2):
+                raise ValueError("rotation table shape %s, expected %s" % (t.shape, (n, D // 2)))
+        rc = lib().orc_quant_head_rope(_p(q), _p(k), _p(v), nq, nkv, D,
+                                       *[_p(t) for t in tabs], *outs)
     if rc:
-        raise MemoryError("orc_quant_head failed")
+        raise MemoryError("oracle quantization failed")
     out["nq"], out["nkv"], out["D"] = nq, nkv, D
     return out
 
 
-def quant(q, k, v):
-    """Quantize [B, H, N, D] bf16-bit tensors head by head; returns stacked arrays."""
+def quant(q, k, v, rope=None):
+    """Quantize [B, H, N, D] bf16-bit tensors head by head; returns stacked arrays.
+    rope: as for quant_head (the same tables for every batch entry and head)."""
     B, H = q.shape[:2]
-    heads = [quant_head(q[b, h], k[b, h], v[b, h]) for b in range(B) for h in range(H)]
+    heads = [quant_head(q[b, h], k[b, h], v[b, h], rope) for b in range(B) for h in range(H)]
     out = {}
     for key in ("q8", "qs", "k8", "ks", "mu", "v8", "vs"):
         a = np.stack([hd[key] for hd in heads])

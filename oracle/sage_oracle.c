@@ -181,6 +181,31 @@ static void quant_blocks_i8(const float *x, long n, int D, int8_t *q, float *sca
     }
 }
 
+/* Rotary position embedding of the rows of an [n, D] fp32 matrix, in place
+ * (the pages' RoPE: features are cached before RoPE and rotated at their
+ * current positions, "Vidu S1" digest, Infra, RoPE Repositioning).
+ * Reading: channel pairs (2p, 2p+1), p < D/2, are rotated as one complex
+ * number by the angle whose cosine and sine the caller supplies per row and
+ * pair (cs, sn: [n, D/2] fp32), which covers 1D and multi-axis (frame,
+ * height, width) RoPE alike:
+ *   x'[2p]   = fma(x[2p], c, -fp32(x[2p+1] * s))
+ *   x'[2p+1] = fma(x[2p], s,  fp32(x[2p+1] * c))
+ * each product and each fma rounded once to fp32; the result is not rounded
+ * to bf16 before quantization. */
+static void rope_rows(float *x, long n, int D, const float *cs, const float *sn)
+{
+    const int P = D / 2;
+    for (long r = 0; r < n; r++)
+        for (int p = 0; p < P; p++) {
+            float x0 = x[r * D + 2 * p], x1 = x[r * D + 2 * p + 1];
+            float c = cs[r * P + p], s = sn[r * P + p];
+            float t = x1 * s;
+            float u = x1 * c;
+            x[r * D + 2 * p] = fmaf(x0, c, -t);
+            x[r * D + 2 * p + 1] = fmaf(x0, s, u);
+        }
+}
+
 /* Quantize one (batch, head): Q [nq, D], K [nkv, D], V [nkv, D] as bf16 bits.
  *
  * Outputs (caller-allocated):
@@ -195,11 +220,18 @@ static void quant_blocks_i8(const float *x, long n, int D, int8_t *q, float *sca
  *
  * V: per channel d over all nkv tokens, a = max |V[:,d]|, vs = a/448,
  * inv = 448/a, v8 = e4m3_rne_satfinite(V * inv); a == 0 gives vs = 0, v8 = 0.
+ *
+ * With rotation tables (q_cos, q_sin: [nq, D/2]; k_cos, k_sin: [nkv, D/2];
+ * all four or none), Q and K are first rotated by rope_rows and everything
+ * above applies to the rotated values (the K mean included); V is not
+ * rotated.
  */
-int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                   long nq, long nkv, int D,
-                   int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
-                   uint8_t *v8, float *vs)
+static int quant_head_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           long nq, long nkv, int D,
+                           const float *q_cos, const float *q_sin,
+                           const float *k_cos, const float *k_sin,
+                           int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
+                           uint8_t *v8, float *vs)
 {
     float *x = (float *)malloc(sizeof(float) * (size_t)((nq > nkv ? nq : nkv) * D));
     if (!x)
@@ -207,8 +239,14 @@ int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     /* Q */
     for (long i = 0; i < nq * D; i++)
         x[i] = bf16_to_f32(q[i]);
+    if (q_cos)
+        rope_rows(x, nq, D, q_cos, q_sin);
     quant_blocks_i8(x, nq, D, q8, qs);
-    /* K channel mean in the canonical fp64 order */
+    /* K (rotated), then its channel mean in the canonical fp64 order */
+    for (long i = 0; i < nkv * D; i++)
+        x[i] = bf16_to_f32(k[i]);
+    if (k_cos)
+        rope_rows(x, nkv, D, k_cos, k_sin);
     long nblk = (nkv + ORC_BLK - 1) / ORC_BLK;
     for (int d = 0; d < D; d++) {
         double total = 0.0;
@@ -216,7 +254,7 @@ int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             double s = 0.0;
             long r1 = (b + 1) * ORC_BLK < nkv ? (b + 1) * ORC_BLK : nkv;
             for (long r = b * ORC_BLK; r < r1; r++)
-                s += (double)bf16_to_f32(k[r * D + d]);
+                s += (double)x[r * D + d];
             total += s;
         }
         mu[d] = (float)(total / (double)nkv);
@@ -224,7 +262,7 @@ int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     /* smoothed K, then block quantization */
     for (long r = 0; r < nkv; r++)
         for (int d = 0; d < D; d++)
-            x[r * D + d] = bf16_to_f32(k[r * D + d]) - mu[d];
+            x[r * D + d] = x[r * D + d] - mu[d];
     quant_blocks_i8(x, nkv, D, k8, ks);
     /* V per channel */
     for (int d = 0; d < D; d++) {
@@ -247,6 +285,28 @@ int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
     free(x);
     return 0;
+}
+
+int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                   long nq, long nkv, int D,
+                   int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
+                   uint8_t *v8, float *vs)
+{
+    return quant_head_impl(q, k, v, nq, nkv, D, NULL, NULL, NULL, NULL,
+                           q8, qs, k8, ks, mu, v8, vs);
+}
+
+int orc_quant_head_rope(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        long nq, long nkv, int D,
+                        const float *q_cos, const float *q_sin,
+                        const float *k_cos, const float *k_sin,
+                        int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
+                        uint8_t *v8, float *vs)
+{
+    if (!q_cos || !q_sin || !k_cos || !k_sin)
+        return 2;
+    return quant_head_impl(q, k, v, nq, nkv, D, q_cos, q_sin, k_cos, k_sin,
+                           q8, qs, k8, ks, mu, v8, vs);
 }
 
 /* Exact integer scores S[i,j] = sum_d q8[i,d] * k8[j,d] for rows i0..i0+ni-1
