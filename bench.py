@@ -59,6 +59,10 @@ def parse():
                     help="time the per-block W8A8 linear layer (activation quantization + INT8 "
                          "GEMM) on Y[M,N] = X[M,K] W[N,K]^T, one JSON line; the bf16 cuBLAS "
                          "matmul of the same shape is timed alongside as a library reference")
+    ap.add_argument("--rope", action="store_true",
+                    help="time sage_quant_qk_rope (RoPE applied to Q and K inside the quantizer, "
+                         "1D angles pos * 10000^(-2p/D)) against sage_quant_qk on the workload, "
+                         "one JSON line")
     ap.add_argument("--sweep-filter", default="",
                     help="only sweep points whose name contains this string")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -594,6 +598,51 @@ def run_w8a8(args):
         "cublas_bf16_TFLOPS": round(ops / (t_ref / 1e3) / 1e12, 1)}), flush=True)
 
 
+# ------------------------------------------------------------------ rotary quantizer
+
+def run_rope(args):
+    import torch
+    import bit_quantized_attention_sage_b200 as sage
+    torch.cuda.set_device(0)
+    sage.lib()
+    w = synth.WORKLOADS[args.workload]
+    g = torch.Generator(device="cuda").manual_seed(12)
+    q, k, v = (torch.randn(w.B, w.H, n, w.D, device="cuda", generator=g).to(torch.bfloat16)
+               for n in (w.Nq, w.Nkv, w.Nkv))
+
+    def tables(n, pos0):
+        pos = torch.arange(pos0, pos0 + n, device="cuda", dtype=torch.float64)[:, None]
+        inv = 10000.0 ** (-2.0 * torch.arange(w.D // 2, device="cuda", dtype=torch.float64) / w.D)
+        ang = pos * inv[None, :]
+        return torch.cos(ang).float().contiguous(), torch.sin(ang).float().contiguous()
+
+    rope = (*tables(w.Nq, w.Nkv - w.Nq), *tables(w.Nkv, 0))
+    out = sage.quant_qk(q, k, v)
+    ws = torch.empty(max(sage.workspace_bytes(out.shape), 16), dtype=torch.uint8, device="cuda")
+
+    def timed(r):
+        for _ in range(args.warmup):
+            sage.quant_qk(q, k, v, out=out, workspace=ws, rope=r)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            sage.quant_qk(q, k, v, out=out, workspace=ws, rope=r)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    t_plain, t_rope = timed(None), timed(rope)
+    if sage.sync_status() != 0:
+        raise RuntimeError("device status error in the rotary quantizer run")
+    alg = 3 * w.B * w.H * (w.Nq + 2 * w.Nkv) * w.D  # one bf16 read + one 8-bit write per element
+    print(json.dumps({
+        "rotary_quantizer": w.name, "quant_ms": round(t_plain, 4), "quant_rope_ms": round(t_rope, 4),
+        "quant_GBps_alg": round(alg / (t_plain / 1e3) / 1e9, 1),
+        "quant_rope_GBps_alg": round(alg / (t_rope / 1e3) / 1e9, 1),
+        "table_bytes": 8 * (w.Nq + w.Nkv) * (w.D // 2)}), flush=True)
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args):
@@ -635,6 +684,8 @@ def main():
         run_block_sparse(args)
     elif args.w8a8:
         run_w8a8(args)
+    elif args.rope:
+        run_rope(args)
     else:
         run_ours(args)
 

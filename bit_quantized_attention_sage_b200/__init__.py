@@ -63,6 +63,8 @@ def lib():
         L.sage_quant_workspace_bytes.argtypes = [P]
         L.sage_quant_qk.restype = I
         L.sage_quant_qk.argtypes = [P, P, P, P, P, P, SZ, P]
+        L.sage_quant_qk_rope.restype = I
+        L.sage_quant_qk_rope.argtypes = [P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.sage_quant_qk_noalloc.restype = I
         L.sage_quant_qk_noalloc.argtypes = [P, P, P, P, P, P]
         L.sage_attn_fwd.restype = I
@@ -151,8 +153,12 @@ class QuantizedQKV:
         return t.view(torch.float32).view(s.B, s.H, s.D)
 
 
-def quant_qk(q, k, v, out=None, workspace=None, stream=None):
-    """sage_quant_qk on bf16 CUDA tensors [B, H, N, D]; returns QuantizedQKV."""
+def quant_qk(q, k, v, out=None, workspace=None, stream=None, rope=None):
+    """sage_quant_qk on bf16 CUDA tensors [B, H, N, D]; returns QuantizedQKV.
+
+    rope: None, or (q_cos, q_sin, k_cos, k_sin), contiguous float32 CUDA
+    tensors [Nq, D/2] and [Nkv, D/2]: Q and K are rotated pairwise by those
+    angles before quantization (sage_quant_qk_rope)."""
     import torch
     B, H, Nq, D = q.shape
     Nkv = k.shape[2]
@@ -160,15 +166,28 @@ def quant_qk(q, k, v, out=None, workspace=None, stream=None):
     for t in (q, k, v):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if rope is not None:
+        for t, n in zip(rope, (Nq, Nq, Nkv, Nkv)):
+            if (t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous()
+                    or tuple(t.shape) != (n, D // 2)):
+                raise ValueError("rotation tables must be contiguous float32 CUDA tensors "
+                                 "[Nq, D/2], [Nq, D/2], [Nkv, D/2], [Nkv, D/2]")
     if out is None:
         out = QuantizedQKV(shape, q.device)
     ws_need = workspace_bytes(shape)
     if workspace is None:
         workspace = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=q.device)
     qs = out.struct()
-    _check(lib().sage_quant_qk(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape), ctypes.byref(qs),
-                               _ptr(workspace), workspace.numel(), _stream(stream)),
-           "sage_quant_qk")
+    if rope is None:
+        _check(lib().sage_quant_qk(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape),
+                                   ctypes.byref(qs), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)),
+               "sage_quant_qk")
+    else:
+        _check(lib().sage_quant_qk_rope(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape),
+                                        *[_ptr(t) for t in rope], ctypes.byref(qs),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+               "sage_quant_qk_rope")
     return out
 
 

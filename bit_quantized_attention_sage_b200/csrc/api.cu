@@ -267,13 +267,18 @@ SAGE_EXPORT size_t sage_quant_workspace_bytes(const sage_shape* shape) {
   return shape_ok(shape) ? workspace_bytes(shape) : 0;
 }
 
-SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, const void* v_bf16,
-                                      const sage_shape* shape, const sage_qkv_quant* out,
-                                      void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+sage_status quant_common(const void* q_bf16, const void* k_bf16, const void* v_bf16,
+                         const sage_shape* shape, const float* const rope[4],
+                         const sage_qkv_quant* out, void* workspace, size_t ws_bytes,
+                         void* stream) {
   if (!shape_ok(shape) || !qkv_ok(out)) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(workspace))
     return SAGE_ERR_INVALID_ARG;
   if (ws_bytes < workspace_bytes(shape)) return SAGE_ERR_INVALID_ARG;
+  if (rope)
+    for (int i = 0; i < 4; i++)
+      if (!aligned16(rope[i])) return SAGE_ERR_INVALID_ARG;
   if (!device_state()) return SAGE_ERR_CUDA;
   QuantArgs a{};
   a.q = static_cast<const uint16_t*>(q_bf16);
@@ -294,8 +299,34 @@ SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, co
   a.ws_ksum = static_cast<double*>(workspace);
   a.ws_vmax = reinterpret_cast<float*>(static_cast<char*>(workspace) + cells * 8);
   a.ws_vinv = reinterpret_cast<float*>(static_cast<char*>(workspace) + cells * 12);
+  if (rope) {
+    a.q_cos = rope[0];
+    a.q_sin = rope[1];
+    a.k_cos = rope[2];
+    a.k_sin = rope[3];
+  }
   return launch_quant(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
                                                                            : SAGE_ERR_CUDA;
+}
+}  // namespace
+
+SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, const void* v_bf16,
+                                      const sage_shape* shape, const sage_qkv_quant* out,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  return quant_common(q_bf16, k_bf16, v_bf16, shape, nullptr, out, workspace, ws_bytes, stream);
+}
+
+SAGE_EXPORT sage_status sage_quant_qk_rope(const void* q_bf16, const void* k_bf16,
+                                           const void* v_bf16, const sage_shape* shape,
+                                           const float* q_cos, const float* q_sin,
+                                           const float* k_cos, const float* k_sin,
+                                           const sage_qkv_quant* out, void* workspace,
+                                           size_t ws_bytes, void* stream) {
+  const float* const rope[4] = {q_cos, q_sin, k_cos, k_sin};
+  // the rotary kernels put the 64-token blocks on the grid's y dimension
+  if (shape && shape_ok(shape) && (pad64(shape->Nq) / 64 > 65535 || pad64(shape->Nkv) / 64 > 65535))
+    return SAGE_ERR_UNSUPPORTED;
+  return quant_common(q_bf16, k_bf16, v_bf16, shape, rope, out, workspace, ws_bytes, stream);
 }
 
 namespace {

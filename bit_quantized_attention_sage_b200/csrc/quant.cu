@@ -19,6 +19,12 @@
 // Memory traffic: 16-byte vectorised bf16 loads; every fp32 operation is an
 // explicit IEEE round-to-nearest intrinsic so the codes match a plain CPU
 // implementation bit for bit.
+//
+// Rotary variant (sage_quant_qk_rope; the digest's RoPE Repositioning: the
+// cache holds features before RoPE, which is applied at their current
+// positions): Q and K are rotated in fp32 as they are loaded, channel pair
+// (2p, 2p+1) of token n by the caller's cos/sin[n][p], and quantized as
+// above; the K mean is that of the rotated keys.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -61,6 +67,32 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int i = 1; i < kThreads / 32; i++) r = fmaxf(r, red[i]);
   return r;
+}
+
+// Pair rotation (x0, x1) -> (x0 c - x1 s, x0 s + x1 c): each product and
+// each fma rounded once.
+__device__ __forceinline__ void rot_pair(float& x0, float& x1, float c, float s) {
+  const float t = __fmul_rn(x1, s), u = __fmul_rn(x1, c);
+  const float r0 = __fmaf_rn(x0, c, -t), r1 = __fmaf_rn(x0, s, u);
+  x0 = r0;
+  x1 = r1;
+}
+
+// The cos / sin of the 4 channel pairs of one 8-channel chunk (channels
+// col..col+7 of token `tok`; tables [N][D/2], 16-byte aligned rows).
+template <int D>
+__device__ __forceinline__ void rope_load(const float* cs, const float* sn, int tok, int col,
+                                          float4& c, float4& s) {
+  const size_t o = static_cast<size_t>(tok) * (D / 2) + col / 2;
+  c = __ldg(reinterpret_cast<const float4*>(cs + o));
+  s = __ldg(reinterpret_cast<const float4*>(sn + o));
+}
+
+__device__ __forceinline__ void rope_apply(float (&x)[8], const float4& c, const float4& s) {
+  rot_pair(x[0], x[1], c.x, s.x);
+  rot_pair(x[2], x[3], c.y, s.y);
+  rot_pair(x[4], x[5], c.z, s.z);
+  rot_pair(x[6], x[7], c.w, s.w);
 }
 
 __device__ __forceinline__ int8_t q_i8(float x, float inv) {
@@ -107,16 +139,21 @@ __device__ __forceinline__ void quant_block_store(float (&x)[CH][8], int valid, 
   if (threadIdx.x == 0) *scale_out = scale;
 }
 
-template <int D>
+template <int D, bool ROPE>
 __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;  // chunks per thread
   __shared__ float red[kThreads / 32];
-  __shared__ __align__(16) uint16_t ks[kBlk * D];
-  __shared__ __align__(16) uint16_t vsm[kBlk * D];
+  // staging of one 64-token block: bf16 K then bf16 V; or (rotary variant)
+  // bf16 V, then the rotated K in fp32
+  __shared__ __align__(16) uint32_t stage[kBlk * D];
+  uint16_t* ks = reinterpret_cast<uint16_t*>(stage);
+  uint16_t* vsm = ks + kBlk * D;
 
-  const int blk = blockIdx.x;
-  const int bh = blockIdx.y;
+  // rotary variant: heads run fastest, so that the CTAs in flight share the
+  // table rows of their tokens through L2
+  const int blk = ROPE ? blockIdx.y : blockIdx.x;
+  const int bh = ROPE ? blockIdx.x : blockIdx.y;
   const int nqb = (a.Nq + kBlk - 1) / kBlk;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
 
@@ -125,20 +162,84 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
     const uint4* src = reinterpret_cast<const uint4*>(
         a.q + (static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(blk) * kBlk) * D);
     float x[CH][8];
+    uint4 u[CH];
+    float4 rc[ROPE ? CH : 1], rs[ROPE ? CH : 1];  // all loads first, then the math
 #pragma unroll
     for (int c = 0; c < CH; c++) {
       const int chunk = c * kThreads + threadIdx.x;
       const int row = chunk / kChunksPerRow;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (row < valid) u = __ldg(src + chunk);
-      unpack8(u, x[c]);
+      u[c] = make_uint4(0, 0, 0, 0);
+      if (row < valid) u[c] = __ldg(src + chunk);
+      if constexpr (ROPE) {
+        rc[c] = rs[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (row < valid)
+          rope_load<D>(a.q_cos, a.q_sin, blk * kBlk + row, (chunk % kChunksPerRow) * 8, rc[c], rs[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      unpack8(u[c], x[c]);
+      if constexpr (ROPE) rope_apply(x[c], rc[c], rs[c]);
     }
     int8_t* codes = a.q_i8 + (static_cast<size_t>(bh) * nqb + blk) * kBlk * D;
     quant_block_store<D, CH>(x, valid, codes, a.q_scale + static_cast<size_t>(bh) * nqb + blk,
                              red);
   }
 
-  if (blk < nkb) {  // K block sums and V block maxima
+  if (blk < nkb && ROPE) {  // V block maxima, then sums of the rotated K block
+    const int valid = min(kBlk, a.Nkv - blk * kBlk);
+    const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
+    const uint4* ksrc = reinterpret_cast<const uint4*>(a.k + base);
+    const uint4* vsrc = reinterpret_cast<const uint4*>(a.v + base);
+    const size_t ws = (static_cast<size_t>(bh) * nkb + blk) * D;
+    const int t = threadIdx.x;
+    // every load of the block first: K chunks and their angles (kept in
+    // registers), V chunks (staged)
+    uint4 ku[CH];
+    float4 kc[CH], ksn[CH];
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      if (row < valid) {
+        ku[c] = __ldg(ksrc + chunk);
+        rope_load<D>(a.k_cos, a.k_sin, blk * kBlk + row, (chunk % kChunksPerRow) * 8, kc[c], ksn[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      if (chunk / kChunksPerRow < valid) reinterpret_cast<uint4*>(ks)[chunk] = __ldg(vsrc + chunk);
+    }
+    __syncthreads();
+    if (t >= D && t < 2 * D) {  // max |V| of channel t - D
+      const int d = t - D;
+      float m = 0.0f;
+      for (int r = 0; r < valid; r++)
+        m = fmaxf(m, fabsf(__uint_as_float(static_cast<uint32_t>(ks[r * D + d]) << 16)));
+      a.ws_vmax[ws + d] = m;
+    }
+    __syncthreads();  // V is read; the rotated K overwrites the staging area
+    float* kf = reinterpret_cast<float*>(stage);
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      const int row = chunk / kChunksPerRow;
+      if (row < valid) {
+        float x[8];
+        unpack8(ku[c], x);
+        rope_apply(x, kc[c], ksn[c]);
+        reinterpret_cast<float4*>(kf)[2 * chunk] = make_float4(x[0], x[1], x[2], x[3]);
+        reinterpret_cast<float4*>(kf)[2 * chunk + 1] = make_float4(x[4], x[5], x[6], x[7]);
+      }
+    }
+    __syncthreads();
+    if (t < D) {  // fp64 sum of channel t, ascending token order
+      double s = 0.0;
+      for (int r = 0; r < valid; r++) s = __dadd_rn(s, static_cast<double>(kf[r * D + t]));
+      a.ws_ksum[ws + t] = s;
+    }
+  } else if (blk < nkb) {  // K block sums and V block maxima
     const int valid = min(kBlk, a.Nkv - blk * kBlk);
     const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
     const uint4* ksrc = reinterpret_cast<const uint4*>(a.k + base);
@@ -213,14 +314,14 @@ __global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
   }
 }
 
-template <int D>
+template <int D, bool ROPE>
 __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;
   __shared__ float red[kThreads / 32];
 
-  const int blk = blockIdx.x;
-  const int bh = blockIdx.y;
+  const int blk = ROPE ? blockIdx.y : blockIdx.x;  // as in pass 1
+  const int bh = ROPE ? blockIdx.x : blockIdx.y;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
   const int nkv_pad = nkb * kBlk;
   const int valid = min(kBlk, a.Nkv - blk * kBlk);
@@ -243,14 +344,25 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
     const uint4* src = reinterpret_cast<const uint4*>(a.k + base);
     const float* mu = a.k_mean + static_cast<size_t>(bh) * D;
     float x[CH][8];
+    uint4 u[CH];
+    float4 rc[ROPE ? CH : 1], rs[ROPE ? CH : 1];  // all loads first, then the math
 #pragma unroll
     for (int c = 0; c < CH; c++) {
       const int chunk = c * kThreads + threadIdx.x;
       const int row = chunk / kChunksPerRow;
-      const int col = (chunk % kChunksPerRow) * 8;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (row < valid) u = __ldg(src + chunk);
-      unpack8(u, x[c]);
+      u[c] = make_uint4(0, 0, 0, 0);
+      if (row < valid) u[c] = __ldg(src + chunk);
+      if constexpr (ROPE) {
+        rc[c] = rs[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (row < valid)
+          rope_load<D>(a.k_cos, a.k_sin, blk * kBlk + row, (chunk % kChunksPerRow) * 8, rc[c], rs[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int col = ((c * kThreads + threadIdx.x) % kChunksPerRow) * 8;
+      unpack8(u[c], x[c]);
+      if constexpr (ROPE) rope_apply(x[c], rc[c], rs[c]);
 #pragma unroll
       for (int e = 0; e < 8; e++) x[c][e] = __fsub_rn(x[c][e], __ldg(mu + col + e));
     }
@@ -298,14 +410,21 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream) {
   dim3 g1(nqb > nkb ? nqb : nkb, a.BH);
   dim3 g2(nkb, a.BH);
   dim3 gf(a.D / kFinCh, a.BH);
+  const bool rope = a.q_cos != nullptr;
+  const dim3 r1(a.BH, g1.x), r2(a.BH, g2.x);  // rotary variant: heads fastest
+  if (rope && g1.x > 65535) return cudaErrorInvalidConfiguration;
   if (a.D == 128) {
-    k_quant_pass1<128><<<g1, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass1<128, true><<<r1, kThreads, 0, stream>>>(a);
+    else k_quant_pass1<128, false><<<g1, kThreads, 0, stream>>>(a);
     k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
-    k_quant_pass2<128><<<g2, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass2<128, true><<<r2, kThreads, 0, stream>>>(a);
+    else k_quant_pass2<128, false><<<g2, kThreads, 0, stream>>>(a);
   } else {
-    k_quant_pass1<64><<<g1, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass1<64, true><<<r1, kThreads, 0, stream>>>(a);
+    else k_quant_pass1<64, false><<<g1, kThreads, 0, stream>>>(a);
     k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
-    k_quant_pass2<64><<<g2, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass2<64, true><<<r2, kThreads, 0, stream>>>(a);
+    else k_quant_pass2<64, false><<<g2, kThreads, 0, stream>>>(a);
   }
   return cudaGetLastError();
 }

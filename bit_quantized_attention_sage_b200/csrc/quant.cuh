@@ -22,6 +22,12 @@ struct QuantArgs {
   double* ws_ksum;  // [BH, nkb, D] fp64 per-block K channel sums
   float* ws_vmax;   // [BH, nkb, D] per-block V channel maxima
   float* ws_vinv;   // [BH, D] 448 / channel absmax (0 for an all-zero channel)
+  // rotation tables [Nq, D/2] / [Nkv, D/2] (cos, sin per token and channel
+  // pair), shared by all (b, h); all four null: no rotation
+  const float* q_cos;
+  const float* q_sin;
+  const float* k_cos;
+  const float* k_sin;
 };
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream);

@@ -132,6 +132,37 @@ sage_status sage_quant_qk(const void *q_bf16, const void *k_bf16, const void *v_
                           const sage_shape *shape, const sage_qkv_quant *out,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* sage_quant_qk with rotary position embedding applied to Q and K first.
+ *
+ * The pages cache features before RoPE and apply RoPE at their current,
+ * re-based positions whenever the streaming window slides ("Vidu S1" digest,
+ * Infra, RoPE Repositioning).  This call fuses that rotation into the
+ * quantizer, so the cache can stay un-rotated in bf16.
+ *
+ *   Rotation: for every (b, h), token n and channel pair (2p, 2p+1), p < D/2,
+ *     with c = cos[n][p], s = sin[n][p] from the tables below:
+ *       x'[2p]   = fma(x[2p], c, -fp32(x[2p+1] * s))
+ *       x'[2p+1] = fma(x[2p], s,  fp32(x[2p+1] * c))
+ *     (each product and fma rounded once to fp32; the result is not rounded
+ *     to bf16).  Per-pair angles cover 1D and multi-axis (frame / height /
+ *     width) RoPE alike.
+ *   Then exactly the steps of sage_quant_qk on Q' and K' (the K mean is that
+ *   of the rotated keys); V is not rotated.
+ *
+ *   q_cos, q_sin: device f32 [Nq, D/2]; k_cos, k_sin: device f32 [Nkv, D/2];
+ *     row n holds token n's values; shared by every batch entry and head;
+ *     read only; 16-byte aligned.
+ *   Other arguments and outputs: as for sage_quant_qk.
+ *
+ * Errors: SAGE_ERR_INVALID_ARG for a null or misaligned table and for every
+ * case sage_quant_qk rejects; SAGE_ERR_UNSUPPORTED for Nq or Nkv above
+ * 65535 * 64 = 4194240 tokens; SAGE_ERR_CUDA if a launch fails. */
+sage_status sage_quant_qk_rope(const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                               const sage_shape *shape, const float *q_cos,
+                               const float *q_sin, const float *k_cos, const float *k_sin,
+                               const sage_qkv_quant *out, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
 /* Size of the fixed device scratch array sage_quant_qk_noalloc uses: 16 MiB
  * on every GPU that loads the library, held until the process exits. */
 #define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

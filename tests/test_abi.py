@@ -104,3 +104,27 @@ def test_block_sparse_and_w8a8_arguments_are_rejected_before_any_launch(L):
     assert L.sage_w8a8_gemm(p, p, p, p, 8, 128, 200, p, None, None) == 1
     assert L.sage_w8a8_gemm(p, p, p, p, 8, 64, 128, p, None, None) == 1
     assert L.sage_w8a8_gemm(ctypes.c_void_p(4100), p, p, p, 8, 128, 128, p, None, None) == 1
+
+
+def test_rope_quantizer_arguments_are_rejected_before_any_launch(L):
+    s = sage.make_shape(1, 1, 64, 64, 128)
+    ok = sage._QKV(*([16 * 1024] * 7))
+    p = ctypes.c_void_p(4096)
+    ws = L.sage_quant_workspace_bytes(ctypes.byref(s))
+    tabs = [p, p, p, p]
+    # every table is required and 16-byte aligned
+    for i in range(4):
+        t = list(tabs)
+        t[i] = None
+        assert L.sage_quant_qk_rope(p, p, p, ctypes.byref(s), *t, ctypes.byref(ok), p, ws,
+                                    None) == 1
+        t[i] = ctypes.c_void_p(4100)
+        assert L.sage_quant_qk_rope(p, p, p, ctypes.byref(s), *t, ctypes.byref(ok), p, ws,
+                                    None) == 1
+    # more than 65535 blocks of 64 tokens is unsupported
+    big = sage.make_shape(1, 1, 64, 65535 * 64 + 1, 128)
+    assert L.sage_quant_qk_rope(p, p, p, ctypes.byref(big), *tabs, ctypes.byref(ok), p, 1 << 40,
+                                None) == 2
+    # the checks of sage_quant_qk still apply (workspace too small)
+    assert L.sage_quant_qk_rope(p, p, p, ctypes.byref(s), *tabs, ctypes.byref(ok), p, ws - 1,
+                                None) == 1
