@@ -121,6 +121,20 @@ bool encode_u8_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [rows][cols] matrix, row-major, box0 columns x box1 rows.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                    uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box0, box1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_maps(const sage_qkv_quant* q, const sage_shape* s, AttnMaps* m) {
   const uint64_t bh = static_cast<uint64_t>(s->B) * s->H, D = s->D;
   const CUtensorMapSwizzle swqk =
@@ -229,7 +243,8 @@ SAGE_EXPORT sage_status sage_w8a8_gemm(const int8_t* xq, const float* sx, const 
   if (!d) return SAGE_ERR_CUDA;
   W8a8Maps maps;
   if (!encode_u8_3d(&maps.x, xq, K, M, 1, kW8a8Group, kW8a8BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_u8_3d(&maps.w, wq, K, N, 1, kW8a8Group, kW8a8BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      !encode_u8_3d(&maps.w, wq, K, N, 1, kW8a8Group, kW8a8BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bf16_2d(&maps.y, y_bf16, N, M, 64, kW8a8BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return SAGE_ERR_CUDA;
   W8a8Params p{};
   p.M = static_cast<int>(M);

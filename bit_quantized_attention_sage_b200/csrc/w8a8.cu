@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(256) k_w8a8_quant_weight(const uint16_t* __res
 struct alignas(1024) GemmSmem {
   uint8_t x[NS][GPS][BM * G];  // int8 X tiles [group][128 rows][128 channels]
   uint8_t w[NS][GPS][BN * G];  // int8 W tiles [group][128 out channels][128 channels]
+  // bf16 Y tile staging for the TMA store, one buffer per column part:
+  // [128 rows][64 columns], 128-byte swizzled like the tensor map
+  uint8_t ystage[kPromWarps / 4][BM * kPromCols * 2];
   uint8_t seed[128];           // f16 broadcast tile of the accumulator seed MMA
   uint64_t full[NS], empty[NS];
   uint64_t acc_full[NPAIR], acc_free[NPAIR];
@@ -156,6 +159,38 @@ struct alignas(1024) GemmSmem {
   int abort;
 };
 static_assert(sizeof(GemmSmem) <= 227 * 1024, "shared memory of one CTA");
+
+// TMA store of one 2-D tile from shared memory (no multicast), and the
+// bulk-group bookkeeping of the issuing thread.
+__device__ __forceinline__ void tma_store_2d(const void* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every committed store has finished reading shared memory / has completed
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Named barrier of `n` threads; the _or form returns, to every thread, whether
+// `pred` held for any of them.
+__device__ __forceinline__ void bar_sync_n(int id, int n) {
+  asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool bar_or_n(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
                                           int site) {
@@ -271,10 +306,15 @@ __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&v)[C]) {
 
 // Promotion warps: rows 32 q + lane, columns kPromCols * c .. + kPromCols - 1
 // of each tile (q = lane quadrant, c = column part).
-__device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, uint32_t tmem,
-                                             const TileSched& ts, int ngroups, const WaitCtx& w) {
+__device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Maps& maps, const W8a8Params& p,
+                                             uint32_t tmem, const TileSched& ts, int ngroups,
+                                             const WaitCtx& w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3, part = (warp - kFirstProm) >> 2;
+  // the first warp of a column part issues its TMA stores
+  const bool storer = ((warp - kFirstProm) & 3) == 0 && lane == 0;
+  const int bar_id = 1 + part;  // named barrier of the part's 4 warps (0 is __syncthreads)
+  uint8_t* stg = s.ystage[part];
   const int r = quad * 32 + lane;
   const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16) + part * kPromCols;
   const float2 nb2 = make_float2(-kBias, -kBias);
@@ -287,9 +327,10 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
   if (lane == 0)
     for (int pr = 0; pr < NPAIR; pr++) mbar_arrive(&s.acc_free[pr]);
 
+  bool ok = true;
   int J = 0;
   for (int i = 0; i < ntile; i++) {
-    const int m = ts.m0(i) + r, n0 = ts.n0(i);
+    const int m0 = ts.m0(i), m = m0 + r, n0 = ts.n0(i);
     const bool valid = m < p.M;
     const float* sxr = p.sx + static_cast<size_t>(valid ? m : 0) * ngroups;
     const float* swr = p.sw + static_cast<size_t>(n0 / BN) * ngroups;
@@ -299,7 +340,10 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
     float sxn = valid ? __ldg(sxr) : 0.0f, swn = __ldg(swr);
     for (int j = 0; j < ts.nsteps; j++, J++) {
       const int pr = J % NPAIR;
-      if (!warp_wait(&s.acc_full[pr], (J / NPAIR) & 1, w, kSitePromFull)) return;
+      if (!warp_wait(&s.acc_full[pr], (J / NPAIR) & 1, w, kSitePromFull)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const bool reuse = J + NPAIR < total;  // a later step fills this pair again
       const int ng = min(GPS, ngroups - j * GPS);
@@ -326,26 +370,40 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Params& p, u
         }
       }
     }
-    // epilogue of this tile (the issuers already run the next tile's steps)
-    if (!valid) continue;
-    const size_t orow = static_cast<size_t>(m) * p.N + n0 + part * kPromCols;
-    uint32_t packed[kPromCols / 2];
+    // epilogue of this tile (the issuers already run the next tile's steps):
+    // bf16 rows into the part's staging buffer, then one TMA store of the
+    // 128 x 64 tile (rows past M are clipped by the tensor map)
+    if (storer) bulk_wait_read_all();  // the previous tile's store has read the buffer
+    bar_sync_n(bar_id, 128);
+    if (ok) {
+      uint8_t* row = stg + r * (kPromCols * 2);
 #pragma unroll
-    for (int e = 0; e < kPromCols / 2; e++) {
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(y[e].x, y[e].y);
-      packed[e] = *reinterpret_cast<uint32_t*>(&h2);
+      for (int c = 0; c < kPromCols / 8; c++) {  // 16-byte chunk c of the row, swizzled
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4 * c + e].x, y[4 * c + e].y);
+          pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
     }
-    uint4* dst = reinterpret_cast<uint4*>(p.y + orow);
-#pragma unroll
-    for (int e = 0; e < kPromCols / 8; e++)
-      dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-    if (p.y_f32) {
-      float4* d32 = reinterpret_cast<float4*>(p.y_f32 + orow);
+    fence_proxy_async_smem();
+    // every warp of the part leaves together after a timeout anywhere
+    if (bar_or_n(bar_id, 128, !ok || *w.abort != 0)) break;
+    if (storer) {
+      tma_store_2d(&maps.y, stg, n0 + part * kPromCols, m0);
+      bulk_commit();
+    }
+    if (valid && p.y_f32) {
+      float4* d32 = reinterpret_cast<float4*>(p.y_f32 + static_cast<size_t>(m) * p.N + n0 +
+                                              part * kPromCols);
 #pragma unroll
       for (int e = 0; e < kPromCols / 4; e++)
         d32[e] = make_float4(y[2 * e].x, y[2 * e].y, y[2 * e + 1].x, y[2 * e + 1].y);
     }
   }
+  if (storer) bulk_wait_all();  // the stores are complete before the CTA exits
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -392,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kFirstProm) {
     if (lane == 0) gemm_mma(s, tmem, ts, ngroups, w, warp - 1);
   } else {
-    gemm_promote(s, p, tmem, ts, ngroups, w);
+    gemm_promote(s, maps, p, tmem, ts, ngroups, w);
   }
   __syncwarp();
   tc_fence_before();

@@ -27,6 +27,7 @@ struct W8a8Params {
 struct W8a8Maps {
   CUtensorMap x;  // int8 [M][K], box 128 x 128
   CUtensorMap w;  // int8 [N][K], box 128 x 128
+  CUtensorMap y;  // bf16 [M][N], box 64 columns x 128 rows, 128-byte swizzle (stores)
 };
 
 cudaError_t w8a8_prepare();
