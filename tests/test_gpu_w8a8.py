@@ -79,3 +79,19 @@ def test_dit_shapes_sampled(M, N, K):
     rng = np.random.default_rng(M + N)
     rows = np.sort(np.concatenate([[0, M - 1], rng.choice(M, 30, replace=False)]))
     check(bits((M, K), 7, outliers=8), bits((N, K), 8), rows=np.unique(rows))
+
+
+def test_bf16_output_alone():
+    # without the optional fp32 output (the layer's usual call): the bf16 tile
+    # stores alone, on a shape with an M tail and several tiles per CTA
+    M, N, K = 2500, 1152, 384
+    x, w = bits((M, K), 21, outliers=2), bits((N, K), 22)
+    xq, sx = sage.w8a8_quant_act(dev(x))
+    wq, sw = sage.w8a8_quant_weight(dev(w))
+    y = sage.w8a8_gemm(xq, sx, wq, sw)
+    assert sage.sync_status() == 0
+    rxq, rsx = oracle.w8a8_quant_act(x)
+    rwq, rsw = oracle.w8a8_quant_weight(w)
+    ry = oracle.w8a8_gemm_rows(rxq, rsx, rwq, rsw, np.arange(M))
+    gotb = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(gotb, synth.f32_to_bf16_bits(ry))
