@@ -160,7 +160,7 @@ struct alignas(1024) GemmSmem {
 };
 static_assert(sizeof(GemmSmem) <= 227 * 1024, "shared memory of one CTA");
 
-// TMA store of one 2-D tile from shared memory (no multicast), and the
+// TMA store of one 2-D tile from this CTA's shared memory, and the
 // bulk-group bookkeeping of the issuing thread.
 __device__ __forceinline__ void tma_store_2d(const void* map, const void* src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
