@@ -66,6 +66,12 @@ def lib():
         L.orc_attn_rows_identity_bs.restype = i32
         L.orc_attn_rows_identity_bs.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
                                                 P, i64, i64, P, i64, P, P, i32]
+        L.orc_attn_rows_split.restype = i32
+        L.orc_attn_rows_split.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
+                                          i32, i64, P, i64, P, P, P, i32]
+        L.orc_attn_rows_identity_split.restype = i32
+        L.orc_attn_rows_identity_split.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64, i32, i64,
+                                                   P, i64, P, P, i32]
         L.orc_w8a8_quant_act.restype = i32
         L.orc_w8a8_quant_act.argtypes = [P, i64, i64, P, P]
         L.orc_w8a8_quant_weight.restype = i32
@@ -176,11 +182,14 @@ def _block_mask(block_mask, nkv, tkv):
 
 
 def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
-              threads=None, block_mask=None):
+              threads=None, block_mask=None, kv_splits=1):
     """Same-quantization attention of one quantized head on the given rows.
 
     block_mask: optional uint8 [ceil(Nq / 128), ceil(Nkv / tkv)] of this head;
     query row i visits KV tile t only if block_mask[i // 128, t] != 0.
+    kv_splits > 1: the split-KV form (``orc_attn_rows_split``): the KV tiles of
+    each 128-query tile in that many ranges, each its own online softmax,
+    merged (not combined with a block mask).
     Returns (o [n, D] float64 of the fp32 recipe, slack [n, D] or None, lse [n]).
     """
     rows = np.ascontiguousarray(rows, np.int64)
@@ -194,19 +203,29 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
     qs = np.ascontiguousarray(qh["qs"])
     ks = np.ascontiguousarray(qh["ks"])
     vs = np.ascontiguousarray(qh["vs"])
-    bptr, bq, n_kt, _keep = _block_mask(block_mask, qh["nkv"], tkv)
-    rc = lib().orc_attn_rows_bs(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
-                                qh["nq"], qh["nkv"], D, mask, mb, tkv, eps, bptr, bq, n_kt,
-                                _p(rows), n, _p(o), _p(slack) if slack is not None else None,
-                                _p(lse), _threads(threads))
+    if kv_splits > 1:
+        if block_mask is not None:
+            raise ValueError("kv_splits and block_mask are not combined")
+        rc = lib().orc_attn_rows_split(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
+                                       qh["nq"], qh["nkv"], D, mask, mb, tkv, eps, kv_splits, BQ,
+                                       _p(rows), n, _p(o),
+                                       _p(slack) if slack is not None else None, _p(lse),
+                                       _threads(threads))
+    else:
+        bptr, bq, n_kt, _keep = _block_mask(block_mask, qh["nkv"], tkv)
+        rc = lib().orc_attn_rows_bs(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
+                                    qh["nq"], qh["nkv"], D, mask, mb, tkv, eps, bptr, bq, n_kt,
+                                    _p(rows), n, _p(o), _p(slack) if slack is not None else None,
+                                    _p(lse), _threads(threads))
     if rc:
         raise ValueError("orc_attn_rows: invalid arguments")
     return o, slack, lse
 
 
 def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=None,
-                       block_mask=None):
-    """The oracle's tiled loop with identity quantizers, fp64 throughout."""
+                       block_mask=None, kv_splits=1):
+    """The oracle's tiled loop with identity quantizers, fp64 throughout
+    (kv_splits > 1: the split-KV form, as for attn_rows)."""
     q = np.ascontiguousarray(q, np.float64)
     k = np.ascontiguousarray(k, np.float64)
     v = np.ascontiguousarray(v, np.float64)
@@ -214,10 +233,17 @@ def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=Non
     n, D = rows.size, q.shape[1]
     o = np.empty((n, D), np.float64)
     lse = np.empty(n, np.float64)
-    bptr, bq, n_kt, _keep = _block_mask(block_mask, k.shape[0], tkv)
-    rc = lib().orc_attn_rows_identity_bs(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
-                                         mask, mb, tkv, bptr, bq, n_kt, _p(rows), n, _p(o),
-                                         _p(lse), _threads(threads))
+    if kv_splits > 1:
+        if block_mask is not None:
+            raise ValueError("kv_splits and block_mask are not combined")
+        rc = lib().orc_attn_rows_identity_split(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
+                                                mask, mb, tkv, kv_splits, BQ, _p(rows), n, _p(o),
+                                                _p(lse), _threads(threads))
+    else:
+        bptr, bq, n_kt, _keep = _block_mask(block_mask, k.shape[0], tkv)
+        rc = lib().orc_attn_rows_identity_bs(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
+                                             mask, mb, tkv, bptr, bq, n_kt, _p(rows), n, _p(o),
+                                             _p(lse), _threads(threads))
     if rc:
         raise ValueError("orc_attn_rows_identity: invalid arguments")
     return o, lse

@@ -380,6 +380,9 @@ typedef struct {
      * visited by query row i only if bmask[(i / bq) * n_kt + t] != 0 */
     const uint8_t *bmask;
     long bq, n_kt;
+    /* split-KV form (see attend_row): number of KV ranges, <= 1 for none;
+     * bq is then the query tile height */
+    int splits;
 } attn_job;
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
@@ -418,32 +421,37 @@ static double e4m3_flip_gap(double y, double eps)
  *   O     = O_acc * vs[d] / l;  lse = (m + log2(l) - 8) * ln 2.
  * Identity mode: t_ij = (q_i . k_j) * log2(e)/sqrt(D), w = p, all fp64.
  */
-static void attend_row(const attn_job *J, long r)
-{
-    const long i = J->rows[r];
-    const int D = J->D;
-    const long lim = orc_row_limit(i, J->nq, J->nkv, J->mask, J->mb);
-    const long tkv = J->tkv;
-    double *o = J->o + r * D;
-    double *sl = J->slack ? J->slack + r * D : NULL;
-    double *acc = (double *)calloc((size_t)D, sizeof(double));
-    double *sacc = (double *)calloc((size_t)D, sizeof(double));
-    int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)tkv);
-    float *c = (float *)malloc(sizeof(float) * (size_t)tkv);
-    double *t = (double *)malloc(sizeof(double) * (size_t)tkv);
+/* Online softmax of query row i over the KV tiles [t_begin, t_end) (keys
+ * below lim only), in ascending order: on return o holds the unnormalized
+ * sum of P.V in the units of the final running maximum (m, or mf and lf in
+ * quantized mode), sl its rounding slack.  o and sl start at zero. */
+typedef struct {
+    double *o, *sl;
+    double m, l;
+    float mf, lf;
+} attn_part;
 
+static void attend_range(const attn_job *J, long i, long lim, long t_begin, long t_end,
+                         attn_part *P, double *acc, double *sacc, int32_t *S, float *c, double *t)
+{
+    const int D = J->D;
+    const long tkv = J->tkv;
+    double *o = P->o;
+    double *sl = P->sl;
     const double C64 = 1.4426950408889634 / sqrt((double)D); /* log2(e)/sqrt(D) */
     const float C0 = (float)C64;
     float sqC = 0.0f;
     if (!J->identity)
         sqC = J->qs[i / ORC_BLK] * C0;
-
     double m = -INFINITY, l = 0.0;
     float mf = -INFINITY, lf = 0.0f;
-    for (int d = 0; d < D; d++)
+    for (int d = 0; d < D; d++) {
         o[d] = 0.0;
+        if (sl)
+            sl[d] = 0.0;
+    }
 
-    for (long j0 = 0; j0 < lim; j0 += tkv) {
+    for (long j0 = t_begin * tkv; j0 < lim && j0 < t_end * tkv; j0 += tkv) {
         if (J->bmask && !J->bmask[(i / J->bq) * J->n_kt + j0 / tkv])
             continue; /* tile switched off by the block mask */
         long j1 = j0 + tkv < lim ? j0 + tkv : lim; /* visible keys of this tile */
@@ -518,6 +526,91 @@ static void attend_row(const attn_job *J, long r)
             l = l * alpha + rowsum;
         else
             lf = lf * (float)alpha + rowsum_f;
+    }
+    P->m = m;
+    P->l = l;
+    P->mf = mf;
+    P->lf = lf;
+}
+
+/* One query row.  Without KV splits: one online softmax over all the row's
+ * tiles.  With J->splits = S > 1 (the split-KV form of the device kernel):
+ * the KV tiles the row's 128-query tile visits, [0, nk) with nk set by the
+ * tile's last row, are cut into S contiguous ranges [floor(s nk / S),
+ * floor((s+1) nk / S)); each range runs its own online softmax; the partial
+ * results are merged with m = max_s m_s, a_s = exp2(m_s - m) (0 for an empty
+ * range), O = sum_s a_s O_s and l = sum_s a_s l_s (fp32, ascending s, each
+ * product and sum rounded once), then normalized as without splits. */
+static void attend_row(const attn_job *J, long r)
+{
+    const long i = J->rows[r];
+    const int D = J->D;
+    const long lim = orc_row_limit(i, J->nq, J->nkv, J->mask, J->mb);
+    const long tkv = J->tkv;
+    double *o = J->o + r * D;
+    double *sl = J->slack ? J->slack + r * D : NULL;
+    double *acc = (double *)calloc((size_t)D, sizeof(double));
+    double *sacc = (double *)calloc((size_t)D, sizeof(double));
+    int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)tkv);
+    float *c = (float *)malloc(sizeof(float) * (size_t)tkv);
+    double *t = (double *)malloc(sizeof(double) * (size_t)tkv);
+
+    double m = -INFINITY, l = 0.0;
+    float mf = -INFINITY, lf = 0.0f;
+    const int nsplit = J->splits > 1 ? J->splits : 1;
+    if (nsplit == 1) {
+        attn_part P = {o, sl, 0, 0, 0, 0};
+        attend_range(J, i, lim, 0, (lim + tkv - 1) / tkv, &P, acc, sacc, S, c, t);
+        m = P.m;
+        l = P.l;
+        mf = P.mf;
+        lf = P.lf;
+    } else {
+        /* tiles of the row's query tile: those of its last row */
+        const long qlast = (i / J->bq + 1) * J->bq - 1 < J->nq - 1 ? (i / J->bq + 1) * J->bq - 1
+                                                                  : J->nq - 1;
+        const long nk = (orc_row_limit(qlast, J->nq, J->nkv, J->mask, J->mb) + tkv - 1) / tkv;
+        double *po = (double *)calloc((size_t)D * nsplit, sizeof(double));
+        double *ps = (double *)calloc((size_t)D * nsplit, sizeof(double));
+        attn_part *parts = (attn_part *)calloc((size_t)nsplit, sizeof(attn_part));
+        for (int sp = 0; sp < nsplit; sp++) {
+            parts[sp].o = po + (size_t)sp * D;
+            parts[sp].sl = sl ? ps + (size_t)sp * D : NULL;
+            attend_range(J, i, lim, nk * sp / nsplit, nk * (sp + 1) / nsplit, &parts[sp],
+                         acc, sacc, S, c, t);
+        }
+        for (int d = 0; d < D; d++) {
+            o[d] = 0.0;
+            if (sl)
+                sl[d] = 0.0;
+        }
+        if (J->identity) {
+            for (int sp = 0; sp < nsplit; sp++)
+                if (parts[sp].m > m)
+                    m = parts[sp].m;
+            for (int sp = 0; sp < nsplit; sp++) {
+                double a = parts[sp].m == -INFINITY ? 0.0 : exp2(parts[sp].m - m);
+                for (int d = 0; d < D; d++)
+                    o[d] += a * parts[sp].o[d];
+                l += a * parts[sp].l;
+            }
+        } else {
+            for (int sp = 0; sp < nsplit; sp++)
+                if (parts[sp].mf > mf)
+                    mf = parts[sp].mf;
+            for (int sp = 0; sp < nsplit; sp++) {
+                float a = parts[sp].mf == -INFINITY ? 0.0f : exp2_f32(parts[sp].mf - mf);
+                for (int d = 0; d < D; d++) {
+                    o[d] += (double)a * parts[sp].o[d];
+                    if (sl)
+                        sl[d] += (double)a * parts[sp].sl[d];
+                }
+                lf = lf + a * parts[sp].lf;
+            }
+        }
+        free(po);
+        free(ps);
+        free(parts);
     }
     /* output; a row that sees no key at all (possible only with a block
      * mask) has no softmax: O = 0 and lse = -inf by definition */
@@ -684,6 +777,80 @@ int orc_attn_rows_identity_bs(const double *q, const double *k, const double *v,
 }
 
 /* Dense forms (no block mask). */
+/* Split-KV forms (attend_row): the KV tiles of each 128-query tile (bq rows)
+ * in `splits` contiguous ranges, each with its own online softmax, merged. */
+int orc_attn_rows_split(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
+                        const uint8_t *v8, const float *vs, long nq, long nkv, int D,
+                        int mask, long mb, long tkv, double eps, int splits, long bq,
+                        const long *rows, long nrows, double *o, double *slack, double *lse,
+                        int nthreads)
+{
+    if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0 || splits < 1 || bq <= 0)
+        return 1;
+    if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
+        return 1;
+    if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
+        return 1;
+    attn_job J = {0};
+    J.identity = 0;
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = mask;
+    J.mb = mb;
+    J.tkv = tkv;
+    J.eps = eps;
+    J.q8 = q8;
+    J.qs = qs;
+    J.k8 = k8;
+    J.ks = ks;
+    J.v8 = v8;
+    J.vs = vs;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.slack = slack;
+    J.lse = lse;
+    J.bq = bq;
+    J.splits = splits;
+    if (slack)
+        memset(slack, 0, sizeof(double) * (size_t)(nrows * D));
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
+}
+
+int orc_attn_rows_identity_split(const double *q, const double *k, const double *v,
+                                 long nq, long nkv, int D, int mask, long mb, long tkv,
+                                 int splits, long bq, const long *rows, long nrows, double *o,
+                                 double *lse, int nthreads)
+{
+    if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0 || splits < 1 || bq <= 0)
+        return 1;
+    if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
+        return 1;
+    if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
+        return 1;
+    attn_job J = {0};
+    J.identity = 1;
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = mask;
+    J.mb = mb;
+    J.tkv = tkv;
+    J.qd = q;
+    J.kd = k;
+    J.vd = v;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.lse = lse;
+    J.bq = bq;
+    J.splits = splits;
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
+}
+
 int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
                   const uint8_t *v8, const float *vs, long nq, long nkv, int D,
                   int mask, long mb, long tkv, double eps,
