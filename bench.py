@@ -35,7 +35,7 @@ from bit_quantized_attention_sage_b200 import synth  # noqa: E402
 
 METRIC = "quantized-attention TOPS at 32k/75k tokens (H=12/40, D=128); % of INT8/FP8 peak"
 UNIT = "TOPS"
-KERNELS_PER_STEP = 4  # quant pass1, finalize, pass2, attention
+KERNELS_PER_STEP = 4  # quant pass1, finalize, pass2, attention (+1 merge with KV splits)
 
 
 def parse():
@@ -169,10 +169,16 @@ def recorded_traffic():
 class Runner:
     """Device buffers and one step of the hot path for a workload."""
 
-    def __init__(self, w, seed_offset, device):
+    def __init__(self, w, seed_offset, device, kv_splits="auto"):
         import torch
         import bit_quantized_attention_sage_b200 as sage
         self.torch, self.sage, self.w = torch, sage, w
+        # split-KV attention where the query tiles alone would leave SMs idle
+        # (e.g. one streaming frame against a long cache); 1 for the video shapes
+        if kv_splits == "auto":
+            sms = torch.cuda.get_device_properties(device).multi_processor_count
+            kv_splits = sage.suggest_kv_splits(w.B, w.H, w.Nq, w.Nkv, sms)
+        self.kv_splits = int(kv_splits)
         wr = synth.Workload(w.name, w.B, w.H, w.Nq, w.Nkv, w.D, w.mask, w.mask_block,
                             w.k_offset_var, w.outlier_mag, w.seed + seed_offset)
         q, k, v = synth.full(wr)
@@ -192,6 +198,10 @@ class Runner:
         self.o = torch.empty((w.B, w.H, w.Nq, w.D), dtype=torch.bfloat16, device=device)
         self.h_o = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         self.stream = torch.cuda.current_stream()
+        self.split_ws = None
+        if self.kv_splits > 1:
+            self.split_ws = torch.empty(sage.attn_split_workspace_bytes(self.shape, self.kv_splits),
+                                        dtype=torch.uint8, device=device)
 
     def step(self, ev=None, bufs=None):
         s = self.sage
@@ -201,7 +211,8 @@ class Runner:
         s.quant_qk(q, k, v, out=self.qkv, workspace=self.ws, stream=self.stream)
         if ev is not None:
             ev[1].record(self.stream)
-        s.attn_fwd(self.qkv, self.w.mask, self.w.mask_block, out=o, stream=self.stream)
+        s.attn_fwd(self.qkv, self.w.mask, self.w.mask_block, out=o, stream=self.stream,
+                   kv_splits=self.kv_splits, workspace=self.split_ws)
         if ev is not None:
             ev[2].record(self.stream)
 
@@ -349,6 +360,7 @@ def run_ours(args):
     sage.lib()
     w = synth.WORKLOADS[args.workload]
     runner = Runner(w, 1000 * rank, device)
+    kv_splits = runner.kv_splits
     ops_rank = w.ops()
     pk = peaks()
 
@@ -383,7 +395,7 @@ def run_ours(args):
 
     value = ops_rank * world / (t["ms"] / 1e3) / 1e12
     achieved = ops_rank / (t["attn_ms"] / 1e3) / 1e12
-    traffic = recorded_traffic()
+    traffic = recorded_traffic() if kv_splits == 1 else None  # the dense kernel's record
     # algorithmic bytes of sage_quant_qk: read bf16 (2 B) and write one 8-bit
     # code (1 B) per element of Q, K and V, plus the scales and the K mean
     quant_bytes = 3 * w.B * w.H * (w.Nq + 2 * w.Nkv) * w.D + 4 * w.B * w.H * (
@@ -398,8 +410,12 @@ def run_ours(args):
                    "mask_block": w.mask_block, "ops_per_step_per_gpu": ops_rank,
                    "l2": "inputs (%.2f GB bf16 Q/K/V per GPU) larger than the 126 MB L2; no flush"
                          % in_gb,
-                   "parallelism": "replica per GPU (dp%d, no collective)" % world},
-        "roofline": {"bound": "tensor", "kernel": "k_attn (sage_attn_fwd)",
+                   "parallelism": "replica per GPU (dp%d, no collective)" % world,
+                   "kv_splits": kv_splits},
+        "roofline": {"bound": "tensor",
+                     "kernel": "k_attn (sage_attn_fwd)" if kv_splits == 1 else
+                               "k_attn_split + k_attn_merge (sage_attn_fwd_split, %d KV ranges)"
+                               % kv_splits,
                      "achieved": round(achieved, 2), "peak": round(pk["i8_sustained"], 1),
                      "unit": "TFLOP/s", "frac": round(achieved / pk["i8_sustained"], 4),
                      "peak_note": "8-bit dense = 2 x %s sustained cuBLAS bf16 (of %s)" % (
@@ -412,7 +428,7 @@ def run_ours(args):
                            "frac": round(quant_bytes / (t["quant_ms"] / 1e3) / 1e9 / pk["hbm"], 4),
                            "ms_per_step": round(t["quant_ms"], 4),
                            "algorithmic_bytes": quant_bytes},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (kv_splits > 1)) * args.steps,
         "clocks": clk,
         "e2e": e2e,
     }

@@ -13,6 +13,7 @@ One-line use, in place of a FlashAttention call on [B, H, N, D] bf16 tensors:
     o = attention(q, k, v, mask=("block_causal", 2040))   # streaming KV cache
 """
 import ctypes
+import math
 import os
 
 MASK_NONE, MASK_CAUSAL, MASK_BLOCK_CAUSAL = 0, 1, 2
@@ -69,6 +70,10 @@ def lib():
         L.sage_quant_qk_noalloc.argtypes = [P, P, P, P, P, P]
         L.sage_attn_fwd.restype = I
         L.sage_attn_fwd.argtypes = [P, P, I, I, P, P, P, P]
+        L.sage_attn_fwd_split.restype = I
+        L.sage_attn_fwd_split.argtypes = [P, P, I, I, I, P, SZ, P, P, P, P]
+        L.sage_attn_split_workspace_bytes.restype = SZ
+        L.sage_attn_split_workspace_bytes.argtypes = [P, I]
         L.sage_attn_fwd_block_sparse.restype = I
         L.sage_attn_fwd_block_sparse.argtypes = [P, P, I, I, P, P, P, P, P]
         L.sage_debug_qk_int32.restype = I
@@ -216,18 +221,63 @@ def block_mask_shape(B, H, Nq, Nkv):
     return (B, H, -(-Nq // 128), -(-Nkv // 128))
 
 
+def suggest_kv_splits(B, H, Nq, Nkv, sm_count, max_splits=16):
+    """A KV split count for sage_attn_fwd_split: 1 when the 128-query tiles
+    already fill the GPU (two CTAs per SM) in well-balanced waves, else the
+    smallest count whose waves are at least 90 % full, keeping at least 8 KV
+    tiles per range."""
+    ctas = B * H * -(-Nq // 128)
+    slots = 2 * sm_count
+    tiles = -(-Nkv // 128)
+    best, best_eff = 1, 0.0
+    for sp in range(1, max_splits + 1):
+        if sp > 1 and tiles // sp < 8:
+            break
+        waves = ctas * sp / slots
+        eff = waves / math.ceil(waves)
+        if eff >= 0.9:
+            return sp
+        if eff > best_eff + 1e-9:
+            best, best_eff = sp, eff
+    return best
+
+
+def attn_split_workspace_bytes(shape, kv_splits):
+    return lib().sage_attn_split_workspace_bytes(ctypes.byref(shape), int(kv_splits))
+
+
 def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, stream=None,
-             block_mask=None):
+             block_mask=None, kv_splits=1, workspace=None):
     """sage_attn_fwd on a QuantizedQKV; returns the bf16 output tensor.
 
     block_mask: optional contiguous uint8 CUDA tensor of block_mask_shape();
-    tiles whose byte is 0 are skipped (sage_attn_fwd_block_sparse)."""
+    tiles whose byte is 0 are skipped (sage_attn_fwd_block_sparse).
+    kv_splits: > 1 runs the split-KV form (sage_attn_fwd_split) with that
+    many KV ranges per query tile; "auto" picks one with suggest_kv_splits.
+    workspace: its device scratch (allocated here when None)."""
     import torch
     s = qkv.shape
     dev = qkv.bufs["q_i8"].device
     if out is None:
         out = torch.empty((s.B, s.H, s.Nq, s.D), dtype=torch.bfloat16, device=dev)
     st = qkv.struct()
+    if kv_splits == "auto":
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        kv_splits = suggest_kv_splits(s.B, s.H, s.Nq, s.Nkv, sms)
+    if kv_splits != 1:
+        if block_mask is not None:
+            raise ValueError("kv_splits and block_mask are not combined")
+        need = attn_split_workspace_bytes(s, kv_splits)
+        if need == 0:
+            raise ValueError("kv_splits must be in 1..16")
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _check(lib().sage_attn_fwd_split(ctypes.byref(st), ctypes.byref(s), int(mask),
+                                         int(mask_block), int(kv_splits), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _ptr(out),
+                                         _ptr(o_f32), _ptr(lse), _stream(stream)),
+               "sage_attn_fwd_split")
+        return out
     if block_mask is None:
         _check(lib().sage_attn_fwd(ctypes.byref(st), ctypes.byref(s), int(mask), int(mask_block),
                                    _ptr(out), _ptr(o_f32), _ptr(lse), _stream(stream)),

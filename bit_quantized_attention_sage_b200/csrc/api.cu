@@ -345,9 +345,16 @@ SAGE_EXPORT sage_status sage_quant_qk_rope(const void* q_bf16, const void* k_bf1
 }
 
 namespace {
+size_t split_ws_bytes(const sage_shape* s, int splits) {
+  const size_t rows = static_cast<size_t>(s->B) * s->H * ((s->Nq + kAttnBM - 1) / kAttnBM) *
+                      kAttnBM;
+  return static_cast<size_t>(splits) * rows * (static_cast<size_t>(s->D) + 2) * 4;
+}
+
 sage_status attn_common(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
                         int mask_block, const uint8_t* block_mask, void* o_bf16, float* o_f32,
-                        float* lse, void* stream) {
+                        float* lse, void* stream, int splits = 1, void* workspace = nullptr,
+                        size_t ws_bytes = 0) {
   if (!shape_ok(shape) || !qkv_ok(qkv) || !aligned16(o_bf16)) return SAGE_ERR_INVALID_ARG;
   if (o_f32 && !aligned16(o_f32)) return SAGE_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SAGE_ERR_INVALID_ARG;
@@ -367,6 +374,17 @@ sage_status attn_common(const sage_qkv_quant* qkv, const sage_shape* shape, int 
   p.bmask = block_mask;
   p.n_qt = (shape->Nq + kAttnBM - 1) / kAttnBM;
   p.n_kt = (shape->Nkv + kAttnBN - 1) / kAttnBN;
+  if (splits > 1) {
+    const size_t rows = static_cast<size_t>(p.BH) * p.n_qt * kAttnBM;
+    p.splits = splits;
+    p.part_o = static_cast<float*>(workspace);
+    p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         static_cast<size_t>(splits) * rows * shape->D * 4);
+    if (launch_attn(maps, p, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+    return launch_attn_merge(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
+                                                                                 : SAGE_ERR_CUDA;
+  }
   return launch_attn(maps, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
                                                                                 : SAGE_ERR_CUDA;
 }
@@ -376,6 +394,26 @@ SAGE_EXPORT sage_status sage_attn_fwd(const sage_qkv_quant* qkv, const sage_shap
                                       int mask_block, void* o_bf16, float* o_f32, float* lse,
                                       void* stream) {
   return attn_common(qkv, shape, mask, mask_block, nullptr, o_bf16, o_f32, lse, stream);
+}
+
+SAGE_EXPORT size_t sage_attn_split_workspace_bytes(const sage_shape* shape, int kv_splits) {
+  if (!shape_ok(shape) || kv_splits < 1 || kv_splits > kAttnMaxSplits) return 0;
+  return kv_splits == 1 ? 0 : split_ws_bytes(shape, kv_splits);
+}
+
+SAGE_EXPORT sage_status sage_attn_fwd_split(const sage_qkv_quant* qkv, const sage_shape* shape,
+                                            int mask, int mask_block, int kv_splits,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* o_bf16, float* o_f32, float* lse,
+                                            void* stream) {
+  if (!shape_ok(shape) || kv_splits < 1 || kv_splits > kAttnMaxSplits)
+    return SAGE_ERR_INVALID_ARG;
+  if (kv_splits == 1)
+    return attn_common(qkv, shape, mask, mask_block, nullptr, o_bf16, o_f32, lse, stream);
+  if (!aligned16(workspace) || workspace_bytes < split_ws_bytes(shape, kv_splits))
+    return SAGE_ERR_INVALID_ARG;
+  return attn_common(qkv, shape, mask, mask_block, nullptr, o_bf16, o_f32, lse, stream,
+                     kv_splits, workspace, workspace_bytes);
 }
 
 SAGE_EXPORT sage_status sage_attn_fwd_block_sparse(const sage_qkv_quant* qkv,

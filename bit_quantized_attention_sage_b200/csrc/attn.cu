@@ -257,10 +257,11 @@ __device__ __forceinline__ void rescale_row(uint32_t tO, float alpha) {
 }
 
 // Softmax / correction / epilogue for one query row per thread.
-template <int D, bool SPARSE>
+template <int D, bool SPARSE, bool SPLIT>
 __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
-                                             uint32_t tmem_O, int bh, int qt, int nk,
+                                             uint32_t tmem_O, int bh, int qt, int kt0, int nk,
                                              const WaitCtx& w) {
+  const int kt_base = SPLIT ? kt0 : 0;  // first KV tile (dense: 0)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;               // TMEM lane quadrant of this warp
   const int r = quad * 32 + lane;          // row within the tile
@@ -275,7 +276,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   uint8_t* prow0 = s.p[0] + r * BN;
 
   TileSeq<SPARSE> seq(s.tile_bits, 0);
-  int kt = (SPARSE && nk > 0) ? seq.next() : 0;  // KV tile of this iteration (sparse)
+  int kt = (SPARSE && nk > 0) ? seq.next() : kt_base;  // KV tile of this iteration
   float ks0 = k_block_scale(ksc, 2 * kt, p.nkv_blocks);
   float ks1 = k_block_scale(ksc, 2 * kt + 1, p.nkv_blocks);
   float m = -INFINITY, l = 0.0f;
@@ -287,7 +288,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   __syncwarp();
   if (lane == 0) mbar_arrive(&s.s_free);
   for (int it = 0; it < nk; it++) {
-    if constexpr (!SPARSE) kt = it;
+    if constexpr (!SPARSE) kt = kt_base + it;
     const int j0 = kt * BN;
     if (!warp_wait(&s.s_full, it & 1, w, kSiteSmS)) { ok = false; break; }
     tc_fence_after();
@@ -398,6 +399,33 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   }
 
   if (!ok) return;
+  if constexpr (SPLIT) {  // this range's partial result: the raw O sum, m, l
+    const size_t rows_pad = static_cast<size_t>(p.n_qt) * BM;
+    const size_t prow = (static_cast<size_t>(blockIdx.z) * p.BH + bh) * rows_pad +
+                        static_cast<size_t>(qt) * BM + r;
+    float4* po = reinterpret_cast<float4*>(p.part_o + prow * D);
+    if (nk == 0) {  // an empty range (fewer tiles than ranges): nothing seen
+#pragma unroll 1
+      for (int e = 0; e < D / 4; e++) po[e] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      p.part_ml[prow * 2] = -INFINITY;
+      p.part_ml[prow * 2 + 1] = 0.0f;
+      return;
+    }
+    if (!warp_wait(&s.o_ready, (nk - 1) & 1, w, kSiteSmEpi)) return;
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < D; c += 32) {
+      uint32_t o[32];
+      tmem_ld32(tO + c, o);
+#pragma unroll
+      for (int e = 0; e < 8; e++)
+        po[c / 4 + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                    __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+    }
+    p.part_ml[prow * 2] = m;
+    p.part_ml[prow * 2 + 1] = l;
+    return;
+  }
   const float* vsc = p.v_scale + static_cast<size_t>(bh) * D;
   const size_t orow = (static_cast<size_t>(bh) * p.Nq + (valid ? i : 0)) * D;
   if (SPARSE && nk == 0) {  // no tile at all for this CTA; O = 0, lse = -inf
@@ -471,9 +499,8 @@ __device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint3
   if (lane == 0) mbar_arrive(&s.s_free);
 }
 
-template <int D, bool DUMP, bool SPARSE>
-__global__ void __launch_bounds__(kThreads, 2)
-    k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+template <int D, bool DUMP, bool SPARSE, bool SPLIT>
+__device__ __forceinline__ void attn_body(const AttnMaps& maps, const AttnParams& p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 128-byte swizzled TMA tiles and the MMA descriptors need 1024-byte
   // aligned tiles; refuse (before any barrier, copy or TMEM use) otherwise.
@@ -496,6 +523,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     const int last = min(p.Nq - 1, qt * BM + BM - 1);
     nk = (row_limit(last, p) + BN - 1) / BN;
+    if constexpr (SPLIT) {  // range blockIdx.z of p.splits contiguous ranges
+      const int sp = static_cast<int>(blockIdx.z);
+      kt0 = nk * sp / p.splits;
+      nk = nk * (sp + 1) / p.splits - kt0;
+    }
   }
   if constexpr (SPARSE) {
     // bitmap of the tiles below nk that the block mask switches on (one
@@ -549,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) mma_issuer<D, DUMP>(s, tmem_S, tmem_O, nk, w);
   } else {
     if (DUMP) dump_rows<D>(s, p, tmem_S, w);
-    else softmax_rows<D, SPARSE>(s, p, tmem_S, tmem_O, bh, qt, nk, w);
+    else softmax_rows<D, SPARSE, SPLIT>(s, p, tmem_S, tmem_O, bh, qt, kt0, nk, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -558,6 +590,73 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+template <int D, bool DUMP, bool SPARSE>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  attn_body<D, DUMP, SPARSE, false>(maps, p);
+}
+
+// Split-KV: CTA (qt, bh, range) over its range of the query tile's KV tiles;
+// writes partial results for k_attn_merge.
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_attn_split(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  attn_body<D, false, false, true>(maps, p);
+}
+
+// Merge of the split-KV partials, 8 rows per 128-thread CTA, thread t: row
+// t / 16, channels 8 (t % 16) .. + 7 (D = 128; D = 64 uses the first 8
+// threads of each row).  m = max_s m_s, a_s = exp2(m_s - m) (0 for a range
+// that saw no key), O = sum_s a_s O_s, l = sum_s a_s l_s in ascending s, each
+// product and sum rounded once; then O vs / l as in the unsplit epilogue.
+template <int D>
+__global__ void __launch_bounds__(128) k_attn_merge(const AttnParams p) {
+  const int bh = blockIdx.y;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 4);  // row of the head
+  const int c8 = (threadIdx.x & 15) * 8;
+  if (r >= p.Nq || c8 >= D) return;
+  const size_t rows_pad = static_cast<size_t>(p.n_qt) * BM;
+  const size_t stride_s = static_cast<size_t>(p.BH) * rows_pad;  // rows per range
+  const size_t row = static_cast<size_t>(bh) * rows_pad + r;
+  float m = -INFINITY;
+  for (int sp = 0; sp < p.splits; sp++) m = fmaxf(m, p.part_ml[(sp * stride_s + row) * 2]);
+  float l = 0.0f;
+  float o[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+  for (int sp = 0; sp < p.splits; sp++) {
+    const float ms = p.part_ml[(sp * stride_s + row) * 2];
+    const float ls = p.part_ml[(sp * stride_s + row) * 2 + 1];
+    const float a = ms == -INFINITY ? 0.0f : ex2_approx(__fsub_rn(ms, m));
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + (sp * stride_s + row) * D + c8);
+    const float4 u = src[0], v = src[1];
+    const float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; e++) o[e] = __fmaf_rn(a, x[e], o[e]);
+    l = __fadd_rn(l, __fmul_rn(a, ls));
+  }
+  const bool seen = l > 0.0f;
+  const float inv = seen ? __frcp_rn(l) : 0.0f;
+  const float* vsc = p.v_scale + static_cast<size_t>(bh) * D + c8;
+  float f[8];
+#pragma unroll
+  for (int e = 0; e < 8; e++) f[e] = o[e] * (__ldg(vsc + e) * inv);
+  uint32_t b[4];
+#pragma unroll
+  for (int e = 0; e < 4; e++) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+    b[e] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  const size_t orow = (static_cast<size_t>(bh) * p.Nq + r) * D + c8;
+  *reinterpret_cast<uint4*>(p.o + orow) = make_uint4(b[0], b[1], b[2], b[3]);
+  if (p.o_f32) {
+    float4* d32 = reinterpret_cast<float4*>(p.o_f32 + orow);
+    d32[0] = make_float4(f[0], f[1], f[2], f[3]);
+    d32[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+  if (p.lse && c8 == 0)
+    p.lse[static_cast<size_t>(bh) * p.Nq + r] =
+        seen ? (m + log2f(l) - 8.0f) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace
@@ -570,6 +669,11 @@ cudaError_t prepare_one() {
   return cudaFuncSetAttribute(k_attn<D, DUMP, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(smem_bytes_for(D)));
 }
+template <int D>
+cudaError_t prepare_split() {
+  return cudaFuncSetAttribute(k_attn_split<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(smem_bytes_for(D)));
+}
 }  // namespace
 
 cudaError_t attn_prepare(int D) {
@@ -578,10 +682,12 @@ cudaError_t attn_prepare(int D) {
     e = prepare_one<128, false, false>();
     if (e == cudaSuccess) e = prepare_one<128, true, false>();
     if (e == cudaSuccess) e = prepare_one<128, false, true>();
+    if (e == cudaSuccess) e = prepare_split<128>();
   } else {
     e = prepare_one<64, false, false>();
     if (e == cudaSuccess) e = prepare_one<64, true, false>();
     if (e == cudaSuccess) e = prepare_one<64, false, true>();
+    if (e == cudaSuccess) e = prepare_split<64>();
   }
   return e;
 }
@@ -589,6 +695,12 @@ cudaError_t attn_prepare(int D) {
 cudaError_t launch_attn(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
   dim3 grid((p.Nq + BM - 1) / BM, p.BH);
   const bool sparse = p.bmask != nullptr;
+  if (p.splits > 1) {  // split-KV partials; launch_attn_merge combines them
+    grid.z = p.splits;
+    if (p.D == 128) k_attn_split<128><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
+    else k_attn_split<64><<<grid, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+    return cudaGetLastError();
+  }
   if (p.D == 128) {
     if (sparse) k_attn<128, false, true><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
     else k_attn<128, false, false><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);
@@ -604,6 +716,13 @@ cudaError_t launch_attn_dump(const AttnMaps& maps, const AttnParams& p, cudaStre
     k_attn<128, true, false><<<1, kThreads, smem_bytes_for(128), stream>>>(maps, p);
   else
     k_attn<64, true, false><<<1, kThreads, smem_bytes_for(64), stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_merge(const AttnParams& p, cudaStream_t stream) {
+  dim3 grid((p.Nq + 7) / 8, p.BH);
+  if (p.D == 128) k_attn_merge<128><<<grid, 128, 0, stream>>>(p);
+  else k_attn_merge<64><<<grid, 128, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -14,6 +14,8 @@ constexpr int kAttnBM = 128;  // query rows per CTA (tcgen05 M)
 constexpr int kAttnBN = 128;  // keys per KV tile
 // block-sparse mode: at most this many KV tiles (786432 keys) per head
 constexpr int kAttnMaxKvTiles = 6144;
+// split-KV mode: at most this many KV ranges per query tile
+constexpr int kAttnMaxSplits = 16;
 
 struct AttnParams {
   int BH, Nq, Nkv, D;
@@ -32,6 +34,12 @@ struct AttnParams {
   // visited only if non-zero
   const uint8_t* bmask;
   int n_qt, n_kt;
+  // split-KV mode (splits > 1): the KV tiles of each query tile in `splits`
+  // ranges, one CTA each (grid z); every CTA writes its unnormalized O and
+  // its running max and sum, which launch_attn_merge combines
+  int splits;
+  float* part_o;   // [splits][BH][n_qt * 128][D] fp32
+  float* part_ml;  // [splits][BH][n_qt * 128][2]: m (log2 units), l
   // score-dump mode (debug): a single tile (bh, qt, kt), int32 [128, 128]
   int dbg_bh, dbg_qt, dbg_kt;
   int32_t* dbg_out;
@@ -47,5 +55,7 @@ size_t attn_smem_bytes(int D);
 cudaError_t attn_prepare(int D);  // one-time function attributes
 cudaError_t launch_attn(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_dump(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream);
+// the merge of a split-KV launch (same params): O, optional fp32 O and lse
+cudaError_t launch_attn_merge(const AttnParams& p, cudaStream_t stream);
 
 }  // namespace sage

@@ -242,6 +242,37 @@ sage_status sage_attn_fwd_block_sparse(const sage_qkv_quant *qkv, const sage_sha
                                        int mask, int mask_block, const uint8_t *block_mask,
                                        void *o_bf16, float *o_f32, float *lse, void *stream);
 
+/* Device workspace sage_attn_fwd_split needs (bytes): kv_splits * B * H *
+ * ceil(Nq/128)*128 * (D + 2) * 4; 0 for kv_splits = 1 or an invalid
+ * argument (kv_splits outside 1..16, bad shape). */
+size_t sage_attn_split_workspace_bytes(const sage_shape *shape, int kv_splits);
+
+/* sage_attn_fwd in split-KV form, for shapes with few query tiles (e.g. one
+ * streaming frame against a long cache), where one CTA per 128-query tile
+ * leaves most of the GPU idle.
+ *
+ * The KV tiles that a query tile visits under `mask` ([0, nk), nk from its
+ * last row) are cut into kv_splits contiguous ranges [floor(s nk / S),
+ * floor((s+1) nk / S)).  Each range runs the online softmax of sage_attn_fwd
+ * on its own CTA, giving an unnormalized O_s with running max m_s and sum l_s;
+ * a second kernel merges them in ascending s:
+ *   m = max_s m_s,  a_s = exp2(m_s - m) (0 for a range that saw no key),
+ *   O = sum_s a_s O_s,  l = sum_s a_s l_s,  o = O * v_scale / l,
+ * lse as for sage_attn_fwd.  P is quantized relative to each range's own
+ * running max, so results differ from sage_attn_fwd by rounding only.
+ * kv_splits = 1 is sage_attn_fwd itself (no workspace needed).
+ *
+ *   kv_splits: 1..16.  workspace: device, 16-byte aligned, at least
+ *   sage_attn_split_workspace_bytes(shape, kv_splits) bytes (contents need
+ *   not be initialised).  Other arguments: as for sage_attn_fwd.
+ * Enqueues two kernels on `stream`.
+ * Errors: as sage_attn_fwd, plus SAGE_ERR_INVALID_ARG for kv_splits outside
+ * 1..16 or a missing, misaligned or too small workspace. */
+sage_status sage_attn_fwd_split(const sage_qkv_quant *qkv, const sage_shape *shape, int mask,
+                                int mask_block, int kv_splits, void *workspace,
+                                size_t workspace_bytes, void *o_bf16, float *o_f32, float *lse,
+                                void *stream);
+
 /* Debug: run the attention kernel's load + INT8 MMA path on selected tiles
  * and copy the int32 score tile it leaves in tensor memory to `out`.
  *   tiles  host int array of n_tiles triples (bh, qt, kt): head index b*H+h,

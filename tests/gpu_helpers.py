@@ -58,10 +58,13 @@ def bf16_half_ulp(x):
     return 0.5 * 2.0 ** (e - 7)
 
 
-def check_rows(ref_head, rows, o_bf16_rows, o_f32_rows, lse_rows, mask, mb, block_mask=None):
+def check_rows(ref_head, rows, o_bf16_rows, o_f32_rows, lse_rows, mask, mb, block_mask=None,
+               kv_splits=1):
     """O and lse of the given rows against the oracle (same quantized inputs;
-    `block_mask`: this head's [n_qt, n_kt] tile mask, if any)."""
-    o_ref, slack, lse_ref = oracle.attn_rows(ref_head, rows, mask, mb, block_mask=block_mask)
+    `block_mask`: this head's [n_qt, n_kt] tile mask, if any; `kv_splits`:
+    the split-KV form's range count)."""
+    o_ref, slack, lse_ref = oracle.attn_rows(ref_head, rows, mask, mb, block_mask=block_mask,
+                                             kv_splits=kv_splits)
     tol = O_ATOL + slack
     err32 = np.abs(o_f32_rows.astype(np.float64) - o_ref)
     bad = err32 > tol

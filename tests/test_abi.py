@@ -128,3 +128,23 @@ def test_rope_quantizer_arguments_are_rejected_before_any_launch(L):
     # the checks of sage_quant_qk still apply (workspace too small)
     assert L.sage_quant_qk_rope(p, p, p, ctypes.byref(s), *tabs, ctypes.byref(ok), p, ws - 1,
                                 None) == 1
+
+
+def test_split_attention_arguments_are_rejected_before_any_launch(L):
+    s = sage.make_shape(1, 2, 300, 700, 128)
+    ok = sage._QKV(*([16 * 1024] * 7))
+    p = ctypes.c_void_p(4096)
+    need = L.sage_attn_split_workspace_bytes(ctypes.byref(s), 3)
+    assert need == 3 * 2 * 384 * 130 * 4
+    assert L.sage_attn_split_workspace_bytes(ctypes.byref(s), 1) == 0
+    assert L.sage_attn_split_workspace_bytes(ctypes.byref(s), 17) == 0
+    for splits in (0, 17):
+        assert L.sage_attn_fwd_split(ctypes.byref(ok), ctypes.byref(s), 0, 0, splits, p, need, p,
+                                     None, None, None) == 1
+    # workspace missing, misaligned or too small
+    assert L.sage_attn_fwd_split(ctypes.byref(ok), ctypes.byref(s), 0, 0, 3, None, need, p,
+                                 None, None, None) == 1
+    assert L.sage_attn_fwd_split(ctypes.byref(ok), ctypes.byref(s), 0, 0, 3, ctypes.c_void_p(4100),
+                                 need, p, None, None, None) == 1
+    assert L.sage_attn_fwd_split(ctypes.byref(ok), ctypes.byref(s), 0, 0, 3, p, need - 1, p,
+                                 None, None, None) == 1
