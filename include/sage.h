@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
     SAGE_OK = 0,
     SAGE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or mask   */
-    SAGE_ERR_UNSUPPORTED = 2, /* valid request outside this build's support  */
+    SAGE_ERR_UNSUPPORTED = 2, /* valid request the library does not support */
     SAGE_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed         */
     SAGE_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out           */
 } sage_status;

@@ -1,7 +1,7 @@
 """Compile the CPU oracle into ``oracle/liboracle.so`` with gcc.
 
 The oracle is test infrastructure: building it is part of ``build()`` so that
-the checker is ready, but only the tests, the smoke check and the benchmark's
+the oracle is ready, but only the tests, the smoke check and the benchmark's
 CPU-baseline / reference arm load it.
 """
 import os
