@@ -89,6 +89,8 @@ def lib():
         L.sage_w8a8_quant_act.argtypes = [P, LL, LL, P, P, P]
         L.sage_w8a8_quant_weight.restype = I
         L.sage_w8a8_quant_weight.argtypes = [P, LL, LL, P, P, P]
+        L.sage_w8a8_gemm_q.restype = I
+        L.sage_w8a8_gemm_q.argtypes = [P, P, P, P, LL, LL, LL, P, P, P, P]
         L.sage_w8a8_gemm.restype = I
         L.sage_w8a8_gemm.argtypes = [P, P, P, P, LL, LL, LL, P, P, P]
         L.sage_sync_status.restype = I
@@ -391,6 +393,23 @@ def w8a8_gemm(xq, sx, wq, sw, out=None, y_f32=None, stream=None):
     _check(lib().sage_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(out),
                                 _ptr(y_f32), _stream(stream)), "sage_w8a8_gemm")
     return out
+
+
+def w8a8_gemm_q(xq, sx, wq, sw, q_i8=None, q_scale=None, y=None, stream=None):
+    """sage_w8a8_gemm_q: the Q projection with Q's per-64-token INT8
+    quantization in the GEMM epilogue.  Returns (q_i8 [N/128, M_pad, 128],
+    q_scale [N/128, M_pad/64], y) where y is the optional bf16 Y passed in."""
+    import torch
+    M, K = xq.shape
+    N = wq.shape[0]
+    mpad = -(-M // 64) * 64
+    if q_i8 is None:
+        q_i8 = torch.empty((N // 128, mpad, 128), dtype=torch.int8, device=xq.device)
+    if q_scale is None:
+        q_scale = torch.empty((N // 128, mpad // 64), dtype=torch.float32, device=xq.device)
+    _check(lib().sage_w8a8_gemm_q(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y),
+                                  _ptr(q_i8), _ptr(q_scale), _stream(stream)), "sage_w8a8_gemm_q")
+    return q_i8, q_scale, y
 
 
 def linear_w8a8(x, wq, sw, stream=None):

@@ -233,18 +233,16 @@ SAGE_EXPORT sage_status sage_w8a8_quant_weight(const void* w_bf16, long long N, 
              : SAGE_ERR_CUDA;
 }
 
-SAGE_EXPORT sage_status sage_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq,
-                                       const float* sw, long long M, long long N, long long K,
-                                       void* y_bf16, float* y_f32, void* stream) {
-  if (!w8a8_dims_ok(M, N, K) || !aligned16(xq) || !aligned16(wq) || !aligned16(y_bf16) || !sx ||
-      !sw || (y_f32 && !aligned16(y_f32)))
-    return SAGE_ERR_INVALID_ARG;
+namespace {
+sage_status w8a8_gemm_common(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                             long long M, long long N, long long K, void* y_bf16, float* y_f32,
+                             int8_t* q_i8, float* q_scale, void* stream) {
   DeviceState* d = device_state();
   if (!d) return SAGE_ERR_CUDA;
-  W8a8Maps maps;
+  W8a8Maps maps{};
   if (!encode_u8_3d(&maps.x, xq, K, M, 1, kW8a8Group, kW8a8BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_u8_3d(&maps.w, wq, K, N, 1, kW8a8Group, kW8a8BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_bf16_2d(&maps.y, y_bf16, N, M, 64, kW8a8BM, CU_TENSOR_MAP_SWIZZLE_128B))
+      (y_bf16 && !encode_bf16_2d(&maps.y, y_bf16, N, M, 64, kW8a8BM, CU_TENSOR_MAP_SWIZZLE_128B)))
     return SAGE_ERR_CUDA;
   W8a8Params p{};
   p.M = static_cast<int>(M);
@@ -254,11 +252,34 @@ SAGE_EXPORT sage_status sage_w8a8_gemm(const int8_t* xq, const float* sx, const 
   p.sw = sw;
   p.y = static_cast<uint16_t*>(y_bf16);
   p.y_f32 = y_f32;
+  p.q_i8 = q_i8;
+  p.q_scale = q_scale;
   p.budget = kWaitBudget;
   p.status = d->status;
   return launch_w8a8_gemm(maps, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SAGE_OK
              : SAGE_ERR_CUDA;
+}
+}  // namespace
+
+SAGE_EXPORT sage_status sage_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq,
+                                       const float* sw, long long M, long long N, long long K,
+                                       void* y_bf16, float* y_f32, void* stream) {
+  if (!w8a8_dims_ok(M, N, K) || !aligned16(xq) || !aligned16(wq) || !aligned16(y_bf16) || !sx ||
+      !sw || (y_f32 && !aligned16(y_f32)))
+    return SAGE_ERR_INVALID_ARG;
+  return w8a8_gemm_common(xq, sx, wq, sw, M, N, K, y_bf16, y_f32, nullptr, nullptr, stream);
+}
+
+SAGE_EXPORT sage_status sage_w8a8_gemm_q(const int8_t* xq, const float* sx, const int8_t* wq,
+                                         const float* sw, long long M, long long N, long long K,
+                                         void* y_bf16, int8_t* q_i8, float* q_scale,
+                                         void* stream) {
+  if (!w8a8_dims_ok(M, N, K) || !aligned16(xq) || !aligned16(wq) || !sx || !sw ||
+      !aligned16(q_i8) || !q_scale || (reinterpret_cast<uintptr_t>(q_scale) & 3u) ||
+      (y_bf16 && !aligned16(y_bf16)))
+    return SAGE_ERR_INVALID_ARG;
+  return w8a8_gemm_common(xq, sx, wq, sw, M, N, K, y_bf16, nullptr, q_i8, q_scale, stream);
 }
 
 SAGE_EXPORT const char* sage_status_string(sage_status st) {

@@ -151,6 +151,7 @@ struct alignas(1024) GemmSmem {
   // bf16 Y tile staging for the TMA store, one buffer per column part:
   // [128 rows][64 columns], 128-byte swizzled like the tensor map
   uint8_t ystage[kPromWarps / 4][BM * kPromCols * 2];
+  float qmax[4][kPromWarps / 4];  // attention-Q mode: |Q| maxima per (quadrant, column part)
   uint8_t seed[128];           // f16 broadcast tile of the accumulator seed MMA
   uint64_t full[NS], empty[NS];
   uint64_t acc_full[NPAIR], acc_free[NPAIR];
@@ -314,6 +315,7 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Maps& maps, 
   // the first warp of a column part issues its TMA stores
   const bool storer = ((warp - kFirstProm) & 3) == 0 && lane == 0;
   const int bar_id = 1 + part;  // named barrier of the part's 4 warps (0 is __syncthreads)
+  const bool qout = p.q_i8 != nullptr;  // attention-Q epilogue (barrier 3: all promotion warps)
   uint8_t* stg = s.ystage[part];
   const int r = quad * 32 + lane;
   const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16) + part * kPromCols;
@@ -369,6 +371,87 @@ __device__ __forceinline__ void gemm_promote(GemmSmem& s, const W8a8Maps& maps, 
           y[e] = __ffma2_rn(pf, sc2, y[e]);
         }
       }
+    }
+    if (qout) {
+      // attention-Q epilogue: every promotion warp leaves together after a
+      // timeout anywhere (one 256-thread barrier for both column parts)
+      if (storer) bulk_wait_read_all();
+      if (bar_or_n(3, 32 * kPromWarps, !ok || *w.abort != 0)) break;
+      float yb[kPromCols];  // Q = bf16(y) as floats
+#pragma unroll
+      for (int e = 0; e < kPromCols / 2; e++) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(y[e].x, y[e].y);
+        yb[2 * e] = __low2float(h2);
+        yb[2 * e + 1] = __high2float(h2);
+      }
+      if (p.y) {
+        uint8_t* row = stg + r * (kPromCols * 2);
+#pragma unroll
+        for (int c = 0; c < kPromCols / 8; c++) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(yb[8 * c + 2 * e], yb[8 * c + 2 * e + 1]);
+            pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        fence_proxy_async_smem();
+      }
+      float a = 0.0f;  // |Q| max of this thread's valid values
+      if (valid) {
+#pragma unroll
+        for (int e = 0; e < kPromCols; e += 2) a = fmax3(a, fabsf(yb[e]), fabsf(yb[e + 1]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+      if (lane == 0) s.qmax[quad][part] = a;
+      bar_sync_n(3, 32 * kPromWarps);
+      if (storer && p.y) {
+        tma_store_2d(&maps.y, stg, n0 + part * kPromCols, m0);
+        bulk_commit();
+      }
+      // 64-token block b = rows 64 b .. 64 b + 63 of the tile: quadrants 2b, 2b + 1
+      const int qb = quad >> 1;
+      a = fmaxf(fmaxf(s.qmax[2 * qb][0], s.qmax[2 * qb][1]),
+                fmaxf(s.qmax[2 * qb + 1][0], s.qmax[2 * qb + 1][1]));
+      const float scale = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
+      const float inv = (a == 0.0f) ? 0.0f : __fdiv_rn(127.0f, a);
+      const int mpad = (p.M + 63) / 64 * 64;
+      const int head = n0 / BN;
+      if (m < mpad) {  // rows past M within the padding get zero codes
+        // code = round_half_even(Q * inv), |Q inv| <= 127 (1 + 2^-22), so no
+        // clamp is needed; adding 1.5 * 2^23 rounds it into the low byte of
+        // the fp32 bit pattern (0x4B400000 + code), which is packed directly
+        // (the product is rounded on its own, as in the plain quantizer: the
+        // scalar intrinsics are never contracted into an fma)
+        uint32_t pk[kPromCols / 4];
+#pragma unroll
+        for (int c = 0; c < kPromCols / 4; c++) {
+          uint32_t t[4];
+#pragma unroll
+          for (int e = 0; e < 4; e++)
+            t[e] = __float_as_uint(__fadd_rn(__fmul_rn(yb[4 * c + e], inv), kBias));
+          const uint32_t lo = __byte_perm(t[0], t[1], 0x0040);
+          const uint32_t hi = __byte_perm(t[2], t[3], 0x0040);
+          pk[c] = (valid && a != 0.0f) ? __byte_perm(lo, hi, 0x5410) : 0u;
+        }
+        uint4* dst = reinterpret_cast<uint4*>(p.q_i8 + (static_cast<size_t>(head) * mpad + m) * BN +
+                                              part * kPromCols);
+#pragma unroll
+        for (int c = 0; c < kPromCols / 16; c++)
+          dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        if (part == 0 && (quad & 1) == 0 && lane == 0)
+          p.q_scale[static_cast<size_t>(head) * (mpad / 64) + m / 64] = scale;
+      }
+      if (valid && p.y_f32) {
+        float4* d32 = reinterpret_cast<float4*>(p.y_f32 + static_cast<size_t>(m) * p.N + n0 +
+                                                part * kPromCols);
+#pragma unroll
+        for (int e = 0; e < kPromCols / 4; e++)
+          d32[e] = make_float4(y[2 * e].x, y[2 * e].y, y[2 * e + 1].x, y[2 * e + 1].y);
+      }
+      continue;
     }
     // epilogue of this tile (the issuers already run the next tile's steps):
     // bf16 rows into the part's staging buffer, then one TMA store of the

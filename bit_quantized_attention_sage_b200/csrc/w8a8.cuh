@@ -18,8 +18,14 @@ struct W8a8Params {
   int M, N, K;            // Y [M, N] = X [M, K] W [N, K]^T; N, K multiples of 128
   const float* sx;        // [M, K/128]
   const float* sw;        // [N/128, K/128]
-  uint16_t* y;            // bf16 bits [M, N]
+  uint16_t* y;            // bf16 bits [M, N], or null when q_i8 is set
   float* y_f32;           // [M, N] or null
+  // attention-Q output (null: none): Y read as Q of N/128 heads of D = 128
+  // (column tile = head), rounded to bf16 and quantized like sage_quant_qk's
+  // Q: int8 [N/128][M_pad][128] codes, per-64-token-block scales
+  // [N/128][M_pad/64], M_pad = M rounded up to 64
+  int8_t* q_i8;
+  float* q_scale;
   long long budget;       // per-wait budget, SM cycles
   int* status;            // device status word pair
 };

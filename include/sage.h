@@ -337,11 +337,36 @@ sage_status sage_w8a8_quant_weight(const void *w_bf16, long long N, long long K,
  * and Y = bf16(y) (round-half-to-even).
  *   y_bf16  device bf16 [M, N] (required)
  *   y_f32   device f32 [M, N] (y before rounding) or NULL
- * One kernel launch (one 128 x 128 output tile per CTA, column tiles
- * fastest). */
+ * One kernel launch (persistent: one CTA per SM loops over the 128 x 128
+ * output tiles, column tiles fastest). */
 sage_status sage_w8a8_gemm(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                            long long M, long long N, long long K, void *y_bf16, float *y_f32,
                            void *stream);
+
+/* sage_w8a8_gemm for the projection that produces attention's Q, with Q's
+ * quantization fused into the GEMM epilogue (the fusion "into the producing
+ * GEMM's epilogue" of the pages' kernel-fusion bullet, for the one operand
+ * whose quantization needs no statistic over all tokens).
+ *
+ * Y [M, N] = X W^T as sage_w8a8_gemm computes it, read as Q of one batch
+ * entry: M tokens, N/128 heads of D = 128 (column c of head h is column
+ * 128 h + c of Y).  The epilogue rounds Y to bf16 and quantizes it exactly as
+ * sage_quant_qk quantizes Q: per head and 64-token block, a = max|Q| over the
+ * block, q_scale = a/127, q_i8 = clamp(round_half_even(Q * fp32(127/a)),
+ * -127, 127); a = 0 gives scale 0 and codes 0; tokens M..M_pad-1 get code 0.
+ * So q_i8 and q_scale equal sage_quant_qk's Q output for that bf16 Q, bit for
+ * bit, without the bf16 round trip of Q through memory.
+ *
+ *   q_i8: device int8 [N/128][M_pad][128], M_pad = M rounded up to 64 (the
+ *     layout of one batch entry of sage_qkv_quant.q_i8), 16-byte aligned.
+ *   q_scale: device f32 [N/128][M_pad/64], 4-byte aligned.
+ *   y_bf16: the bf16 Y as well, or NULL.
+ *   Other arguments: as for sage_w8a8_gemm (N a multiple of 128).
+ * Errors: as sage_w8a8_gemm, plus SAGE_ERR_INVALID_ARG for a null or
+ * misaligned q_i8 or q_scale. */
+sage_status sage_w8a8_gemm_q(const int8_t *xq, const float *sx, const int8_t *wq,
+                             const float *sw, long long M, long long N, long long K,
+                             void *y_bf16, int8_t *q_i8, float *q_scale, void *stream);
 
 /* Static description of a status code (never NULL). */
 const char *sage_status_string(sage_status status);

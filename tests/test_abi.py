@@ -104,6 +104,11 @@ def test_block_sparse_and_w8a8_arguments_are_rejected_before_any_launch(L):
     assert L.sage_w8a8_gemm(p, p, p, p, 8, 128, 200, p, None, None) == 1
     assert L.sage_w8a8_gemm(p, p, p, p, 8, 64, 128, p, None, None) == 1
     assert L.sage_w8a8_gemm(ctypes.c_void_p(4100), p, p, p, 8, 128, 128, p, None, None) == 1
+    # the Q-fused form: q codes and scales required and aligned
+    assert L.sage_w8a8_gemm_q(p, p, p, p, 8, 128, 128, None, None, p, None) == 1
+    assert L.sage_w8a8_gemm_q(p, p, p, p, 8, 128, 128, None, ctypes.c_void_p(4100), p, None) == 1
+    assert L.sage_w8a8_gemm_q(p, p, p, p, 8, 128, 128, None, p, None, None) == 1
+    assert L.sage_w8a8_gemm_q(p, p, p, p, 8, 128, 128, None, p, ctypes.c_void_p(4098), None) == 1
 
 
 def test_rope_quantizer_arguments_are_rejected_before_any_launch(L):

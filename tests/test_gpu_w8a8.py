@@ -95,3 +95,33 @@ def test_bf16_output_alone():
     ry = oracle.w8a8_gemm_rows(rxq, rsx, rwq, rsw, np.arange(M))
     gotb = y.view(torch.int16).cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(gotb, synth.f32_to_bf16_bits(ry))
+
+
+@pytest.mark.parametrize("M,H,K,keep_y", [(300, 2, 256, True), (1000, 3, 640, False),
+                                          (2040, 4, 1536, True)])
+def test_q_quantization_fused_in_the_epilogue(M, H, K, keep_y):
+    # the Q projection with attention's per-64-token INT8 Q quantization in the
+    # GEMM epilogue: equal to sage_quant_qk's Q of the bf16 Y, bit for bit
+    N = 128 * H
+    x, w = bits((M, K), M + 1, outliers=3), bits((N, K), M + 2)
+    xq, sx = sage.w8a8_quant_act(dev(x))
+    wq, sw = sage.w8a8_quant_weight(dev(w))
+    y = sage.w8a8_gemm(xq, sx, wq, sw)
+    yq = torch.empty_like(y) if keep_y else None
+    q8, qs, yq = sage.w8a8_gemm_q(xq, sx, wq, sw, y=yq)
+    assert sage.sync_status() == 0
+    if keep_y:
+        assert torch.equal(yq, y)
+    qh = y.view(M, H, 128).permute(1, 0, 2).contiguous().unsqueeze(0)  # [1, H, M, 128]
+    ref = sage.quant_qk(qh, qh, qh)
+    assert torch.equal(q8, ref.view("q_i8")[0])
+    assert torch.equal(qs.view(torch.int32), ref.view("q_scale")[0].view(torch.int32))
+    # and the oracle: its fp32 Y, rounded to bf16, quantized as Q
+    rxq, rsx = oracle.w8a8_quant_act(x)
+    rwq, rsw = oracle.w8a8_quant_weight(w)
+    ry = synth.f32_to_bf16_bits(oracle.w8a8_gemm_rows(rxq, rsx, rwq, rsw, np.arange(M)))
+    for h in range(H):
+        qb = np.ascontiguousarray(ry[:, h * 128:(h + 1) * 128])
+        rq = oracle.quant_head(qb, qb[:64], qb[:64])
+        np.testing.assert_array_equal(q8[h].cpu().numpy(), rq["q8"])
+        np.testing.assert_array_equal(qs[h].cpu().numpy().view(np.int32), rq["qs"].view(np.int32))
