@@ -297,8 +297,12 @@ def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, 
     return out
 
 
-def attention(q, k, v, mask=None, stream=None):
-    """Drop-in quantized attention: bf16 [B, H, N, D] in, bf16 out."""
+def attention(q, k, v, mask=None, stream=None, kv_splits="auto"):
+    """Drop-in quantized attention: bf16 [B, H, N, D] in, bf16 out.
+
+    kv_splits: "auto" runs the split-KV form when the query tiles alone would
+    leave the GPU idle (e.g. one streaming frame against a long cache); an
+    int forces a split count (1: never split)."""
     if mask is None or mask == "none":
         m, mb = MASK_NONE, 0
     elif mask == "causal":
@@ -308,7 +312,7 @@ def attention(q, k, v, mask=None, stream=None):
     else:
         raise ValueError("mask must be None, 'causal' or ('block_causal', n)")
     qkv = quant_qk(q, k, v, stream=stream)
-    return attn_fwd(qkv, m, mb, stream=stream)
+    return attn_fwd(qkv, m, mb, stream=stream, kv_splits=kv_splits)
 
 
 def debug_qk_int32(qkv, tiles, stream=None):

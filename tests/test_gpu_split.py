@@ -57,3 +57,18 @@ def test_streaming_frame_sampled():
         ref = oracle.quant_head(q[0, h], k[0, h], v[0, h])
         check_rows(ref, rows, rows_of(o, 0, h, rows), rows_of(o32, 0, h, rows),
                    rows_of(lse, 0, h, rows), 2, 2040, kv_splits=splits)
+
+
+def test_drop_in_attention_picks_the_split_form():
+    w = synth.Workload("split_dropin", 1, 4, 2040, 26520, 128, mask=2, mask_block=2040, seed=92)
+    q, k, v = synth.full(w)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    splits = sage.suggest_kv_splits(1, 4, 2040, 26520, sms)
+    o_auto = sage.attention(qd, kd, vd, mask=("block_causal", 2040))
+    qkv = sage.quant_qk(qd, kd, vd)
+    o_split = sage.attn_fwd(qkv, 2, 2040, kv_splits=splits)
+    o_one = sage.attention(qd, kd, vd, mask=("block_causal", 2040), kv_splits=1)
+    o_plain = sage.attn_fwd(qkv, 2, 2040)
+    assert sage.sync_status() == 0
+    assert torch.equal(o_auto, o_split) and torch.equal(o_one, o_plain)
