@@ -17,7 +17,7 @@ import numpy as np
 
 from . import build as _build
 
-MASK_NONE, MASK_CAUSAL, MASK_BLOCK_CAUSAL = 0, 1, 2
+MASK_NONE, MASK_CAUSAL, MASK_BLOCK_CAUSAL, MASK_SLIDING_WINDOW = 0, 1, 2, 3
 BLK = 64          # Q/K quantization block (tokens)
 TKV = 128         # KV tile width of the online softmax (the device kernel's)
 BQ = 128          # query rows per block of a block-sparse mask (one query tile)
@@ -80,6 +80,17 @@ def lib():
         L.orc_w8a8_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, i32]
         L.orc_attn_fp64_rows.restype = i32
         L.orc_attn_fp64_rows.argtypes = [P, P, P, i64, i64, i32, i32, i64, P, i64, P, i32]
+        L.orc_attn_fp64_rows_win.restype = i32
+        L.orc_attn_fp64_rows_win.argtypes = [P, P, P, i64, i64, i32, i64, i64, i64, P, i64, P,
+                                             i32]
+        L.orc_attn_rows_win.restype = i32
+        L.orc_attn_rows_win.argtypes = [P, P, P, P, P, P, i64, i64, i32, i64, i64, i64, i64, f64,
+                                        i32, i64, P, i64, P, P, P, i32]
+        L.orc_attn_rows_identity_win.restype = i32
+        L.orc_attn_rows_identity_win.argtypes = [P, P, P, i64, i64, i32, i64, i64, i64, i64, i32,
+                                                 i64, P, i64, P, P, i32]
+        L.orc_row_window_export.restype = None
+        L.orc_row_window_export.argtypes = [i64, i64, i64, i32, i64, i64, i64, P]
         _lib = L
     return _lib
 
@@ -169,6 +180,18 @@ def row_limit(i, nq, nkv, mask, mb):
     return lib().orc_row_limit(i, nq, nkv, mask, mb)
 
 
+def row_window(i, nq, nkv, mask, mb, win=0, sink=0):
+    """(sink_end, lo, hi): query row i sees keys [0, sink_end) and [lo, hi)."""
+    out = np.empty(3, np.int64)
+    lib().orc_row_window_export(i, nq, nkv, mask, mb, win, sink, _p(out))
+    return tuple(int(x) for x in out)
+
+
+def _window(window):
+    frame, win, sink = (int(x) for x in window)
+    return frame, win, sink
+
+
 # ---------------------------------------------------------------- attention
 
 def _block_mask(block_mask, nkv, tkv):
@@ -182,7 +205,7 @@ def _block_mask(block_mask, nkv, tkv):
 
 
 def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
-              threads=None, block_mask=None, kv_splits=1):
+              threads=None, block_mask=None, kv_splits=1, window=None):
     """Same-quantization attention of one quantized head on the given rows.
 
     block_mask: optional uint8 [ceil(Nq / 128), ceil(Nkv / tkv)] of this head;
@@ -190,6 +213,8 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
     kv_splits > 1: the split-KV form (``orc_attn_rows_split``): the KV tiles of
     each 128-query tile in that many ranges, each its own online softmax,
     merged (not combined with a block mask).
+    window: (frame, win, sink) for the sliding-window mask with a reference
+    context (``orc_attn_rows_win``; mask and mb are then ignored).
     Returns (o [n, D] float64 of the fp32 recipe, slack [n, D] or None, lse [n]).
     """
     rows = np.ascontiguousarray(rows, np.int64)
@@ -203,7 +228,16 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
     qs = np.ascontiguousarray(qh["qs"])
     ks = np.ascontiguousarray(qh["ks"])
     vs = np.ascontiguousarray(qh["vs"])
-    if kv_splits > 1:
+    if window is not None:
+        if block_mask is not None:
+            raise ValueError("window and block_mask are not combined")
+        frame, win, sink = _window(window)
+        rc = lib().orc_attn_rows_win(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
+                                     qh["nq"], qh["nkv"], D, frame, win, sink, tkv, eps,
+                                     max(int(kv_splits), 1), BQ, _p(rows), n, _p(o),
+                                     _p(slack) if slack is not None else None, _p(lse),
+                                     _threads(threads))
+    elif kv_splits > 1:
         if block_mask is not None:
             raise ValueError("kv_splits and block_mask are not combined")
         rc = lib().orc_attn_rows_split(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
@@ -223,9 +257,10 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
 
 
 def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=None,
-                       block_mask=None, kv_splits=1):
+                       block_mask=None, kv_splits=1, window=None):
     """The oracle's tiled loop with identity quantizers, fp64 throughout
-    (kv_splits > 1: the split-KV form, as for attn_rows)."""
+    (kv_splits > 1: the split-KV form; window: the sliding-window mask; as
+    for attn_rows)."""
     q = np.ascontiguousarray(q, np.float64)
     k = np.ascontiguousarray(k, np.float64)
     v = np.ascontiguousarray(v, np.float64)
@@ -233,7 +268,14 @@ def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=Non
     n, D = rows.size, q.shape[1]
     o = np.empty((n, D), np.float64)
     lse = np.empty(n, np.float64)
-    if kv_splits > 1:
+    if window is not None:
+        if block_mask is not None:
+            raise ValueError("window and block_mask are not combined")
+        frame, win, sink = _window(window)
+        rc = lib().orc_attn_rows_identity_win(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
+                                              frame, win, sink, tkv, max(int(kv_splits), 1), BQ,
+                                              _p(rows), n, _p(o), _p(lse), _threads(threads))
+    elif kv_splits > 1:
         if block_mask is not None:
             raise ValueError("kv_splits and block_mask are not combined")
         rc = lib().orc_attn_rows_identity_split(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D,
@@ -249,16 +291,22 @@ def attn_rows_identity(q, k, v, rows, mask=MASK_NONE, mb=0, tkv=TKV, threads=Non
     return o, lse
 
 
-def attn_fp64_rows(q, k, v, rows, mask=MASK_NONE, mb=0, threads=None):
-    """Full-precision softmax attention of one head from bf16 bits, fp64."""
+def attn_fp64_rows(q, k, v, rows, mask=MASK_NONE, mb=0, threads=None, window=None):
+    """Full-precision softmax attention of one head from bf16 bits, fp64
+    (window: (frame, win, sink), the sliding-window mask)."""
     q = np.ascontiguousarray(q, np.uint16)
     k = np.ascontiguousarray(k, np.uint16)
     v = np.ascontiguousarray(v, np.uint16)
     rows = np.ascontiguousarray(rows, np.int64)
     n, D = rows.size, q.shape[1]
     o = np.empty((n, D), np.float64)
-    rc = lib().orc_attn_fp64_rows(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D, mask, mb,
-                                  _p(rows), n, _p(o), _threads(threads))
+    if window is not None:
+        frame, win, sink = _window(window)
+        rc = lib().orc_attn_fp64_rows_win(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D, frame,
+                                          win, sink, _p(rows), n, _p(o), _threads(threads))
+    else:
+        rc = lib().orc_attn_fp64_rows(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], D, mask, mb,
+                                      _p(rows), n, _p(o), _threads(threads))
     if rc:
         raise ValueError("orc_attn_fp64_rows: invalid arguments")
     return o

@@ -38,6 +38,13 @@
  *                              row and block mask to 1e-12; an all-ones mask
  *                              reproduces the dense result bit for bit; rows
  *                              that see no key give O = 0, lse = -inf.
+ *   orc_attn_rows_win / _identity_win / orc_attn_fp64_rows_win (sliding
+ *                              window + reference context): identity mode
+ *                              against textbook attention over the gathered
+ *                              visible keys to 1e-12; sink = 0 with a window
+ *                              wider than the cache reproduces the
+ *                              block-causal result bit for bit; brute-force
+ *                              visibility on small grids.
  *   orc_w8a8_quant_act / _weight : quantizer invariants (max code 127, half-
  *                              step reconstruction, zero groups, RNE ties,
  *                              block shapes).
@@ -53,7 +60,12 @@
 
 #define ORC_BLK 64 /* Q/K quantization block: 64 tokens */
 
-enum { ORC_MASK_NONE = 0, ORC_MASK_CAUSAL = 1, ORC_MASK_BLOCK_CAUSAL = 2 };
+enum {
+    ORC_MASK_NONE = 0,
+    ORC_MASK_CAUSAL = 1,
+    ORC_MASK_BLOCK_CAUSAL = 2,
+    ORC_MASK_SLIDING_WINDOW = 3
+};
 
 /* ------------------------------------------------------------------ */
 /* bf16                                                               */
@@ -351,6 +363,51 @@ long orc_row_limit(long i, long nq, long nkv, int mask, long mb)
     return lim < nkv ? lim : nkv;
 }
 
+/* The keys visible to query row i, as the union [0, sink_end) u [lo, hi).
+ * For the none / causal / block-causal masks: sink_end = 0, lo = 0 and
+ * hi = orc_row_limit.
+ *
+ * Sliding window with a persistent reference context (Vidu S1 digest,
+ * section "Infra", the sliding-window decoding paragraph): every step
+ * attends to a fixed-length window made of (1) the reference context, the
+ * tokens taken once from the first frame and the first generated state and
+ * kept for the whole stream (the role of a sink token), (2) the cached
+ * history states inside the window, (3) the state being denoised.  Reading
+ * taken: the cache holds the reference context at positions [0, sink) and
+ * then frames of mb tokens; a query at position g >= sink belongs to frame
+ * f = (g - sink) / mb and sees the whole reference context plus frames
+ * f - win + 1 .. f (its own frame in full, as the block-causal mask does);
+ * a query inside the reference context sees the reference context only.
+ * With sink = 0 and win >= the number of frames this is the block-causal
+ * mask with block mb. */
+static void orc_row_window(long i, long nq, long nkv, int mask, long mb, long win, long sink,
+                           long *sink_end, long *lo, long *hi)
+{
+    *sink_end = 0;
+    *lo = 0;
+    if (mask != ORC_MASK_SLIDING_WINDOW) {
+        *hi = orc_row_limit(i, nq, nkv, mask, mb);
+        return;
+    }
+    const long g = i + (nkv - nq);
+    const long s0 = sink < nkv ? sink : nkv;
+    if (g < s0) {
+        *hi = s0;
+        return;
+    }
+    const long f = (g - s0) / mb;
+    const long end = s0 + (f + 1) * mb;
+    const long first = f - win + 1 > 0 ? f - win + 1 : 0;
+    *sink_end = s0;
+    *lo = s0 + first * mb;
+    *hi = end < nkv ? end : nkv;
+}
+
+static int key_visible(long j, long sink_end, long lo, long hi)
+{
+    return j < sink_end || (j >= lo && j < hi);
+}
+
 /* ------------------------------------------------------------------ */
 /* Attention, one query row at a time                                  */
 /* ------------------------------------------------------------------ */
@@ -383,6 +440,9 @@ typedef struct {
     /* split-KV form (see attend_row): number of KV ranges, <= 1 for none;
      * bq is then the query tile height */
     int splits;
+    /* sliding-window mask (mask == ORC_MASK_SLIDING_WINDOW): frames of mb
+     * tokens, win frames per window, sink reference-context tokens */
+    long win, sink;
 } attn_job;
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
@@ -421,9 +481,10 @@ static double e4m3_flip_gap(double y, double eps)
  *   O     = O_acc * vs[d] / l;  lse = (m + log2(l) - 8) * ln 2.
  * Identity mode: t_ij = (q_i . k_j) * log2(e)/sqrt(D), w = p, all fp64.
  */
-/* Online softmax of query row i over the KV tiles [t_begin, t_end) (keys
- * below lim only), in ascending order: on return o holds the unnormalized
- * sum of P.V in the units of the final running maximum (m, or mf and lf in
+/* Online softmax of query row i over the KV tiles tl[0 .. nt) (ascending),
+ * keys [0, se) u [lo, hi) only; a tile without a visible key leaves the row
+ * unchanged and is passed over.  On return o holds the unnormalized sum of
+ * P.V in the units of the final running maximum (m, or mf and lf in
  * quantized mode), sl its rounding slack.  o and sl start at zero. */
 typedef struct {
     double *o, *sl;
@@ -431,8 +492,9 @@ typedef struct {
     float mf, lf;
 } attn_part;
 
-static void attend_range(const attn_job *J, long i, long lim, long t_begin, long t_end,
-                         attn_part *P, double *acc, double *sacc, int32_t *S, float *c, double *t)
+static void attend_range(const attn_job *J, long i, long se, long lo, long hi, const long *tl,
+                         long nt, attn_part *P, double *acc, double *sacc, int32_t *S, float *c,
+                         double *t, long *js)
 {
     const int D = J->D;
     const long tkv = J->tkv;
@@ -451,14 +513,19 @@ static void attend_range(const attn_job *J, long i, long lim, long t_begin, long
             sl[d] = 0.0;
     }
 
-    for (long j0 = t_begin * tkv; j0 < lim && j0 < t_end * tkv; j0 += tkv) {
-        if (J->bmask && !J->bmask[(i / J->bq) * J->n_kt + j0 / tkv])
+    for (long ti = 0; ti < nt; ti++) {
+        const long j0 = tl[ti] * tkv;
+        if (J->bmask && !J->bmask[(i / J->bq) * J->n_kt + tl[ti]])
             continue; /* tile switched off by the block mask */
-        long j1 = j0 + tkv < lim ? j0 + tkv : lim; /* visible keys of this tile */
-        long nj = j1 - j0;
+        long nj = 0; /* visible keys of this tile, ascending */
+        for (long j = j0; j < j0 + tkv && j < J->nkv; j++)
+            if (key_visible(j, se, lo, hi))
+                js[nj++] = j;
+        if (nj == 0)
+            continue;
         /* scores */
         for (long jj = 0; jj < nj; jj++) {
-            long j = j0 + jj;
+            long j = js[jj];
             if (J->identity) {
                 double s = 0.0;
                 for (int d = 0; d < D; d++)
@@ -497,7 +564,7 @@ static void attend_range(const attn_job *J, long i, long lim, long t_begin, long
         double rowsum = 0.0;
         float rowsum_f = 0.0f;
         for (long jj = 0; jj < nj; jj++) {
-            long j = j0 + jj;
+            long j = js[jj];
             if (J->identity) {
                 double p = exp2(t[jj] - m);
                 rowsum += p;
@@ -535,8 +602,9 @@ static void attend_range(const attn_job *J, long i, long lim, long t_begin, long
 
 /* One query row.  Without KV splits: one online softmax over all the row's
  * tiles.  With J->splits = S > 1 (the split-KV form of the device kernel):
- * the KV tiles the row's 128-query tile visits, [0, nk) with nk set by the
- * tile's last row, are cut into S contiguous ranges [floor(s nk / S),
+ * the KV tiles of the row's query tile (bq rows), i.e. the tiles holding a
+ * key visible to at least one of its rows, ascending, nk of them, are cut
+ * into S contiguous ranges of that sequence [floor(s nk / S),
  * floor((s+1) nk / S)); each range runs its own online softmax; the partial
  * results are merged with m = max_s m_s, a_s = exp2(m_s - m) (0 for an empty
  * range), O = sum_s a_s O_s and l = sum_s a_s l_s (fp32, ascending s, each
@@ -545,8 +613,12 @@ static void attend_row(const attn_job *J, long r)
 {
     const long i = J->rows[r];
     const int D = J->D;
-    const long lim = orc_row_limit(i, J->nq, J->nkv, J->mask, J->mb);
+    long se, lo, hi;
+    orc_row_window(i, J->nq, J->nkv, J->mask, J->mb, J->win, J->sink, &se, &lo, &hi);
     const long tkv = J->tkv;
+    const long n_all = (J->nkv + tkv - 1) / tkv;
+    long *tl = (long *)malloc(sizeof(long) * (size_t)(n_all > 0 ? n_all : 1));
+    long *js = (long *)malloc(sizeof(long) * (size_t)tkv);
     double *o = J->o + r * D;
     double *sl = J->slack ? J->slack + r * D : NULL;
     double *acc = (double *)calloc((size_t)D, sizeof(double));
@@ -560,24 +632,39 @@ static void attend_row(const attn_job *J, long r)
     const int nsplit = J->splits > 1 ? J->splits : 1;
     if (nsplit == 1) {
         attn_part P = {o, sl, 0, 0, 0, 0};
-        attend_range(J, i, lim, 0, (lim + tkv - 1) / tkv, &P, acc, sacc, S, c, t);
+        long nt = 0;
+        for (long tt = 0; tt * tkv < hi; tt++)
+            tl[nt++] = tt;
+        attend_range(J, i, se, lo, hi, tl, nt, &P, acc, sacc, S, c, t, js);
         m = P.m;
         l = P.l;
         mf = P.mf;
         lf = P.lf;
     } else {
-        /* tiles of the row's query tile: those of its last row */
-        const long qlast = (i / J->bq + 1) * J->bq - 1 < J->nq - 1 ? (i / J->bq + 1) * J->bq - 1
-                                                                  : J->nq - 1;
-        const long nk = (orc_row_limit(qlast, J->nq, J->nkv, J->mask, J->mb) + tkv - 1) / tkv;
+        /* the query tile's KV tiles, by brute force over its rows */
+        const long q0 = (i / J->bq) * J->bq;
+        const long q1 = q0 + J->bq < J->nq ? q0 + J->bq : J->nq;
+        long nk = 0;
+        for (long tt = 0; tt < n_all; tt++) {
+            const long a = tt * tkv, b = a + tkv;
+            for (long rr = q0; rr < q1; rr++) {
+                long se2, lo2, hi2;
+                orc_row_window(rr, J->nq, J->nkv, J->mask, J->mb, J->win, J->sink, &se2, &lo2,
+                               &hi2);
+                if (a < se2 || (a < hi2 && lo2 < b && lo2 < hi2)) {
+                    tl[nk++] = tt;
+                    break;
+                }
+            }
+        }
         double *po = (double *)calloc((size_t)D * nsplit, sizeof(double));
         double *ps = (double *)calloc((size_t)D * nsplit, sizeof(double));
         attn_part *parts = (attn_part *)calloc((size_t)nsplit, sizeof(attn_part));
         for (int sp = 0; sp < nsplit; sp++) {
             parts[sp].o = po + (size_t)sp * D;
             parts[sp].sl = sl ? ps + (size_t)sp * D : NULL;
-            attend_range(J, i, lim, nk * sp / nsplit, nk * (sp + 1) / nsplit, &parts[sp],
-                         acc, sacc, S, c, t);
+            const long b0 = nk * sp / nsplit, b1 = nk * (sp + 1) / nsplit;
+            attend_range(J, i, se, lo, hi, tl + b0, b1 - b0, &parts[sp], acc, sacc, S, c, t, js);
         }
         for (int d = 0; d < D; d++) {
             o[d] = 0.0;
@@ -642,6 +729,8 @@ static void attend_row(const attn_job *J, long r)
     free(S);
     free(c);
     free(t);
+    free(tl);
+    free(js);
 }
 
 /* ------------------------------------------------------------------ */
@@ -883,6 +972,7 @@ typedef struct {
     long mb;
     const long *rows;
     double *o;
+    long win, sink; /* sliding-window mask only */
 } fp64_job;
 
 static void fp64_row(const void *job, long r)
@@ -890,7 +980,8 @@ static void fp64_row(const void *job, long r)
     const fp64_job *J = (const fp64_job *)job;
     const int D = J->D;
     const long i = J->rows[r];
-    const long lim = orc_row_limit(i, J->nq, J->nkv, J->mask, J->mb);
+    long se, lo, lim;
+    orc_row_window(i, J->nq, J->nkv, J->mask, J->mb, J->win, J->sink, &se, &lo, &lim);
     double *s = (double *)malloc(sizeof(double) * (size_t)lim);
     double *qi = (double *)malloc(sizeof(double) * (size_t)D);
     double *o = J->o + r * D;
@@ -899,6 +990,8 @@ static void fp64_row(const void *job, long r)
         qi[d] = (double)bf16_to_f32(J->q[i * D + d]);
     double mx = -INFINITY;
     for (long j = 0; j < lim; j++) {
+        if (!key_visible(j, se, lo, lim))
+            continue;
         double a = 0.0;
         for (int d = 0; d < D; d++)
             a += qi[d] * (double)bf16_to_f32(J->k[j * D + d]);
@@ -910,6 +1003,8 @@ static void fp64_row(const void *job, long r)
     for (int d = 0; d < D; d++)
         o[d] = 0.0;
     for (long j = 0; j < lim; j++) {
+        if (!key_visible(j, se, lo, lim))
+            continue;
         double p = exp(s[j] - mx);
         den += p;
         for (int d = 0; d < D; d++)
@@ -931,9 +1026,108 @@ int orc_attn_fp64_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         return 1;
     if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
         return 1;
-    fp64_job J = {q, k, v, nq, nkv, D, mask, mb, rows, o};
+    fp64_job J = {q, k, v, nq, nkv, D, mask, mb, rows, o, 0, 0};
     for_rows(&J, fp64_row, nrows, nthreads);
     return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Sliding-window forms (orc_row_window): frames of mb tokens, win      */
+/* frames per window, sink reference-context tokens.                    */
+/* ------------------------------------------------------------------ */
+
+static int window_ok(long nq, long nkv, int D, long mb, long win, long sink)
+{
+    return nq > 0 && nkv >= nq && D > 0 && mb > 0 && win > 0 && sink >= 0;
+}
+
+int orc_attn_fp64_rows_win(const uint16_t *q, const uint16_t *k, const uint16_t *v, long nq,
+                           long nkv, int D, long mb, long win, long sink, const long *rows,
+                           long nrows, double *o, int nthreads)
+{
+    if (!window_ok(nq, nkv, D, mb, win, sink))
+        return 1;
+    fp64_job J = {q, k, v, nq, nkv, D, ORC_MASK_SLIDING_WINDOW, mb, rows, o, win, sink};
+    for_rows(&J, fp64_row, nrows, nthreads);
+    return 0;
+}
+
+/* Same-quantization attention under the sliding-window mask; splits > 1 is
+ * the split-KV form over the query tile's KV tiles (bq query rows). */
+int orc_attn_rows_win(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
+                      const uint8_t *v8, const float *vs, long nq, long nkv, int D, long mb,
+                      long win, long sink, long tkv, double eps, int splits, long bq,
+                      const long *rows, long nrows, double *o, double *slack, double *lse,
+                      int nthreads)
+{
+    if (!window_ok(nq, nkv, D, mb, win, sink) || tkv <= 0 || splits < 1 || bq <= 0)
+        return 1;
+    attn_job J = {0};
+    J.identity = 0;
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = ORC_MASK_SLIDING_WINDOW;
+    J.mb = mb;
+    J.win = win;
+    J.sink = sink;
+    J.tkv = tkv;
+    J.eps = eps;
+    J.q8 = q8;
+    J.qs = qs;
+    J.k8 = k8;
+    J.ks = ks;
+    J.v8 = v8;
+    J.vs = vs;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.slack = slack;
+    J.lse = lse;
+    J.bq = bq;
+    J.splits = splits;
+    if (slack)
+        memset(slack, 0, sizeof(double) * (size_t)(nrows * D));
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
+}
+
+int orc_attn_rows_identity_win(const double *q, const double *k, const double *v, long nq,
+                               long nkv, int D, long mb, long win, long sink, long tkv,
+                               int splits, long bq, const long *rows, long nrows, double *o,
+                               double *lse, int nthreads)
+{
+    if (!window_ok(nq, nkv, D, mb, win, sink) || tkv <= 0 || splits < 1 || bq <= 0)
+        return 1;
+    attn_job J = {0};
+    J.identity = 1;
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = ORC_MASK_SLIDING_WINDOW;
+    J.mb = mb;
+    J.win = win;
+    J.sink = sink;
+    J.tkv = tkv;
+    J.qd = q;
+    J.kd = k;
+    J.vd = v;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.lse = lse;
+    J.bq = bq;
+    J.splits = splits;
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
+}
+
+/* The visible-key description of one row (for the tests): out[0..2] =
+ * sink_end, lo, hi. */
+void orc_row_window_export(long i, long nq, long nkv, int mask, long mb, long win, long sink,
+                           long *out)
+{
+    orc_row_window(i, nq, nkv, mask, mb, win, sink, &out[0], &out[1], &out[2]);
 }
 
 /* ------------------------------------------------------------------ */
