@@ -17,6 +17,7 @@ the max over ranks.  `--impl reference` times the CPU oracle (the only
 reference of this method here) on a bounded sample of the same workload.
 """
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -175,12 +176,15 @@ class Runner:
         self.torch, self.sage, self.w = torch, sage, w
         # split-KV attention where the query tiles alone would leave SMs idle
         # (e.g. one streaming frame against a long cache); 1 for the video shapes
+        self.window = (w.mask_block, w.win, w.sink) if w.mask == 3 else None
         if kv_splits == "auto":
             sms = torch.cuda.get_device_properties(device).multi_processor_count
-            kv_splits = sage.suggest_kv_splits(w.B, w.H, w.Nq, w.Nkv, sms)
+            nkv = w.Nkv
+            if self.window:  # keys a query tile visits, at most
+                nkv = min(w.Nkv, w.sink + (w.win + 1) * w.mask_block + 128)
+            kv_splits = sage.suggest_kv_splits(w.B, w.H, w.Nq, nkv, sms)
         self.kv_splits = int(kv_splits)
-        wr = synth.Workload(w.name, w.B, w.H, w.Nq, w.Nkv, w.D, w.mask, w.mask_block,
-                            w.k_offset_var, w.outlier_mag, w.seed + seed_offset)
+        wr = dataclasses.replace(w, seed=w.seed + seed_offset)
         q, k, v = synth.full(wr)
 
         def pin(bits):
@@ -212,7 +216,7 @@ class Runner:
         if ev is not None:
             ev[1].record(self.stream)
         s.attn_fwd(self.qkv, self.w.mask, self.w.mask_block, out=o, stream=self.stream,
-                   kv_splits=self.kv_splits, workspace=self.split_ws)
+                   kv_splits=self.kv_splits, workspace=self.split_ws, window=self.window)
         if ev is not None:
             ev[2].record(self.stream)
 
@@ -327,14 +331,23 @@ def cpu_baseline(w, target_s):
     # calibrate on one row per thread, then size the sample to ~target_s
     cal = rng.choice(w.Nq, size=min(threads, w.Nq), replace=False)
     t0 = time.perf_counter()
-    oracle.attn_rows(qh, cal, w.mask, w.mask_block, with_slack=False, threads=threads)
+    window = (w.mask_block, w.win, w.sink) if w.mask == 3 else None
+    oracle.attn_rows(qh, cal, w.mask, w.mask_block, with_slack=False, threads=threads,
+                     window=window)
     t_cal = max(time.perf_counter() - t0, 1e-3)
     n_rows = int(min(w.Nq, max(threads, len(cal) * target_s / t_cal)))
     rows = np.sort(rng.choice(w.Nq, size=n_rows, replace=False))
     t0 = time.perf_counter()
-    oracle.attn_rows(qh, rows, w.mask, w.mask_block, with_slack=False, threads=threads)
+    oracle.attn_rows(qh, rows, w.mask, w.mask_block, with_slack=False, threads=threads,
+                     window=window)
     t_attn = time.perf_counter() - t0
-    pairs = sum(oracle.row_limit(int(i), w.Nq, w.Nkv, w.mask, max(w.mask_block, 1)) for i in rows)
+    if window:
+        vis = [oracle.row_window(int(i), w.Nq, w.Nkv, 3, w.mask_block, w.win, w.sink)
+               for i in rows]
+        pairs = sum(se + hi - lo for se, lo, hi in vis)
+    else:
+        pairs = sum(oracle.row_limit(int(i), w.Nq, w.Nkv, w.mask, max(w.mask_block, 1))
+                    for i in rows)
     ops = 4 * w.D * pairs
     # charge the whole head's quantization pro rata to the sampled rows
     t = t_attn + t_quant * n_rows / w.Nq
@@ -342,6 +355,17 @@ def cpu_baseline(w, target_s):
             "sample": "%s: oracle quantization of head 0 and same-quantization attention of %d "
                       "of its %d query rows (%d threads, %.1f s)" % (w.name, n_rows, w.Nq,
                                                                       threads, t)}
+
+
+MASK_NAMES = ["none", "causal", "block_causal", "sliding_window"]
+
+
+def attn_kernel_label(w, kv_splits):
+    if w.mask == 3:
+        return ("k_attn_win (sage_attn_fwd_window)" if kv_splits == 1 else
+                "k_attn_win split + k_attn_merge (sage_attn_fwd_window, %d KV ranges)" % kv_splits)
+    return ("k_attn (sage_attn_fwd)" if kv_splits == 1 else
+            "k_attn_split + k_attn_merge (sage_attn_fwd_split, %d KV ranges)" % kv_splits)
 
 
 def run_ours(args):
@@ -395,7 +419,8 @@ def run_ours(args):
 
     value = ops_rank * world / (t["ms"] / 1e3) / 1e12
     achieved = ops_rank / (t["attn_ms"] / 1e3) / 1e12
-    traffic = recorded_traffic() if kv_splits == 1 else None  # the dense kernel's record
+    # the dense kernel's record
+    traffic = recorded_traffic() if kv_splits == 1 and w.mask != 3 else None
     # algorithmic bytes of sage_quant_qk: read bf16 (2 B) and write one 8-bit
     # code (1 B) per element of Q, K and V, plus the scales and the K mean
     quant_bytes = 3 * w.B * w.H * (w.Nq + 2 * w.Nkv) * w.D + 4 * w.B * w.H * (
@@ -406,16 +431,13 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "i8+e4m3 (fp32 softmax)", "data": "synthetic (seeded N(0,1) bf16, K outliers)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nkv": w.Nkv, "D": w.D,
-                   "mask": ["none", "causal", "block_causal"][w.mask],
+                   "mask": MASK_NAMES[w.mask],
                    "mask_block": w.mask_block, "ops_per_step_per_gpu": ops_rank,
                    "l2": "inputs (%.2f GB bf16 Q/K/V per GPU) larger than the 126 MB L2; no flush"
                          % in_gb,
                    "parallelism": "replica per GPU (dp%d, no collective)" % world,
                    "kv_splits": kv_splits},
-        "roofline": {"bound": "tensor",
-                     "kernel": "k_attn (sage_attn_fwd)" if kv_splits == 1 else
-                               "k_attn_split + k_attn_merge (sage_attn_fwd_split, %d KV ranges)"
-                               % kv_splits,
+        "roofline": {"bound": "tensor", "kernel": attn_kernel_label(w, kv_splits),
                      "achieved": round(achieved, 2), "peak": round(pk["i8_sustained"], 1),
                      "unit": "TFLOP/s", "frac": round(achieved / pk["i8_sustained"], 4),
                      "peak_note": "8-bit dense = 2 x %s sustained cuBLAS bf16 (of %s)" % (
@@ -432,6 +454,8 @@ def run_ours(args):
         "clocks": clk,
         "e2e": e2e,
     }
+    if w.mask == 3:
+        line["config"].update(window_frames=w.win, sink_tokens=w.sink)
     if secondary:
         line["also"] = secondary
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -74,6 +74,8 @@ def lib():
         L.sage_attn_fwd_split.argtypes = [P, P, I, I, I, P, SZ, P, P, P, P]
         L.sage_attn_split_workspace_bytes.restype = SZ
         L.sage_attn_split_workspace_bytes.argtypes = [P, I]
+        L.sage_attn_fwd_window.restype = I
+        L.sage_attn_fwd_window.argtypes = [P, P, I, I, I, I, P, SZ, P, P, P, P]
         L.sage_attn_fwd_block_sparse.restype = I
         L.sage_attn_fwd_block_sparse.argtypes = [P, P, I, I, P, P, P, P, P]
         L.sage_debug_qk_int32.restype = I
@@ -249,14 +251,17 @@ def attn_split_workspace_bytes(shape, kv_splits):
 
 
 def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, stream=None,
-             block_mask=None, kv_splits=1, workspace=None):
+             block_mask=None, kv_splits=1, workspace=None, window=None):
     """sage_attn_fwd on a QuantizedQKV; returns the bf16 output tensor.
 
     block_mask: optional contiguous uint8 CUDA tensor of block_mask_shape();
     tiles whose byte is 0 are skipped (sage_attn_fwd_block_sparse).
     kv_splits: > 1 runs the split-KV form (sage_attn_fwd_split) with that
     many KV ranges per query tile; "auto" picks one with suggest_kv_splits.
-    workspace: its device scratch (allocated here when None)."""
+    workspace: its device scratch (allocated here when None).
+    window: (frame_len, window_frames, sink_tokens) runs the sliding-window
+    mask with a reference context (sage_attn_fwd_window; mask and mask_block
+    are then ignored)."""
     import torch
     s = qkv.shape
     dev = qkv.bufs["q_i8"].device
@@ -265,7 +270,28 @@ def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, 
     st = qkv.struct()
     if kv_splits == "auto":
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        kv_splits = suggest_kv_splits(s.B, s.H, s.Nq, s.Nkv, sms)
+        nkv = s.Nkv
+        if window is not None:  # keys a query tile visits, at most
+            frame, win, sink = (int(x) for x in window)
+            nkv = min(s.Nkv, sink + (win + 1) * frame + 128)
+        kv_splits = suggest_kv_splits(s.B, s.H, s.Nq, nkv, sms)
+    if window is not None:
+        if block_mask is not None:
+            raise ValueError("window and block_mask are not combined")
+        frame, win, sink = (int(x) for x in window)
+        ws_ptr, ws_bytes = None, 0
+        if kv_splits != 1:
+            need = attn_split_workspace_bytes(s, kv_splits)
+            if need == 0:
+                raise ValueError("kv_splits must be in 1..16")
+            if workspace is None:
+                workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+            ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+        _check(lib().sage_attn_fwd_window(ctypes.byref(st), ctypes.byref(s), frame, win, sink,
+                                          int(kv_splits), ws_ptr, ws_bytes, _ptr(out),
+                                          _ptr(o_f32), _ptr(lse), _stream(stream)),
+               "sage_attn_fwd_window")
+        return out
     if kv_splits != 1:
         if block_mask is not None:
             raise ValueError("kv_splits and block_mask are not combined")
@@ -300,19 +326,26 @@ def attn_fwd(qkv, mask=MASK_NONE, mask_block=0, out=None, o_f32=None, lse=None, 
 def attention(q, k, v, mask=None, stream=None, kv_splits="auto"):
     """Drop-in quantized attention: bf16 [B, H, N, D] in, bf16 out.
 
+    mask: None, "causal", ("block_causal", n) or ("window", frame_len,
+    window_frames, sink_tokens) -- the sliding window with a reference context
+    of streaming generation (sage_attn_fwd_window).
     kv_splits: "auto" runs the split-KV form when the query tiles alone would
     leave the GPU idle (e.g. one streaming frame against a long cache); an
     int forces a split count (1: never split)."""
+    window = None
     if mask is None or mask == "none":
         m, mb = MASK_NONE, 0
     elif mask == "causal":
         m, mb = MASK_CAUSAL, 0
     elif isinstance(mask, tuple) and mask[0] == "block_causal":
         m, mb = MASK_BLOCK_CAUSAL, int(mask[1])
+    elif isinstance(mask, tuple) and mask[0] == "window" and len(mask) == 4:
+        m, mb, window = MASK_NONE, 0, tuple(int(x) for x in mask[1:])
     else:
-        raise ValueError("mask must be None, 'causal' or ('block_causal', n)")
+        raise ValueError("mask must be None, 'causal', ('block_causal', n) or "
+                         "('window', frame_len, window_frames, sink_tokens)")
     qkv = quant_qk(q, k, v, stream=stream)
-    return attn_fwd(qkv, m, mb, stream=stream, kv_splits=kv_splits)
+    return attn_fwd(qkv, m, mb, stream=stream, kv_splits=kv_splits, window=window)
 
 
 def debug_qk_int32(qkv, tiles, stream=None):

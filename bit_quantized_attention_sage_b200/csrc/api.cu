@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -372,16 +373,23 @@ size_t split_ws_bytes(const sage_shape* s, int splits) {
   return static_cast<size_t>(splits) * rows * (static_cast<size_t>(s->D) + 2) * 4;
 }
 
+// The sliding-window parameters (mask == kMaskSlidingWindow only).
+struct WindowSpec {
+  int frame, win, sink;
+};
+
 sage_status attn_common(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
                         int mask_block, const uint8_t* block_mask, void* o_bf16, float* o_f32,
                         float* lse, void* stream, int splits = 1, void* workspace = nullptr,
-                        size_t ws_bytes = 0) {
+                        size_t ws_bytes = 0, WindowSpec ws = WindowSpec{1, 1, 0}) {
   if (!shape_ok(shape) || !qkv_ok(qkv) || !aligned16(o_bf16)) return SAGE_ERR_INVALID_ARG;
   if (o_f32 && !aligned16(o_f32)) return SAGE_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SAGE_ERR_INVALID_ARG;
-  if (mask < SAGE_MASK_NONE || mask > SAGE_MASK_BLOCK_CAUSAL) return SAGE_ERR_INVALID_ARG;
+  if (mask < SAGE_MASK_NONE || mask > kMaskSlidingWindow) return SAGE_ERR_INVALID_ARG;
   if (mask != SAGE_MASK_NONE && shape->Nkv < shape->Nq) return SAGE_ERR_INVALID_ARG;
   if (mask == SAGE_MASK_BLOCK_CAUSAL && mask_block < 1) return SAGE_ERR_INVALID_ARG;
+  if (mask == kMaskSlidingWindow && (block_mask || ws.frame < 1 || ws.win < 1 || ws.sink < 0))
+    return SAGE_ERR_INVALID_ARG;
   DeviceState* d = device_state();
   if (!d) return SAGE_ERR_CUDA;
   AttnMaps maps;
@@ -389,6 +397,13 @@ sage_status attn_common(const sage_qkv_quant* qkv, const sage_shape* shape, int 
   AttnParams p = base_params(qkv, shape, d);
   p.mask = mask;
   p.mask_block = mask == SAGE_MASK_BLOCK_CAUSAL ? mask_block : 1;
+  if (mask == kMaskSlidingWindow) {
+    // frames, windows or a reference context longer than the keys act as if
+    // they were Nkv long; clamping keeps the kernel's key arithmetic in int
+    p.mask_block = std::min(ws.frame, shape->Nkv);
+    p.win = std::min(ws.win, shape->Nkv);
+    p.sink = std::min(ws.sink, shape->Nkv);
+  }
   p.o = static_cast<__nv_bfloat16*>(o_bf16);
   p.o_f32 = o_f32;
   p.lse = lse;
@@ -409,11 +424,14 @@ sage_status attn_common(const sage_qkv_quant* qkv, const sage_shape* shape, int 
   return launch_attn(maps, p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
                                                                                 : SAGE_ERR_CUDA;
 }
+
+bool public_mask(int mask) { return mask >= SAGE_MASK_NONE && mask <= SAGE_MASK_BLOCK_CAUSAL; }
 }  // namespace
 
 SAGE_EXPORT sage_status sage_attn_fwd(const sage_qkv_quant* qkv, const sage_shape* shape, int mask,
                                       int mask_block, void* o_bf16, float* o_f32, float* lse,
                                       void* stream) {
+  if (!public_mask(mask)) return SAGE_ERR_INVALID_ARG;
   return attn_common(qkv, shape, mask, mask_block, nullptr, o_bf16, o_f32, lse, stream);
 }
 
@@ -427,7 +445,7 @@ SAGE_EXPORT sage_status sage_attn_fwd_split(const sage_qkv_quant* qkv, const sag
                                             void* workspace, size_t workspace_bytes,
                                             void* o_bf16, float* o_f32, float* lse,
                                             void* stream) {
-  if (!shape_ok(shape) || kv_splits < 1 || kv_splits > kAttnMaxSplits)
+  if (!shape_ok(shape) || kv_splits < 1 || kv_splits > kAttnMaxSplits || !public_mask(mask))
     return SAGE_ERR_INVALID_ARG;
   if (kv_splits == 1)
     return attn_common(qkv, shape, mask, mask_block, nullptr, o_bf16, o_f32, lse, stream);
@@ -442,9 +460,26 @@ SAGE_EXPORT sage_status sage_attn_fwd_block_sparse(const sage_qkv_quant* qkv,
                                                    int mask_block, const uint8_t* block_mask,
                                                    void* o_bf16, float* o_f32, float* lse,
                                                    void* stream) {
-  if (!block_mask || !shape_ok(shape)) return SAGE_ERR_INVALID_ARG;
+  if (!block_mask || !shape_ok(shape) || !public_mask(mask)) return SAGE_ERR_INVALID_ARG;
   if ((shape->Nkv + kAttnBN - 1) / kAttnBN > kAttnMaxKvTiles) return SAGE_ERR_UNSUPPORTED;
   return attn_common(qkv, shape, mask, mask_block, block_mask, o_bf16, o_f32, lse, stream);
+}
+
+SAGE_EXPORT sage_status sage_attn_fwd_window(const sage_qkv_quant* qkv, const sage_shape* shape,
+                                             int frame_len, int window_frames, int sink_tokens,
+                                             int kv_splits, void* workspace,
+                                             size_t workspace_bytes, void* o_bf16, float* o_f32,
+                                             float* lse, void* stream) {
+  if (!shape_ok(shape) || kv_splits < 1 || kv_splits > kAttnMaxSplits)
+    return SAGE_ERR_INVALID_ARG;
+  const WindowSpec ws{frame_len, window_frames, sink_tokens};
+  if (kv_splits == 1)
+    return attn_common(qkv, shape, kMaskSlidingWindow, 0, nullptr, o_bf16, o_f32, lse, stream, 1,
+                       nullptr, 0, ws);
+  if (!aligned16(workspace) || workspace_bytes < split_ws_bytes(shape, kv_splits))
+    return SAGE_ERR_INVALID_ARG;
+  return attn_common(qkv, shape, kMaskSlidingWindow, 0, nullptr, o_bf16, o_f32, lse, stream,
+                     kv_splits, workspace, workspace_bytes, ws);
 }
 
 SAGE_EXPORT sage_status sage_debug_qk_int32(const sage_qkv_quant* qkv, const sage_shape* shape,

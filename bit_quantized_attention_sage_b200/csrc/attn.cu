@@ -64,6 +64,50 @@ enum : int {
   kSiteMmaV, kSiteMmaP, kSiteSmS, kSiteSmO, kSiteSmEpi, kSiteDrain, kSiteSmemAlign
 };
 
+// The keys query row i sees: [0, sink_end) and [lo, hi).  Queries are the
+// newest Nq positions of the Nkv keys (position g = i + Nkv - Nq).
+//   none / causal / block-causal: sink_end = lo = 0; hi = Nkv, g + 1, or the
+//     end of g's block of mask_block keys.
+//   sliding window: sink_end = sink, the reference context, for every row;
+//     for g >= sink, [lo, hi) = frames f - win + 1 .. f of
+//     f = (g - sink) / mask_block (frames of mask_block keys after the
+//     reference context); a query inside the reference context has the
+//     empty window lo = hi = sink, i.e. sees the reference context only.
+// lo and hi never decrease with g, and hi(g) >= lo(g + 1): the rows of a
+// query tile together see [0, sink_end) and one contiguous key range.
+struct RowKeys {
+  int sink_end, lo, hi;
+};
+
+__device__ __forceinline__ RowKeys row_keys(int i, const AttnParams& p) {
+  const int g = i + (p.Nkv - p.Nq);
+  RowKeys r{0, 0, p.Nkv};
+  if (p.mask == 1) {
+    r.hi = g + 1;
+  } else if (p.mask == 2) {
+    r.hi = (g / p.mask_block + 1) * p.mask_block;
+  } else if (p.mask == kMaskSlidingWindow) {
+    r.sink_end = p.sink;
+    if (g < p.sink) {
+      r.lo = r.hi = p.sink;
+    } else {
+      const int f = (g - p.sink) / p.mask_block;
+      r.lo = p.sink + max(f - p.win + 1, 0) * p.mask_block;
+      r.hi = p.sink + (f + 1) * p.mask_block;
+    }
+  }
+  r.hi = min(r.hi, p.Nkv);
+  return r;
+}
+
+// The KV tiles of a query tile form the sequence [0, ns) then [ns + gap, ...):
+// a gap of tiles that no row sees lies between the reference context and the
+// window (sliding-window mask only; gap = 0 otherwise).
+struct TileGap {
+  int ns, gap;
+  __device__ __forceinline__ int tile(int idx) const { return idx < ns ? idx : idx + gap; }
+};
+
 template <int D>
 struct alignas(1024) Smem {
   uint8_t q[BM * D];         // int8 Q tile [128 rows][D]
@@ -96,15 +140,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(kFull, mbar_wait(bar, parity, w, site));
 }
 
-// First key index that query row i (global row) may NOT see.
-__device__ __forceinline__ int row_limit(int i, const AttnParams& p) {
-  const int g = i + (p.Nkv - p.Nq);
-  int lim = p.Nkv;
-  if (p.mask == 1) lim = g + 1;
-  else if (p.mask == 2) lim = (g / p.mask_block + 1) * p.mask_block;
-  return lim < p.Nkv ? lim : p.Nkv;
-}
-
 // Bounded wait that ignores the abort flag: used while draining copies and
 // MMAs that were already issued, so that the CTA never frees shared memory
 // or TMEM under an operation in flight.
@@ -118,19 +153,21 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
   }
 }
 
-// The KV tiles a CTA visits, in ascending order: kt0, kt0 + 1, ... (dense) or
-// the set bits of the CTA's tile bitmap (block-sparse).  next() must be
+// The KV tiles a CTA visits, in ascending order: entries kt0, kt0 + 1, ... of
+// the tile sequence (dense) or the set bits of the CTA's tile bitmap
+// (block-sparse).  next() must be
 // called at most as many times as there are tiles.
 template <bool SPARSE>
 struct TileSeq {
   const uint32_t* bits;
   int w;
   uint32_t cur;
-  __device__ __forceinline__ TileSeq(const uint32_t* b, int kt0)
-      : bits(b), w(SPARSE ? 0 : kt0), cur(SPARSE ? b[0] : 0u) {}
+  TileGap tg;
+  __device__ __forceinline__ TileSeq(const uint32_t* b, int kt0, TileGap g)
+      : bits(b), w(SPARSE ? 0 : kt0), cur(SPARSE ? b[0] : 0u), tg(g) {}
   __device__ __forceinline__ int next() {
     if constexpr (!SPARSE) {
-      return w++;
+      return tg.tile(w++);
     } else {
       while (cur == 0u) cur = bits[++w];
       const int t = w * 32 + __ffs(static_cast<int>(cur)) - 1;
@@ -142,14 +179,14 @@ struct TileSeq {
 
 template <int D, bool DUMP, bool SPARSE>
 __device__ __forceinline__ void producer(Smem<D>& s, const AttnMaps& maps, int bh, int qt,
-                                         int kt0, int nk, const WaitCtx& w) {
+                                         int kt0, int nk, TileGap tg, const WaitCtx& w) {
   tma_prefetch_desc(&maps.q);
   tma_prefetch_desc(&maps.k);
   tma_prefetch_desc(&maps.v);
   mbar_arrive_expect_tx(&s.q_full, BM * D);
   tma_load_3d(s.q, &maps.q, &s.q_full, 0, qt * BM, bh);
   int k_issued = 0, v_issued = 0;
-  TileSeq<SPARSE> seq(s.tile_bits, kt0);
+  TileSeq<SPARSE> seq(s.tile_bits, kt0, tg);
   for (int it = 0; it < nk; it++) {
     const int st = it % NS;
     const uint32_t ph = (it / NS) & 1;
@@ -257,26 +294,36 @@ __device__ __forceinline__ void rescale_row(uint32_t tO, float alpha) {
 }
 
 // Softmax / correction / epilogue for one query row per thread.
-template <int D, bool SPARSE, bool SPLIT>
+template <int D, bool SPARSE, bool SPLIT, bool WIN>
 __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, uint32_t tmem_S,
                                              uint32_t tmem_O, int bh, int qt, int kt0, int nk,
-                                             const WaitCtx& w) {
-  const int kt_base = SPLIT ? kt0 : 0;  // first KV tile (dense: 0)
+                                             TileGap tg, const WaitCtx& w) {
+  const int kt_base = SPLIT ? kt0 : 0;  // first entry of the tile sequence (dense: 0)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;               // TMEM lane quadrant of this warp
   const int r = quad * 32 + lane;          // row within the tile
   const int i = qt * BM + r;               // query row
   const bool valid = i < p.Nq;
+  // visible keys of this row: [0, p.sink) and [rk.lo, rk.hi) (sliding
+  // window), or [0, lim) (the prefix masks).  Rows past Nq are never
+  // stored; they see no key, or the reference context alone (all their
+  // scores are 0: their Q codes are zero).
+  RowKeys rk{0, 0, 0};
+  int lim = 0;
+  if (valid) {
+    if constexpr (WIN) rk = row_keys(i, p);
+    else lim = row_keys(i, p).hi;
+  }
   const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
   const uint32_t tS = tmem_S + lane_off, tO = tmem_O + lane_off;
-  const int lim = valid ? row_limit(i, p) : 0;
   const float sqC = valid ? __fmul_rn(__ldg(p.q_scale + static_cast<size_t>(bh) * p.nq_blocks + i / 64), p.c0)
                           : 0.0f;
   const float* ksc = p.k_scale + static_cast<size_t>(bh) * p.nkv_blocks;
   uint8_t* prow0 = s.p[0] + r * BN;
 
-  TileSeq<SPARSE> seq(s.tile_bits, 0);
-  int kt = (SPARSE && nk > 0) ? seq.next() : kt_base;  // KV tile of this iteration
+  TileSeq<SPARSE> seq(s.tile_bits, 0, tg);
+  // KV tile of this iteration
+  int kt = (SPARSE && nk > 0) ? seq.next() : (WIN ? tg.tile(kt_base) : kt_base);
   float ks0 = k_block_scale(ksc, 2 * kt, p.nkv_blocks);
   float ks1 = k_block_scale(ksc, 2 * kt + 1, p.nkv_blocks);
   float m = -INFINITY, l = 0.0f;
@@ -288,7 +335,7 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
   __syncwarp();
   if (lane == 0) mbar_arrive(&s.s_free);
   for (int it = 0; it < nk; it++) {
-    if constexpr (!SPARSE) kt = kt_base + it;
+    if constexpr (!SPARSE) kt = WIN ? tg.tile(kt_base + it) : kt_base + it;
     const int j0 = kt * BN;
     if (!warp_wait(&s.s_full, it & 1, w, kSiteSmS)) { ok = false; break; }
     tc_fence_after();
@@ -300,17 +347,30 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     // scale of each 64-key group of the tile; the next tile's K scales are
     // loaded now so that their latency is hidden behind this tile
     const float c0 = __fmul_rn(sqC, ks0), c1 = __fmul_rn(sqC, ks1);
-    const int kt_next = (SPARSE && more) ? seq.next() : kt + 1;
+    const int kt_next = (SPARSE && more) ? seq.next()
+                        : WIN            ? tg.tile(kt_base + it + 1)
+                                         : kt + 1;
     ks0 = k_block_scale(ksc, 2 * kt_next, p.nkv_blocks);
     ks1 = k_block_scale(ksc, 2 * kt_next + 1, p.nkv_blocks);
-    const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
-    const bool full = __all_sync(kFull, nvis == BN);
-
     // masked keys read as -inf: below every seeded score (> 2^23) in the
     // max, and exp2 of their argument is exactly 0 (see ce0, ce1, nm8)
-    if (!full) {
+    if constexpr (WIN) {
+      // visible keys of this tile: [0, na) (reference context) and [nb, nc)
+      const int na = min(max(p.sink - j0, 0), BN);
+      const int nb = min(max(rk.lo - j0, 0), BN);
+      const int nc = min(max(rk.hi - j0, 0), BN);
+      if (!__all_sync(kFull, na == BN || (nb == 0 && nc == BN))) {
+        const uint32_t nbc = static_cast<uint32_t>(nc - nb);  // nb <= nc
 #pragma unroll
-      for (int j = 0; j < BN; j++) sv[j] = j < nvis ? sv[j] : kNegInfBits;
+        for (int j = 0; j < BN; j++)
+          sv[j] = (j < na || static_cast<uint32_t>(j - nb) < nbc) ? sv[j] : kNegInfBits;
+      }
+    } else {
+      const int nvis = min(max(lim - j0, 0), BN);  // visible keys of this tile
+      if (!__all_sync(kFull, nvis == BN)) {
+#pragma unroll
+        for (int j = 0; j < BN; j++) sv[j] = j < nvis ? sv[j] : kNegInfBits;
+      }
     }
     // masked max per 64-key group on the seeded values, a tree of 3-input
     // maxima (monotone in S; for c >= 0, max_j fp32(S_j c) = fp32(max_j S_j c))
@@ -499,7 +559,7 @@ __device__ __forceinline__ void dump_rows(Smem<D>& s, const AttnParams& p, uint3
   if (lane == 0) mbar_arrive(&s.s_free);
 }
 
-template <int D, bool DUMP, bool SPARSE, bool SPLIT>
+template <int D, bool DUMP, bool SPARSE, bool SPLIT, bool WIN>
 __device__ __forceinline__ void attn_body(const AttnMaps& maps, const AttnParams& p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 128-byte swizzled TMA tiles and the MMA descriptors need 1024-byte
@@ -514,15 +574,27 @@ __device__ __forceinline__ void attn_body(const AttnMaps& maps, const AttnParams
   const int qt = DUMP ? p.dbg_qt : static_cast<int>(blockIdx.x);
   const int bh = DUMP ? p.dbg_bh : static_cast<int>(blockIdx.y);
 
-  // KV tiles this CTA visits: those holding a key visible to its last valid
-  // row (the masks' limits grow with the row index).
+  // KV tiles this CTA visits: those holding a key visible to one of its
+  // rows, i.e. the reference context's tiles [0, ns) and the tiles of
+  // [lo(first row), hi(last row)) -- one run unless a gap separates them.
   int kt0 = 0, nk;
+  TileGap tg{0, 0};
   if (DUMP) {
     kt0 = p.dbg_kt;
     nk = 1;
   } else {
     const int last = min(p.Nq - 1, qt * BM + BM - 1);
-    nk = (row_limit(last, p) + BN - 1) / BN;
+    nk = (row_keys(last, p).hi + BN - 1) / BN;
+    tg.ns = nk;
+    if (WIN) {
+      const int ts = (p.sink + BN - 1) / BN;
+      const int t_lo = row_keys(qt * BM, p).lo / BN;
+      if (t_lo > ts) {
+        tg.ns = ts;
+        tg.gap = t_lo - ts;
+        nk -= tg.gap;
+      }
+    }
     if constexpr (SPLIT) {  // range blockIdx.z of p.splits contiguous ranges
       const int sp = static_cast<int>(blockIdx.z);
       kt0 = nk * sp / p.splits;
@@ -576,12 +648,12 @@ __device__ __forceinline__ void attn_body(const AttnMaps& maps, const AttnParams
   const WaitCtx w{p.budget, p.status, &s.abort};
 
   if (warp == 0) {
-    if (lane == 0) producer<D, DUMP, SPARSE>(s, maps, bh, qt, kt0, nk, w);
+    if (lane == 0) producer<D, DUMP, SPARSE>(s, maps, bh, qt, kt0, nk, tg, w);
   } else if (warp == 1) {
     if (lane == 0) mma_issuer<D, DUMP>(s, tmem_S, tmem_O, nk, w);
   } else {
     if (DUMP) dump_rows<D>(s, p, tmem_S, w);
-    else softmax_rows<D, SPARSE, SPLIT>(s, p, tmem_S, tmem_O, bh, qt, kt0, nk, w);
+    else softmax_rows<D, SPARSE, SPLIT, WIN>(s, p, tmem_S, tmem_O, bh, qt, kt0, nk, tg, w);
   }
   __syncwarp();
   tc_fence_before();
@@ -595,7 +667,7 @@ __device__ __forceinline__ void attn_body(const AttnMaps& maps, const AttnParams
 template <int D, bool DUMP, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 2)
     k_attn(const __grid_constant__ AttnMaps maps, const AttnParams p) {
-  attn_body<D, DUMP, SPARSE, false>(maps, p);
+  attn_body<D, DUMP, SPARSE, false, false>(maps, p);
 }
 
 // Split-KV: CTA (qt, bh, range) over its range of the query tile's KV tiles;
@@ -603,7 +675,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     k_attn_split(const __grid_constant__ AttnMaps maps, const AttnParams p) {
-  attn_body<D, false, false, true>(maps, p);
+  attn_body<D, false, false, true, false>(maps, p);
+}
+
+// Sliding window with a reference context (mask kMaskSlidingWindow): the
+// query tile's tiles are the reference context's and the window's, with the
+// gap between them skipped; SPLIT as k_attn_split.
+template <int D, bool SPLIT>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_attn_win(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  attn_body<D, false, false, SPLIT, true>(maps, p);
 }
 
 // Merge of the split-KV partials, 8 rows per 128-thread CTA, thread t: row
@@ -671,8 +752,15 @@ cudaError_t prepare_one() {
 }
 template <int D>
 cudaError_t prepare_split() {
-  return cudaFuncSetAttribute(k_attn_split<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(smem_bytes_for(D)));
+  cudaError_t e = cudaFuncSetAttribute(k_attn_split<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_bytes_for(D)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_attn_win<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for(D)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_attn_win<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_for(D)));
+  return e;
 }
 }  // namespace
 
@@ -695,6 +783,18 @@ cudaError_t attn_prepare(int D) {
 cudaError_t launch_attn(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
   dim3 grid((p.Nq + BM - 1) / BM, p.BH);
   const bool sparse = p.bmask != nullptr;
+  if (p.mask == kMaskSlidingWindow) {  // never block-sparse
+    const size_t sm = smem_bytes_for(p.D);
+    if (p.splits > 1) {
+      grid.z = p.splits;
+      if (p.D == 128) k_attn_win<128, true><<<grid, kThreads, sm, stream>>>(maps, p);
+      else k_attn_win<64, true><<<grid, kThreads, sm, stream>>>(maps, p);
+    } else {
+      if (p.D == 128) k_attn_win<128, false><<<grid, kThreads, sm, stream>>>(maps, p);
+      else k_attn_win<64, false><<<grid, kThreads, sm, stream>>>(maps, p);
+    }
+    return cudaGetLastError();
+  }
   if (p.splits > 1) {  // split-KV partials; launch_attn_merge combines them
     grid.z = p.splits;
     if (p.D == 128) k_attn_split<128><<<grid, kThreads, smem_bytes_for(128), stream>>>(maps, p);

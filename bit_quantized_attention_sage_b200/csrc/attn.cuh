@@ -17,9 +17,15 @@ constexpr int kAttnMaxKvTiles = 6144;
 // split-KV mode: at most this many KV ranges per query tile
 constexpr int kAttnMaxSplits = 16;
 
+// mask ids: 0 none, 1 causal, 2 block-causal (block mask_block), 3 sliding
+// window with a reference context (frames of mask_block tokens after `sink`
+// reference tokens, `win` frames per window)
+constexpr int kMaskSlidingWindow = 3;
+
 struct AttnParams {
   int BH, Nq, Nkv, D;
   int mask, mask_block;
+  int win, sink;              // sliding-window mask only (sink <= Nkv, mask_block <= Nkv)
   int nq_blocks, nkv_blocks;  // ceil(N / 64)
   const float* q_scale;       // [BH, nq_blocks]
   const float* k_scale;       // [BH, nkv_blocks]

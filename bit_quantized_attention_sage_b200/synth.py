@@ -31,12 +31,14 @@ class Workload:
     Nq: int
     Nkv: int
     D: int
-    mask: int = 0          # 0 none, 1 causal, 2 block-causal
-    mask_block: int = 0
+    mask: int = 0          # 0 none, 1 causal, 2 block-causal, 3 sliding window
+    mask_block: int = 0    # block (2) or frame (3) length
     k_offset_var: float = 0.0
     outlier_mag: float = 0.0
     seed: int = 0
     extra: dict = field(default_factory=dict, compare=False, hash=False)
+    win: int = 0           # sliding window: frames per window
+    sink: int = 0          # sliding window: reference-context tokens
 
     def visible_pairs(self) -> int:
         """Number of (query, key) pairs that the mask leaves visible, per head."""
@@ -46,6 +48,12 @@ class Workload:
             lim = g + 1
         elif self.mask == 2:
             lim = (g // self.mask_block + 1) * self.mask_block
+        elif self.mask == 3:
+            s0 = min(self.sink, nkv)
+            f = np.maximum(g - s0, 0) // self.mask_block
+            hi = np.minimum(s0 + (f + 1) * self.mask_block, nkv)
+            lo = s0 + np.maximum(f - self.win + 1, 0) * self.mask_block
+            return int(np.where(g < s0, s0, s0 + hi - lo).sum())
         else:
             lim = np.full(nq, nkv, np.int64)
         return int(np.minimum(lim, nkv).sum())
@@ -107,6 +115,12 @@ def full(w: Workload, threads: int = 8):
 TINY = Workload("tiny_b1h2_n1024_d128", 1, 2, 1024, 1024, 128, k_offset_var=4.0, seed=1001)
 STREAMING = Workload("streaming_b1h24_nq2040_nkv26520_d128_blockcausal2040", 1, 24, 2040, 26520,
                      128, mask=2, mask_block=2040, k_offset_var=4.0, seed=1002)
+# one streaming step under the sliding window: the newest frame (2040
+# tokens) against a cache whose first frame is the reference context,
+# attending to it and the 4 newest frames (its own included)
+STREAMING_WINDOW = Workload("streaming_window_b1h24_nq2040_nkv26520_d128_frame2040_win4_sink2040",
+                            1, 24, 2040, 26520, 128, mask=3, mask_block=2040, k_offset_var=4.0,
+                            seed=1005, win=4, sink=2040)
 P480 = Workload("video480p_b1h12_n32760_d128", 1, 12, 32760, 32760, 128, outlier_mag=20.0,
                 seed=1003)
 P720 = Workload("video720p_b1h40_n75600_d128", 1, 40, 75600, 75600, 128, outlier_mag=20.0,
@@ -129,4 +143,4 @@ def sweep():
     return pts
 
 
-WORKLOADS = {w.name: w for w in (TINY, STREAMING, P480, P720)}
+WORKLOADS = {w.name: w for w in (TINY, STREAMING, STREAMING_WINDOW, P480, P720)}

@@ -273,6 +273,41 @@ sage_status sage_attn_fwd_split(const sage_qkv_quant *qkv, const sage_shape *sha
                                 size_t workspace_bytes, void *o_bf16, float *o_f32, float *lse,
                                 void *stream);
 
+/* sage_attn_fwd under a sliding window with a persistent reference context:
+ * the attention of streaming generation, where every step attends to a
+ * fixed-length window made of the reference context (tokens taken once
+ * from the first frame and the first generated state, kept for the whole
+ * stream, in the role of a sink token), the cached history frames inside
+ * the window and the frame being denoised (Vidu S1 digest, section "Infra",
+ * sliding-window decoding paragraph).
+ *
+ * Key layout read: the reference context at positions [0, sink_tokens),
+ * then frames of frame_len tokens.  Queries are the newest Nq of the Nkv
+ * positions (query i sits at g = i + Nkv - Nq).  A query with g >= sink_tokens
+ * in frame f = (g - sink_tokens) / frame_len sees the whole reference
+ * context and frames f - window_frames + 1 .. f (its own frame in full);
+ * a query inside the reference context sees the reference context only.
+ * With sink_tokens = 0 and a window of at least Nkv / frame_len + 1 frames
+ * this is SAGE_MASK_BLOCK_CAUSAL with mask_block = frame_len, bit for bit.
+ *
+ * Only tiles holding a visible key are computed: a query tile visits the
+ * reference context's tiles and then, past a gap it never touches, the
+ * window's; the online softmax runs over that sequence in ascending order.
+ * kv_splits > 1 cuts the sequence into ranges and merges them as
+ * sage_attn_fwd_split does (workspace: sage_attn_split_workspace_bytes);
+ * kv_splits = 1 needs no workspace (pass NULL, 0).
+ *
+ *   frame_len >= 1, window_frames >= 1, sink_tokens >= 0 (values above Nkv
+ *   act as Nkv).  Other arguments: as for sage_attn_fwd_split.
+ * Enqueues one kernel (kv_splits = 1) or two on `stream`.
+ * Errors: SAGE_ERR_INVALID_ARG for Nkv < Nq, a parameter out of range, or a
+ * missing, misaligned or too small workspace when kv_splits > 1; otherwise
+ * as sage_attn_fwd. */
+sage_status sage_attn_fwd_window(const sage_qkv_quant *qkv, const sage_shape *shape,
+                                 int frame_len, int window_frames, int sink_tokens,
+                                 int kv_splits, void *workspace, size_t workspace_bytes,
+                                 void *o_bf16, float *o_f32, float *lse, void *stream);
+
 /* Debug: run the attention kernel's load + INT8 MMA path on selected tiles
  * and copy the int32 score tile it leaves in tensor memory to `out`.
  *   tiles  host int array of n_tiles triples (bh, qt, kt): head index b*H+h,

@@ -59,12 +59,13 @@ def bf16_half_ulp(x):
 
 
 def check_rows(ref_head, rows, o_bf16_rows, o_f32_rows, lse_rows, mask, mb, block_mask=None,
-               kv_splits=1):
+               kv_splits=1, window=None):
     """O and lse of the given rows against the oracle (same quantized inputs;
     `block_mask`: this head's [n_qt, n_kt] tile mask, if any; `kv_splits`:
-    the split-KV form's range count)."""
+    the split-KV form's range count; `window`: (frame, win, sink) of the
+    sliding-window mask)."""
     o_ref, slack, lse_ref = oracle.attn_rows(ref_head, rows, mask, mb, block_mask=block_mask,
-                                             kv_splits=kv_splits)
+                                             kv_splits=kv_splits, window=window)
     tol = O_ATOL + slack
     err32 = np.abs(o_f32_rows.astype(np.float64) - o_ref)
     bad = err32 > tol

@@ -153,3 +153,31 @@ def test_split_attention_arguments_are_rejected_before_any_launch(L):
                                  need, p, None, None, None) == 1
     assert L.sage_attn_fwd_split(ctypes.byref(ok), ctypes.byref(s), 0, 0, 3, p, need - 1, p,
                                  None, None, None) == 1
+
+
+def test_window_attention_arguments_are_rejected_before_any_launch(L):
+    s = sage.make_shape(1, 2, 300, 700, 128)
+    ok = sage._QKV(*([16 * 1024] * 7))
+    p = ctypes.c_void_p(4096)
+    need = L.sage_attn_split_workspace_bytes(ctypes.byref(s), 3)
+
+    def call(frame, win, sink, splits=1, ws=None, nbytes=0, shape=s):
+        return L.sage_attn_fwd_window(ctypes.byref(ok), ctypes.byref(shape), frame, win, sink,
+                                      splits, ws, nbytes, p, None, None, None)
+
+    for frame, win, sink in [(0, 1, 0), (64, 0, 0), (64, 1, -1), (-5, 2, 10)]:
+        assert call(frame, win, sink) == 1
+    for splits in (0, 17):
+        assert call(64, 2, 0, splits, p, need) == 1
+    # a window needs Nkv >= Nq
+    assert call(64, 2, 0, shape=sage.make_shape(1, 2, 701, 700, 128)) == 1
+    # workspace missing, misaligned or too small when kv_splits > 1
+    assert call(64, 2, 0, 3, None, need) == 1
+    assert call(64, 2, 0, 3, ctypes.c_void_p(4100), need) == 1
+    assert call(64, 2, 0, 3, p, need - 1) == 1
+    # the window mask id is not a public sage_mask value
+    assert L.sage_attn_fwd(ctypes.byref(ok), ctypes.byref(s), 3, 64, p, None, None, None) == 1
+    assert L.sage_attn_fwd_split(ctypes.byref(ok), ctypes.byref(s), 3, 64, 3, p, need, p,
+                                 None, None, None) == 1
+    assert L.sage_attn_fwd_block_sparse(ctypes.byref(ok), ctypes.byref(s), 3, 64, p, p, None,
+                                        None, None) == 1
