@@ -1,5 +1,6 @@
 """The path captured in a CUDA graph: quantization + attention (dense and
-split-KV) and the W8A8 layer replay bit-identically to eager calls, and a
+split-KV), the streaming step (RoPE in the quantizer, sliding-window
+attention) and the W8A8 layer replay bit-identically to eager calls, and a
 replay after new inputs are copied into the captured buffers recomputes."""
 import numpy as np
 import pytest
@@ -82,3 +83,49 @@ def test_w8a8_layer_replays():
     torch.cuda.synchronize()
     assert sage.sync_status() == 0
     assert torch.equal(y, ref)
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+def test_streaming_window_step_replays(splits):
+    # the streaming step of the pages: RoPE applied to Q and K at their
+    # positions inside the quantizer, then attention under the sliding window
+    # with a reference context; captured once, replayed per step
+    Nq, Nkv, D = 600, 4000, 128
+    w = synth.Workload("graph_win", 1, 3, Nq, Nkv, D, outlier_mag=5.0, seed=21)
+    w2 = synth.Workload("graph_win2", 1, 3, Nq, Nkv, D, outlier_mag=5.0, seed=22)
+    (q, k, v), (q2, k2, v2) = synth.full(w), synth.full(w2)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    inv = 1.0 / (10000.0 ** (np.arange(D // 2) / (D // 2)))
+    ang_k = np.arange(Nkv)[:, None] * inv[None, :]
+    ang_q = ang_k[Nkv - Nq:]
+    rope = tuple(torch.from_numpy(np.ascontiguousarray(f(a)).astype(np.float32)).cuda()
+                 for a, f in ((ang_q, np.cos), (ang_q, np.sin), (ang_k, np.cos), (ang_k, np.sin)))
+    window = (600, 3, 400)
+    qkv = sage.quant_qk(qd, kd, vd, rope=rope)
+    ws = torch.empty(max(sage.workspace_bytes(qkv.shape), 16), dtype=torch.uint8, device="cuda")
+    sws = None
+    if splits > 1:
+        sws = torch.empty(sage.attn_split_workspace_bytes(qkv.shape, splits), dtype=torch.uint8,
+                          device="cuda")
+    o = torch.empty((1, 3, Nq, D), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        sage.quant_qk(qd, kd, vd, out=qkv, workspace=ws, rope=rope)
+        sage.attn_fwd(qkv, out=o, kv_splits=splits, workspace=sws, window=window)
+
+    step()
+    torch.cuda.synchronize()
+    ref = o.clone()
+    g = _capture(step)
+    o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert sage.sync_status() == 0
+    assert torch.equal(o, ref)
+    qd.copy_(to_dev(q2)); kd.copy_(to_dev(k2)); vd.copy_(to_dev(v2))
+    g.replay()
+    torch.cuda.synchronize()
+    got = o.clone()
+    step()
+    torch.cuda.synchronize()
+    assert torch.equal(got, o) and not torch.equal(got, ref)
