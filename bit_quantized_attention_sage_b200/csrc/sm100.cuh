@@ -126,7 +126,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
 
 // 3-D tiled TMA load of one box into shared memory; completion is signalled
 // as transaction bytes on `bar`.  Coordinates are element offsets, x
-// innermost.  No multicast.
+// innermost.  The box lands in this CTA's own shared memory only.
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, uint64_t* bar, int x,
                                             int y, int z) {
   asm volatile(
@@ -137,7 +137,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, uint64_t
 }
 
 // Prefetch one 3-D tile into L2 (no shared memory involved; coordinates
-// outside the tensor are ignored).  No multicast.
+// outside the tensor are ignored).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const void* map, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
