@@ -571,7 +571,10 @@ __device__ __forceinline__ void attn_body(const AttnMaps& maps, const AttnParams
   }
   Smem<D>& s = *reinterpret_cast<Smem<D>*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = DUMP ? p.dbg_qt : static_cast<int>(blockIdx.x);
+  // masked shapes: the query tiles' work grows with their index, so the
+  // heaviest are dispatched first and the last wave holds the lightest
+  const int qt = DUMP ? p.dbg_qt
+                      : static_cast<int>(p.mask != 0 ? gridDim.x - 1 - blockIdx.x : blockIdx.x);
   const int bh = DUMP ? p.dbg_bh : static_cast<int>(blockIdx.y);
 
   // KV tiles this CTA visits: those holding a key visible to one of its
