@@ -170,7 +170,7 @@ def recorded_traffic():
 class Runner:
     """Device buffers and one step of the hot path for a workload."""
 
-    def __init__(self, w, seed_offset, device, kv_splits="auto"):
+    def __init__(self, w, rank, device, kv_splits="auto"):
         import torch
         import bit_quantized_attention_sage_b200 as sage
         self.torch, self.sage, self.w = torch, sage, w
@@ -184,7 +184,7 @@ class Runner:
                 nkv = min(w.Nkv, w.sink + (w.win + 1) * w.mask_block + 128)
             kv_splits = sage.suggest_kv_splits(w.B, w.H, w.Nq, nkv, sms)
         self.kv_splits = int(kv_splits)
-        wr = dataclasses.replace(w, seed=w.seed + seed_offset)
+        wr = rank_workload(w, rank)
         q, k, v = synth.full(wr)
 
         def pin(bits):
@@ -278,13 +278,27 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of x over all ranks (a device tensor under NCCL, a host
+    tensor under gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([float(x)], device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w, rank):
+    """Each rank's replica of the workload: same shape, its own seeds (weak
+    scaling, no data exchange)."""
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def aggregate_value(ops_per_rank, world, ms_max):
+    """Whole-job TOPS: the work of all ranks over the slowest rank's time."""
+    return ops_per_rank * world / (ms_max / 1e3) / 1e12
 
 
 def time_steps(runner, steps, warmup, world, e2e=False, per_kernel=False):
@@ -383,7 +397,7 @@ def run_ours(args):
     import bit_quantized_attention_sage_b200 as sage
     sage.lib()
     w = synth.WORKLOADS[args.workload]
-    runner = Runner(w, 1000 * rank, device)
+    runner = Runner(w, rank, device)
     kv_splits = runner.kv_splits
     ops_rank = w.ops()
     pk = peaks()
@@ -399,7 +413,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         te = time_steps(runner, args.steps, max(1, args.warmup), world, e2e=True)
-        e2e = {"value": ops_rank * world / (te["ms"] / 1e3) / 1e12, "unit": UNIT,
+        e2e = {"value": aggregate_value(ops_rank, world, te["ms"]), "unit": UNIT,
                "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
                "ms_per_step": te["ms"],
                "copies": "pinned host <-> device every step; the H2D of step i+1 and the D2H of "
@@ -409,15 +423,15 @@ def run_ours(args):
     if not args.no_secondary and w.name != synth.P480.name:
         del runner
         torch.cuda.empty_cache()
-        r2 = Runner(synth.P480, 1000 * rank, device)
+        r2 = Runner(synth.P480, rank, device)
         t2 = time_steps(r2, args.steps, args.warmup, world, per_kernel=True)
         secondary[synth.P480.name] = {
-            "value": synth.P480.ops() * world / (t2["ms"] / 1e3) / 1e12, "unit": UNIT,
+            "value": aggregate_value(synth.P480.ops(), world, t2["ms"]), "unit": UNIT,
             "ms_per_step": t2["ms"], "attn_ms": t2["attn_ms"], "quant_ms": t2["quant_ms"],
             "attn_frac_of_peak": synth.P480.ops() / (t2["attn_ms"] / 1e3) / 1e12 / pk["i8_sustained"]}
         del r2
 
-    value = ops_rank * world / (t["ms"] / 1e3) / 1e12
+    value = aggregate_value(ops_rank, world, t["ms"])
     achieved = ops_rank / (t["attn_ms"] / 1e3) / 1e12
     # the dense kernel's record
     traffic = recorded_traffic() if kv_splits == 1 and w.mask != 3 else None
