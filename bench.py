@@ -470,6 +470,11 @@ def run_ours(args):
     }
     if w.mask == 3:
         line["config"].update(window_frames=w.win, sink_tokens=w.sink)
+    if w.mask != 0:  # value counts visible pairs only; the dense formula, labelled
+        dense = 4 * w.D * w.B * w.H * w.Nq * w.Nkv
+        line["value_dense_formula"] = {
+            "value": round(aggregate_value(dense, world, t["ms"]), 3), "unit": UNIT,
+            "note": "4 Nq Nkv D H per step, masked pairs included (not the metric)"}
     if secondary:
         line["also"] = secondary
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
