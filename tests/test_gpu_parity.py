@@ -30,6 +30,10 @@ SMALL = [
       seed=36),
     W("causal_square_d64", 1, 1, 640, 640, 64, mask=1, outlier_mag=5.0, seed=37),
     W("nkv_tail_16", 1, 1, 256, 1168, 128, outlier_mag=20.0, seed=38),
+    # one row or token either side of the 64-token block and 128-row tile edges
+    W("n63_nkv65_causal", 1, 2, 63, 65, 128, mask=1, k_offset_var=4.0, seed=39),
+    W("n65_nkv127_block64_d64", 1, 1, 65, 127, 64, mask=2, mask_block=64, seed=40),
+    W("n127_none", 1, 1, 127, 127, 128, outlier_mag=5.0, seed=41),
 ]
 
 
