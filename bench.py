@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--ceilings", action="store_true",
+                    help="microbenchmarks of the hardware rates the rooflines rest on")
     ap.add_argument("--sweep", action="store_true",
                     help="time the 72-point sweep (N x D x mask x K outlier magnitude) and report "
                          "TOPS and accuracy against fp64 attention per point, one JSON line each")
@@ -708,6 +710,50 @@ def run_rope(args):
 
 # ------------------------------------------------------------------ reference arm
 
+CEILING_PLAN = [  # kind, iters, MMA N, unit of one operation
+    ("ex2", 20000, 256, "exp2 results"),
+    ("ffma2", 20000, 256, "fp32 fma lanes (packed fp32x2)"),
+    ("cvt_e4m3x2", 20000, 256, "fp32-pair -> e4m3x2 conversions"),
+    ("copy", 1, 256, "bytes read + written"),
+    ("mma_i8", 4096, 256, "int8 multiply-adds x 2 (M128 N256 K32 MMAs)"),
+    ("mma_i8", 4096, 128, "int8 multiply-adds x 2 (M128 N128 K32 MMAs)"),
+    ("mma_e4m3", 4096, 256, "e4m3 multiply-adds x 2 (M128 N256 K32 MMAs)"),
+    ("mma_e4m3", 4096, 128, "e4m3 multiply-adds x 2 (M128 N128 K32 MMAs)"),
+]
+
+
+def run_ceilings(args):
+    """Hardware ceilings (sage_ceiling): per-SM-per-clock and whole-GPU
+    rates of the exp2 unit, packed fma, e4m3 conversion, device copy and the
+    tcgen05 i8 / e4m3 MMA, the best of 3 launches each after one warm-up."""
+    import torch
+    torch.cuda.set_device(0)
+    import bit_quantized_attention_sage_b200 as sage
+    sage.lib()
+    scratch = torch.empty(4 << 30, dtype=torch.uint8, device="cuda")  # a 2 GiB copy
+    clocks = ClockSampler(0)
+    clocks.start()
+    out = []
+    for kind, iters, n, unit in CEILING_PLAN:
+        sc = scratch if kind == "copy" else None
+        sage.ceiling(kind, iters=max(1, iters // 20), n=n, scratch=sc)
+        runs = [sage.ceiling(kind, iters=iters, n=n, scratch=sc) for _ in range(3)]
+        best = max(runs, key=lambda r: r["per_second"])
+        out.append({"kind": kind, "n": n if kind.startswith("mma") else None, "unit": unit,
+                    "per_sm_per_clock": round(best["per_sm_per_clock"], 2),
+                    "per_second": best["per_second"], "ms": round(best["ms"], 4)})
+    clk = clocks.stop()
+    if sage.sync_status() != 0:
+        raise RuntimeError("device status error during the ceiling runs")
+    pk = peaks()
+    mma = {(r["kind"], r["n"]): r["per_second"] / 1e12 for r in out if r["kind"].startswith("mma")}
+    print(json.dumps({"ceilings": out, "clocks": clk,
+                      "mma_vs_peak": {"%s_n%d" % k: round(v / pk["i8_sustained"], 4)
+                                      for k, v in mma.items()},
+                      "peak_note": "8-bit sustained peak = 2 x %s cuBLAS bf16 = %.1f TOPS" % (
+                          pk["source"], pk["i8_sustained"])}), flush=True)
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -749,6 +795,8 @@ def main():
         run_w8a8(args)
     elif args.rope:
         run_rope(args)
+    elif args.ceilings:
+        run_ceilings(args)
     else:
         run_ours(args)
 

@@ -74,6 +74,8 @@ def lib():
         L.sage_attn_fwd_split.argtypes = [P, P, I, I, I, P, SZ, P, P, P, P]
         L.sage_attn_split_workspace_bytes.restype = SZ
         L.sage_attn_split_workspace_bytes.argtypes = [P, I]
+        L.sage_ceiling.restype = I
+        L.sage_ceiling.argtypes = [I, I, I, P, SZ, P, P, P, P, P]
         L.sage_attn_fwd_window.restype = I
         L.sage_attn_fwd_window.argtypes = [P, P, I, I, I, I, P, SZ, P, P, P, P]
         L.sage_attn_fwd_block_sparse.restype = I
@@ -393,6 +395,40 @@ def sync_status(stream=None):
 # ---------------------------------------------------------------- W8A8 linear layer
 
 W8A8_GROUP = 128
+
+
+CEILINGS = {"ex2": 0, "ffma2": 1, "cvt_e4m3x2": 2, "copy": 3, "mma_i8": 4, "mma_e4m3": 5}
+
+
+def ceiling(kind, iters=4096, n=256, scratch=None, stream=None):
+    """Run one hardware-ceiling microbenchmark (sage_ceiling) and return
+    {"per_sm_per_clock": median over blocks of ops_per_block * blocks_per_sm
+    / cycles, "per_second": ops of the whole launch / its CUDA-event time,
+    "ms": that time, "blocks": ...}.  kind: a key of CEILINGS.  scratch: the
+    copy's device buffer (its two halves), required for "copy"."""
+    import torch
+    k = CEILINGS[kind]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    cycles = torch.zeros(8 * sms, dtype=torch.int64, device=dev)
+    blocks, bps, opb = ctypes.c_int(), ctypes.c_int(), ctypes.c_double()
+    st = torch.cuda.current_stream(dev) if stream is None else stream
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    _check(lib().sage_ceiling(k, int(iters), int(n), _ptr(scratch),
+                              0 if scratch is None else scratch.numel() * scratch.element_size(),
+                              _ptr(cycles), ctypes.byref(blocks), ctypes.byref(bps),
+                              ctypes.byref(opb), _stream(st)), "sage_ceiling")
+    b.record(st)
+    b.synchronize()
+    ms = a.elapsed_time(b)
+    cyc = cycles[:blocks.value].float().cpu()
+    if bool((cyc <= 0).any()):
+        raise SageError(3, "sage_ceiling: a block did not record its cycles")
+    med = float(cyc.median())
+    return {"kind": kind, "per_sm_per_clock": opb.value * bps.value / med,
+            "per_second": opb.value * blocks.value / (ms / 1e3), "ms": ms,
+            "blocks": blocks.value, "blocks_per_sm": bps.value, "median_cycles": med}
 
 
 def w8a8_quant_act(x, xq=None, sx=None, stream=None):

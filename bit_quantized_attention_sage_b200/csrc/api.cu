@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "attn.cuh"
+#include "ceilings.cuh"
 #include "quant.cuh"
 #include "sage.h"
 #include "w8a8.cuh"
@@ -532,6 +533,32 @@ SAGE_EXPORT sage_status sage_debug_exp2(const float* x, float* y, size_t n, void
   if (n == 0) return SAGE_OK;
   k_exp2<<<1184, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+SAGE_EXPORT sage_status sage_ceiling(int kind, int iters, int n, void* scratch,
+                                     size_t scratch_bytes, long long* cycles, int* blocks,
+                                     int* blocks_per_sm, double* ops_per_block, void* stream) {
+  if (!cycles || (reinterpret_cast<uintptr_t>(cycles) & 7u) || !blocks || !blocks_per_sm ||
+      !ops_per_block)
+    return SAGE_ERR_INVALID_ARG;
+  if (kind < kCeilEx2 || kind > kCeilMmaF8) return SAGE_ERR_INVALID_ARG;
+  if (kind == kCeilCopy) {
+    if (!aligned16(scratch) || scratch_bytes < (1u << 20)) return SAGE_ERR_INVALID_ARG;
+  } else if (iters < 1 || iters > (1 << 24)) {
+    return SAGE_ERR_INVALID_ARG;
+  }
+  if ((kind == kCeilMmaI8 || kind == kCeilMmaF8) && n != 64 && n != 128 && n != 256)
+    return SAGE_ERR_INVALID_ARG;
+  DeviceState* d = device_state();
+  if (!d) return SAGE_ERR_CUDA;
+  CeilingArgs a{kind, iters, n, scratch, scratch_bytes, cycles, kWaitBudget, d->status};
+  CeilingInfo info{};
+  if (launch_ceiling(a, &info, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  *blocks = info.blocks;
+  *blocks_per_sm = info.blocks_per_sm;
+  *ops_per_block = info.ops_per_block;
+  return SAGE_OK;
 }
 
 SAGE_EXPORT sage_status sage_sync_status(void* stream) {

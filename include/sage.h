@@ -406,6 +406,35 @@ sage_status sage_w8a8_gemm_q(const int8_t *xq, const float *sx, const int8_t *wq
 /* Static description of a status code (never NULL). */
 const char *sage_status_string(sage_status status);
 
+/* Hardware ceilings: microbenchmarks of the rates the kernels' rooflines rest
+ * on.  One kernel launch on `stream`, whose blocks are all resident at once
+ * (one wave); block i writes the SM clock cycles of its timed loop to
+ * cycles[i].  On return (before the kernel has run) *blocks, *blocks_per_sm
+ * and *ops_per_block describe the launch, so that
+ *   rate per SM per clock = ops_per_block * blocks_per_sm / cycles[i]
+ *   whole-GPU rate        = ops_per_block * blocks / (the launch's duration).
+ *   kind 0  exp2 unit (ex2.approx.f32): iters rounds of 8 dependent chains
+ *           per thread; an operation is one exp2 result.
+ *   kind 1  packed fp32x2 fma: an operation is one fma lane.
+ *   kind 2  fp32 pair -> e4m3x2 conversion (satfinite): an operation is one
+ *           conversion instruction (two values).
+ *   kind 3  device memory copy of scratch's first half into its second half
+ *           (16-byte vectors); an operation is one byte read or written.
+ *           scratch: device, 16-byte aligned, at least 1 MiB; iters unused.
+ *   kind 4  tcgen05 kind::i8 MMA (M 128, N n, K 32, int32 accumulator in
+ *           tensor memory), one CTA per SM, one issuing thread, iters groups
+ *           of 4 MMAs; an operation is one multiply or add (2 M N K per MMA).
+ *   kind 5  the same with kind::f8f6f4, e4m3 operands, fp32 accumulator.
+ *   iters: 1 .. 2^24 (kinds 0-2, 4, 5); n: 64, 128 or 256 (kinds 4, 5).
+ *   cycles: device int64, 8-byte aligned, at least 8 x (number of SMs)
+ *   entries.  The MMA kinds' completion wait is bounded: a timeout is
+ *   reported by sage_sync_status.
+ * Errors: SAGE_ERR_INVALID_ARG for an unknown kind or an argument out of
+ * range, SAGE_ERR_CUDA if the launch fails. */
+sage_status sage_ceiling(int kind, int iters, int n, void *scratch, size_t scratch_bytes,
+                         long long *cycles, int *blocks, int *blocks_per_sm,
+                         double *ops_per_block, void *stream);
+
 /* SAGE_ABI_VERSION of the loaded library. */
 int sage_abi_version(void);
 

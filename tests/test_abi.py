@@ -181,3 +181,20 @@ def test_window_attention_arguments_are_rejected_before_any_launch(L):
                                  None, None, None) == 1
     assert L.sage_attn_fwd_block_sparse(ctypes.byref(ok), ctypes.byref(s), 3, 64, p, p, None,
                                         None, None) == 1
+
+
+def test_ceiling_arguments_are_rejected_before_any_launch(L):
+    blocks, bps, opb = ctypes.c_int(), ctypes.c_int(), ctypes.c_double()
+    cyc = ctypes.c_void_p(4096)
+
+    def call(kind, iters=10, n=256, scratch=None, nbytes=0, cycles=cyc):
+        return L.sage_ceiling(kind, iters, n, scratch, nbytes, cycles, ctypes.byref(blocks),
+                              ctypes.byref(bps), ctypes.byref(opb), None)
+
+    assert call(-1) == 1 and call(6) == 1               # unknown kinds
+    assert call(0, iters=0) == 1 and call(1, iters=(1 << 24) + 1) == 1
+    assert call(4, n=100) == 1 and call(5, n=512) == 1  # MMA N must be 64, 128 or 256
+    assert call(3, scratch=None, nbytes=1 << 30) == 1   # copy needs a scratch buffer
+    assert call(3, scratch=ctypes.c_void_p(4096), nbytes=1 << 19) == 1  # of at least 1 MiB
+    assert call(3, scratch=ctypes.c_void_p(4104), nbytes=1 << 30) == 1  # 16-byte aligned
+    assert call(0, cycles=None) == 1 and call(0, cycles=ctypes.c_void_p(4100)) == 1
