@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--ceilings", action="store_true",
                     help="microbenchmarks of the hardware rates the rooflines rest on")
+    ap.add_argument("--ceil-seconds", type=float, default=0.0,
+                    help="with --ceilings: also hold the 8-bit MMA rate this long (power cap)")
     ap.add_argument("--sweep", action="store_true",
                     help="time the 72-point sweep (N x D x mask x K outlier magnitude) and report "
                          "TOPS and accuracy against fp64 attention per point, one JSON line each")
@@ -743,11 +745,26 @@ def run_ceilings(args):
                     "per_sm_per_clock": round(best["per_sm_per_clock"], 2),
                     "per_second": best["per_second"], "ms": round(best["ms"], 4)})
     clk = clocks.stop()
+    sustained = []
+    if args.ceil_seconds > 0:
+        # the attention's MMA shapes held for ceil_seconds each: back-to-back
+        # launches of about 0.25 s, the median rate of the second half
+        for kind in ("mma_i8", "mma_e4m3"):
+            clocks = ClockSampler(0)
+            clocks.start()
+            rates, t0 = [], time.perf_counter()
+            while time.perf_counter() - t0 < args.ceil_seconds:
+                rates.append(sage.ceiling(kind, iters=1 << 21, n=128)["per_second"])
+            c2 = clocks.stop()
+            tail = rates[len(rates) // 2:]
+            sustained.append({"kind": kind, "n": 128, "seconds": args.ceil_seconds,
+                              "launches": len(rates), "per_second": float(np.median(tail)),
+                              "clocks": c2})
     if sage.sync_status() != 0:
         raise RuntimeError("device status error during the ceiling runs")
     pk = peaks()
     mma = {(r["kind"], r["n"]): r["per_second"] / 1e12 for r in out if r["kind"].startswith("mma")}
-    print(json.dumps({"ceilings": out, "clocks": clk,
+    print(json.dumps({"ceilings": out, "clocks": clk, "sustained": sustained,
                       "mma_vs_peak": {"%s_n%d" % k: round(v / pk["i8_sustained"], 4)
                                       for k, v in mma.items()},
                       "peak_note": "8-bit sustained peak = 2 x %s cuBLAS bf16 = %.1f TOPS" % (
