@@ -31,3 +31,16 @@ def test_oracle_matches_regression_fixture():
     for r, row in enumerate(make_golden.ROWS):
         assert np.allclose(orows[row]["o"], o[r, :8], rtol=1e-8, atol=1e-12)
         assert abs(orows[row]["lse"][0] - lse[r]) < 1e-10
+
+
+def test_window_oracle_matches_regression_fixture():
+    o1, l1, o3, l3 = make_golden.compute_window()
+    got = {}
+    for parts in (l.split() for l in open(make_golden.OUT_WIN) if not l.startswith("#")):
+        got[(parts[0], parts[1], int(parts[2]))] = [float(x) for x in parts[3:]]
+    for tag, o, lse in (("s1", o1, l1), ("s3", o3, l3)):
+        for r, row in enumerate(make_golden.WIN_ROWS):
+            assert np.allclose(got[("o", tag, row)], o[r, :8], rtol=1e-8, atol=1e-12)
+            assert abs(got[("lse", tag, row)][0] - lse[r]) < 1e-10
+    # the split form differs from the unsplit one by P rounding points only
+    assert np.abs(o1 - o3).max() < 0.05 and np.abs(o1 - o3).max() > 0
