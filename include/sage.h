@@ -69,6 +69,9 @@ typedef enum {
      * streaming video step): key j visible to query i iff
      * floor(j / mask_block) <= floor((i + Nkv - Nq) / mask_block). */
     SAGE_MASK_BLOCK_CAUSAL = 2
+    /* The sliding window with a persistent reference context has its own
+     * call, sage_attn_fwd_window, because it takes three parameters; it is
+     * not a sage_mask value, and the mask-taking calls reject any other. */
 } sage_mask;
 
 /* Problem shape.  Inputs are [B, H, Nq, D] (Q) and [B, H, Nkv, D] (K, V).
