@@ -218,8 +218,24 @@ cudaError_t launch_ceiling(const CeilingArgs& a, CeilingInfo* info, cudaStream_t
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const int per_sm = 8;  // 8 x 256 threads: a full SM of resident threads
   const double thr = static_cast<double>(kCeilThreads);
+  // Blocks per SM: as many as are co-resident (the occupancy calculator, for
+  // the kernel's own register use), so that every block's clock64 span
+  // covers the whole launch and ops_per_block x blocks_per_sm / cycles is a
+  // per-SM rate.  Launching more blocks than are resident runs several waves,
+  // each block spans only its own wave and that ratio over-counts the rate
+  // by the number of waves.
+  int per_sm = 0;
+  const void* fn = a.kind == kCeilEx2     ? reinterpret_cast<const void*>(k_ceil_ex2)
+                   : a.kind == kCeilFfma2 ? reinterpret_cast<const void*>(k_ceil_ffma2)
+                   : a.kind == kCeilCvt   ? reinterpret_cast<const void*>(k_ceil_cvt)
+                                          : reinterpret_cast<const void*>(k_ceil_copy);
+  if (a.kind <= kCeilCopy) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kCeilThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    per_sm = per_sm > 8 ? 8 : per_sm;  // the caller's cycles buffer holds 8 per SM
+  }
   switch (a.kind) {
     case kCeilEx2:
     case kCeilFfma2:

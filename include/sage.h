@@ -115,6 +115,14 @@ size_t sage_quant_workspace_bytes(const sage_shape *shape);
 
 /* Quantize Q, K and V (all device, bf16, contiguous [B,H,N,D]).
  *
+ * This is the quantization half of low-bit quantized attention: Q and K to
+ * 8-bit codes with per-block scales, so that Q K^T runs on INT8 tensor cores
+ * (reportify.cn TurboDiffusion notes, "混合注意力加速" and "W8A8线性层量化"
+ * bullets: SageAttention is 8-bit block-wise quantized attention on INT8
+ * tensor cores; "Vidu S1" digest, section "Infra": per-block scales because
+ * per-tensor and per-channel scales are stretched by outliers).  The block
+ * size, rounding, K smoothing and the e4m3 V are this library's readings.
+ *
  *   Q: per (b, h, 64-token block): a = max|Q| over the block, q_scale = a/127,
  *      q_i8 = clamp(round_half_even(Q * fp32(127/a)), -127, 127); a = 0 gives
  *      scale 0 and codes 0.
@@ -197,22 +205,38 @@ sage_status sage_quant_qk_rope(const void *q_bf16, const void *k_bf16, const voi
  * give undefined results; order such calls on one stream.
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current).  Make that first call
- * before any stream capture. */
+ * before any stream capture.  It sets up only this array: the attention and
+ * GEMM calls do their own one-time set-up on their first call, so a program
+ * that captures those calls needs one eager call of each before capturing. */
 sage_status sage_quant_qk_noalloc(const void *q_bf16, const void *k_bf16, const void *v_bf16,
                                   const sage_shape *shape, const sage_qkv_quant *out,
                                   void *stream);
 
 /* Fused quantized attention over the output of sage_quant_qk.
  *
+ * SageAttention-style low-bit attention, the plug-and-play replacement of
+ * FlashAttention that moves both matmuls onto 8-bit tensor cores (Crossing
+ * podcast show notes, section "硬件上明明有更快的计算单元"; reportify.cn
+ * TurboDiffusion notes, "混合注意力加速" bullet).  The arithmetic below is
+ * this library's reading of it; every step is one IEEE fp32 operation
+ * rounded to nearest-even unless stated.
+ *
  * Per query row i (row limit lim_i from `mask`, see sage_mask), over KV tiles
  * of 128 keys in ascending order (only tiles holding a visible key):
  *   S    = q_i8 . k_i8 (exact int32 on the INT8 tensor cores)
- *   c    = fp32(fp32(q_scale * C0) * k_scale), C0 = fp32(log2(e)/sqrt(D))
+ *   c    = fp32(fp32(q_scale * C0) * k_scale[j/64]), C0 = fp32(log2(e)/sqrt(D))
  *   m    = max(m, max_j fp32(S*c))   (running max in the log2 domain)
- *   p    = exp2(fma(S, c, -m)) in fp32; l = l*alpha + sum_j p
- *   P    = e4m3(p * 256); O_acc = O_acc*alpha + P . v_f8 (FP8 tensor cores,
- *          fp32 accumulation), alpha = exp2(m_old - m_new)
- *   O    = O_acc * v_scale[d] / (256 * l), rounded to bf16.
+ *   y    = exp2(fma(S, c, fp32(8 - m)))  (= 2^8 p: the fixed P scale 2^8 is
+ *          folded into the exponent argument; exp2 is the hardware
+ *          approximation, relative error below 2^-21)
+ *   l    = l*alpha + sum_j y   (fp32, from y before quantization)
+ *   P    = e4m3(y) (round to nearest even; y <= 2^8 (1 + 2^-21) never
+ *          saturates); O_acc = O_acc*alpha + P . v_f8 (FP8 tensor cores,
+ *          fp32 accumulation), alpha = exp2(m_old - m_new) (exactly 1 when
+ *          the maximum did not move, 0 before the first tile)
+ *   O    = O_acc * (v_scale[d] * (1 / l)), rounded to bf16 (l is in units of
+ *          2^8 p, so the 2^8 cancels).
+ *   lse  = (m + log2(l) - 8) * ln 2.
  * Softmax invariance makes the K-mean subtraction exact in real arithmetic.
  *
  *   mask        a sage_mask value; CAUSAL and BLOCK_CAUSAL need Nkv >= Nq

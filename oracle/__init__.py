@@ -9,6 +9,7 @@ Every array here is numpy.  bf16 tensors travel as their uint16 bit patterns.
 Layouts follow the library's logical layout [B, H, N, D]; V codes are
 token-major [N_kv, D] here (the device library stores them in its own order).
 """
+import contextlib
 import ctypes
 import math
 import os
@@ -36,63 +37,84 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        i64, i32, f64 = ctypes.c_long, ctypes.c_int, ctypes.c_double
-        L.orc_e4m3_decode.restype = f64
-        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
-        L.orc_e4m3_encode.restype = ctypes.c_uint8
-        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
-        L.orc_e4m3_encode_n.restype = None
-        L.orc_e4m3_encode_n.argtypes = [P, i64, P]
-        L.orc_quant_head.restype = i32
-        L.orc_quant_head.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P]
-        L.orc_quant_head_rope.restype = i32
-        L.orc_quant_head_rope.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P]
-        L.orc_qk_int32.restype = None
-        L.orc_qk_int32.argtypes = [P, P, i32, i64, i64, i64, i64, P]
-        L.orc_row_limit.restype = i64
-        L.orc_row_limit.argtypes = [i64, i64, i64, i32, i64]
-        L.orc_attn_rows.restype = i32
-        L.orc_attn_rows.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
-                                    P, i64, P, P, P, i32]
-        L.orc_attn_rows_identity.restype = i32
-        L.orc_attn_rows_identity.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
-                                             P, i64, P, P, i32]
-        L.orc_attn_rows_bs.restype = i32
-        L.orc_attn_rows_bs.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
-                                       P, i64, i64, P, i64, P, P, P, i32]
-        L.orc_attn_rows_identity_bs.restype = i32
-        L.orc_attn_rows_identity_bs.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
-                                                P, i64, i64, P, i64, P, P, i32]
-        L.orc_attn_rows_split.restype = i32
-        L.orc_attn_rows_split.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
-                                          i32, i64, P, i64, P, P, P, i32]
-        L.orc_attn_rows_identity_split.restype = i32
-        L.orc_attn_rows_identity_split.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64, i32, i64,
-                                                   P, i64, P, P, i32]
-        L.orc_w8a8_quant_act.restype = i32
-        L.orc_w8a8_quant_act.argtypes = [P, i64, i64, P, P]
-        L.orc_w8a8_quant_weight.restype = i32
-        L.orc_w8a8_quant_weight.argtypes = [P, i64, i64, P, P]
-        L.orc_w8a8_gemm_rows.restype = i32
-        L.orc_w8a8_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, i32]
-        L.orc_attn_fp64_rows.restype = i32
-        L.orc_attn_fp64_rows.argtypes = [P, P, P, i64, i64, i32, i32, i64, P, i64, P, i32]
-        L.orc_attn_fp64_rows_win.restype = i32
-        L.orc_attn_fp64_rows_win.argtypes = [P, P, P, i64, i64, i32, i64, i64, i64, P, i64, P,
-                                             i32]
-        L.orc_attn_rows_win.restype = i32
-        L.orc_attn_rows_win.argtypes = [P, P, P, P, P, P, i64, i64, i32, i64, i64, i64, i64, f64,
-                                        i32, i64, P, i64, P, P, P, i32]
-        L.orc_attn_rows_identity_win.restype = i32
-        L.orc_attn_rows_identity_win.argtypes = [P, P, P, i64, i64, i32, i64, i64, i64, i64, i32,
-                                                 i64, P, i64, P, P, i32]
-        L.orc_row_window_export.restype = None
-        L.orc_row_window_export.argtypes = [i64, i64, i64, i32, i64, i64, i64, P]
-        _lib = L
+        _lib = _load(_build.build())
     return _lib
+
+
+@contextlib.contextmanager
+def variant(**defines):
+    """Within the block, every function of this module runs on a separately
+    compiled copy of the oracle with the given preprocessor defines (the
+    planted mistakes and the alternative P-scale reading listed in
+    sage_oracle.c).  Test-suite only."""
+    global _lib
+    saved = lib()
+    _lib = _load(_build.build_variant(defines))
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _load(path):
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i64, i32, f64 = ctypes.c_long, ctypes.c_int, ctypes.c_double
+    L.orc_e4m3_decode.restype = f64
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    L.orc_e4m3_encode_n.restype = None
+    L.orc_e4m3_encode_n.argtypes = [P, i64, P]
+    L.orc_quant_head.restype = i32
+    L.orc_quant_head.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P]
+    L.orc_quant_head_rope.restype = i32
+    L.orc_quant_head_rope.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P]
+    L.orc_qk_int32.restype = None
+    L.orc_qk_int32.argtypes = [P, P, i32, i64, i64, i64, i64, P]
+    L.orc_row_limit.restype = i64
+    L.orc_row_limit.argtypes = [i64, i64, i64, i32, i64]
+    L.orc_attn_rows.restype = i32
+    L.orc_attn_rows.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
+                                P, i64, P, P, P, i32]
+    L.orc_attn_rows_identity.restype = i32
+    L.orc_attn_rows_identity.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
+                                         P, i64, P, P, i32]
+    L.orc_attn_rows_bs.restype = i32
+    L.orc_attn_rows_bs.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
+                                   P, i64, i64, P, i64, P, P, P, i32]
+    L.orc_attn_rows_identity_bs.restype = i32
+    L.orc_attn_rows_identity_bs.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64,
+                                            P, i64, i64, P, i64, P, P, i32]
+    L.orc_attn_rows_split.restype = i32
+    L.orc_attn_rows_split.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64,
+                                      i32, i64, P, i64, P, P, P, i32]
+    L.orc_attn_rows_identity_split.restype = i32
+    L.orc_attn_rows_identity_split.argtypes = [P, P, P, i64, i64, i32, i32, i64, i64, i32, i64,
+                                               P, i64, P, P, i32]
+    L.orc_w8a8_quant_act.restype = i32
+    L.orc_w8a8_quant_act.argtypes = [P, i64, i64, P, P]
+    L.orc_w8a8_quant_weight.restype = i32
+    L.orc_w8a8_quant_weight.argtypes = [P, i64, i64, P, P]
+    L.orc_w8a8_gemm_rows.restype = i32
+    L.orc_w8a8_gemm_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, i32]
+    L.orc_attn_fp64_rows.restype = i32
+    L.orc_attn_fp64_rows.argtypes = [P, P, P, i64, i64, i32, i32, i64, P, i64, P, i32]
+    L.orc_attn_fp64_rows_win.restype = i32
+    L.orc_attn_fp64_rows_win.argtypes = [P, P, P, i64, i64, i32, i64, i64, i64, P, i64, P,
+                                         i32]
+    L.orc_attn_rows_win.restype = i32
+    L.orc_attn_rows_win.argtypes = [P, P, P, P, P, P, i64, i64, i32, i64, i64, i64, i64, f64,
+                                    i32, i64, P, i64, P, P, P, i32]
+    L.orc_attn_rows_identity_win.restype = i32
+    L.orc_attn_rows_identity_win.argtypes = [P, P, P, i64, i64, i32, i64, i64, i64, i64, i32,
+                                             i64, P, i64, P, P, i32]
+    L.orc_row_window_export.restype = None
+    L.orc_row_window_export.argtypes = [i64, i64, i64, i32, i64, i64, i64, P]
+    L.orc_attn_rows_pert.restype = i32
+    L.orc_attn_rows_pert.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64, P,
+                                     f64, P, i64, P, P, P, i32]
+    return L
 
 
 def _p(a):
@@ -205,7 +227,8 @@ def _block_mask(block_mask, nkv, tkv):
 
 
 def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
-              threads=None, block_mask=None, kv_splits=1, window=None):
+              threads=None, block_mask=None, kv_splits=1, window=None, pert=None,
+              pert_eps=0.0):
     """Same-quantization attention of one quantized head on the given rows.
 
     block_mask: optional uint8 [ceil(Nq / 128), ceil(Nkv / tkv)] of this head;
@@ -215,6 +238,9 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
     merged (not combined with a block mask).
     window: (frame, win, sink) for the sliding-window mask with a reference
     context (``orc_attn_rows_win``; mask and mb are then ignored).
+    pert, pert_eps (test hook, dense form only): int8 [Nq, Nkv] of -1, 0, +1;
+    the exp2 result y of row i and key j becomes the fp32 value nearest to
+    y (1 + pert[i, j] pert_eps) on y's side (``orc_attn_rows_pert``).
     Returns (o [n, D] float64 of the fp32 recipe, slack [n, D] or None, lse [n]).
     """
     rows = np.ascontiguousarray(rows, np.int64)
@@ -228,7 +254,18 @@ def attn_rows(qh, rows, mask=MASK_NONE, mb=0, tkv=TKV, eps=EPS, with_slack=True,
     qs = np.ascontiguousarray(qh["qs"])
     ks = np.ascontiguousarray(qh["ks"])
     vs = np.ascontiguousarray(qh["vs"])
-    if window is not None:
+    if pert is not None:
+        if window is not None or block_mask is not None or kv_splits > 1:
+            raise ValueError("pert is supported on the dense form only")
+        pert = np.ascontiguousarray(pert, np.int8)
+        if pert.shape != (qh["nq"], qh["nkv"]):
+            raise ValueError("pert must be int8 [Nq, Nkv]")
+        rc = lib().orc_attn_rows_pert(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs),
+                                      qh["nq"], qh["nkv"], D, mask, mb, tkv, eps, _p(pert),
+                                      float(pert_eps), _p(rows), n, _p(o),
+                                      _p(slack) if slack is not None else None, _p(lse),
+                                      _threads(threads))
+    elif window is not None:
         if block_mask is not None:
             raise ValueError("window and block_mask are not combined")
         frame, win, sink = _window(window)

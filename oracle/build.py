@@ -28,5 +28,24 @@ def build(force: bool = False) -> str:
     return LIB
 
 
+def build_variant(defines, out_dir=None) -> str:
+    """Compile a separate copy of the oracle with extra preprocessor defines
+    (``{"ORC_PLANT": 2}``, ``{"ORC_PSCALE_UNFOLDED": 1}``) for the tests that
+    show which mistakes or alternative readings the pins detect.  The default
+    library is never replaced."""
+    import tempfile
+    tag = "_".join("%s%s" % (k, v) for k, v in sorted(defines.items()))
+    out_dir = out_dir or os.path.join(tempfile.gettempdir(), "sage_oracle_variants")
+    os.makedirs(out_dir, exist_ok=True)
+    path = os.path.join(out_dir, "liboracle_%s.so" % tag)
+    if os.path.exists(path) and os.path.getmtime(path) >= os.path.getmtime(SRC):
+        return path
+    tmp = path + ".tmp%d" % os.getpid()
+    flags = ["-D%s=%s" % (k, v) for k, v in sorted(defines.items())]
+    subprocess.run(["gcc", *CFLAGS, *flags, SRC, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, path)
+    return path
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv))

@@ -30,8 +30,15 @@
  *   orc_quant_head           : quantizer invariants, numpy mean for mu.
  *   orc_qk_int32             : numpy int64 brute force.
  *   orc_attn_rows (identity) : textbook softmax attention to 1e-12.
- *   orc_attn_rows (quant)    : closed forms (Q = 0, single visible key) and
- *                              the error bound against fp64 attention.
+ *   orc_attn_rows (quant)    : closed forms (Q = 0, single visible key);
+ *                              plain fp64 attention over the dequantized
+ *                              operands within the rigorous bound of P's
+ *                              e4m3 rounding, lse to 1e-5; the error bound
+ *                              against fp64 attention.
+ *   rounding slack           : exp2 results moved to the edges of their
+ *                              uncertainty interval (orc_attn_rows_pert)
+ *                              stay within it and, pushed per channel to
+ *                              the extreme codes, span it exactly.
  *   orc_attn_fp64_rows       : textbook softmax attention (torch) to 1e-12.
  *   orc_attn_rows_bs / _identity_bs (block mask): identity mode against
  *                              textbook softmax attention under the combined
@@ -443,19 +450,59 @@ typedef struct {
     /* sliding-window mask (mask == ORC_MASK_SLIDING_WINDOW): frames of mb
      * tokens, win frames per window, sink reference-context tokens */
     long win, sink;
+    /* test hook (NULL: off): pert[i * nkv + j] = +1 replaces the exp2 result
+     * y of query row i and key j by the largest fp32 value <= y (1 +
+     * pert_eps), -1 by the smallest fp32 value >= y (1 - pert_eps): the
+     * extreme results of an exp2 whose relative error is up to pert_eps, the
+     * uncertainty that the rounding slack is meant to cover */
+    const int8_t *pert;
+    double pert_eps;
 } attn_job;
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
 
-/* Width, in units of y = p*2^8, of the set of e4m3 codes that y*(1 +- eps)
- * can round to; zero when the uncertainty interval does not straddle a
- * rounding boundary. */
+/* Compile-time switches used only by the test-suite, which builds separate
+ * copies of this library with them to show that its pins catch plausible
+ * mistakes (the product build defines neither):
+ *   ORC_PLANT = 1  the K scale of key j taken from block j / 128, not j / 64
+ *             = 2  l summed from the decoded e4m3 codes instead of from y
+ *             = 3  the slack not rescaled by alpha when the running max moves
+ *             = 4  the slack gap measured in code units instead of values
+ *             = 5  the slack not divided by l
+ *   ORC_PSCALE_UNFOLDED  the other admissible reading of the 2^8 P scale:
+ *             y = 2^8 * fp32(exp2(fmaf(S, c, -m))) instead of
+ *             y = fp32(exp2(fmaf(S, c, fp32(8 - m)))) */
+#ifndef ORC_PLANT
+#define ORC_PLANT 0
+#endif
+
+/* Width, in units of y = p*2^8, of the set of e4m3 codes that an fp32 value
+ * within relative distance eps of y can round to; zero when that set is one
+ * code.  The device's y is an fp32 value, so its admissible values are the
+ * fp32 numbers in [y (1 - eps), y (1 + eps)]: the smallest of them is the
+ * lower end rounded up to fp32, the largest the upper end rounded down
+ * (y (1 +- eps) itself is exact in double for the eps used here). */
+static float f32_at_least(double a)
+{
+    float f = (float)a;
+    return (double)f < a ? nextafterf(f, INFINITY) : f;
+}
+
+static float f32_at_most(double b)
+{
+    float f = (float)b;
+    return (double)f > b ? nextafterf(f, -INFINITY) : f;
+}
+
 static double e4m3_flip_gap(double y, double eps)
 {
-    uint8_t lo = e4m3_encode_d(y * (1.0 - eps));
-    uint8_t hi = e4m3_encode_d(y * (1.0 + eps));
+    uint8_t lo = e4m3_encode_d((double)f32_at_least(y * (1.0 - eps)));
+    uint8_t hi = e4m3_encode_d((double)f32_at_most(y * (1.0 + eps)));
     if (lo == hi)
         return 0.0;
+#if ORC_PLANT == 4
+    return fabs((double)hi - (double)lo);
+#endif
     return fabs(orc_e4m3_decode(hi) - orc_e4m3_decode(lo));
 }
 
@@ -536,7 +583,11 @@ static void attend_range(const attn_job *J, long i, long se, long lo, long hi, c
                 for (int d = 0; d < D; d++)
                     s += (int64_t)J->q8[i * D + d] * (int64_t)J->k8[j * D + d];
                 S[jj] = (int32_t)s;
+#if ORC_PLANT == 1
+                c[jj] = sqC * J->ks[j / 128];
+#else
                 c[jj] = sqC * J->ks[j / ORC_BLK];
+#endif
                 t[jj] = (double)((float)S[jj] * c[jj]);
             }
         }
@@ -571,10 +622,23 @@ static void attend_range(const attn_job *J, long i, long se, long lo, long hi, c
                 for (int d = 0; d < D; d++)
                     acc[d] += p * J->vd[j * D + d];
             } else {
+#ifdef ORC_PSCALE_UNFOLDED
+                (void)nm8;
+                float y = 256.0f * exp2_f32(fmaf((float)S[jj], c[jj], -mf));
+#else
                 float x = fmaf((float)S[jj], c[jj], nm8);
                 float y = exp2_f32(x);
-                rowsum_f += y;
+#endif
+                if (J->pert && J->pert[i * J->nkv + j] > 0)
+                    y = f32_at_most((double)y * (1.0 + J->pert_eps));
+                else if (J->pert && J->pert[i * J->nkv + j] < 0)
+                    y = f32_at_least((double)y * (1.0 - J->pert_eps));
                 double w = orc_e4m3_decode(orc_e4m3_encode(y));
+#if ORC_PLANT == 2
+                rowsum_f += (float)w;
+#else
+                rowsum_f += y;
+#endif
                 double gap = sl ? e4m3_flip_gap((double)y, J->eps) : 0.0;
                 for (int d = 0; d < D; d++) {
                     double vv = orc_e4m3_decode(J->v8[j * D + d]);
@@ -586,8 +650,13 @@ static void attend_range(const attn_job *J, long i, long se, long lo, long hi, c
         }
         for (int d = 0; d < D; d++) {
             o[d] = o[d] * alpha + acc[d];
+#if ORC_PLANT == 3
+            if (sl)
+                sl[d] = sl[d] + sacc[d];
+#else
             if (sl)
                 sl[d] = sl[d] * alpha + sacc[d];
+#endif
         }
         if (J->identity)
             l = l * alpha + rowsum;
@@ -718,8 +787,13 @@ static void attend_row(const attn_job *J, long r)
         for (int d = 0; d < D; d++) {
             double f = (double)J->vs[d] / (double)lf;
             o[d] = o[d] * f;
+#if ORC_PLANT == 5
+            if (sl)
+                sl[d] = sl[d] * (double)J->vs[d];
+#else
             if (sl)
                 sl[d] = sl[d] * f;
+#endif
         }
         if (J->lse)
             J->lse[r] = ((double)mf + log2((double)lf) - 8.0) * 0.6931471805599453;
@@ -948,6 +1022,47 @@ int orc_attn_rows(const int8_t *q8, const float *qs, const int8_t *k8, const flo
 {
     return orc_attn_rows_bs(q8, qs, k8, ks, v8, vs, nq, nkv, D, mask, mb, tkv, eps, NULL, 0, 0,
                             rows, nrows, o, slack, lse, nthreads);
+}
+
+/* orc_attn_rows with the exp2 perturbation hook (test-suite only): pert is
+ * int8 [nq, nkv] of -1, 0, +1, see attn_job.pert. */
+int orc_attn_rows_pert(const int8_t *q8, const float *qs, const int8_t *k8, const float *ks,
+                       const uint8_t *v8, const float *vs, long nq, long nkv, int D,
+                       int mask, long mb, long tkv, double eps, const int8_t *pert,
+                       double pert_eps, const long *rows, long nrows, double *o, double *slack,
+                       double *lse, int nthreads)
+{
+    if (tkv <= 0 || nq <= 0 || nkv <= 0 || D <= 0 || !pert)
+        return 1;
+    if ((mask == ORC_MASK_CAUSAL || mask == ORC_MASK_BLOCK_CAUSAL) && nkv < nq)
+        return 1;
+    if (mask == ORC_MASK_BLOCK_CAUSAL && mb <= 0)
+        return 1;
+    attn_job J = {0};
+    J.nq = nq;
+    J.nkv = nkv;
+    J.D = D;
+    J.mask = mask;
+    J.mb = mb;
+    J.tkv = tkv;
+    J.eps = eps;
+    J.q8 = q8;
+    J.qs = qs;
+    J.k8 = k8;
+    J.ks = ks;
+    J.v8 = v8;
+    J.vs = vs;
+    J.rows = rows;
+    J.nrows = nrows;
+    J.o = o;
+    J.slack = slack;
+    J.lse = lse;
+    J.pert = pert;
+    J.pert_eps = pert_eps;
+    if (slack)
+        memset(slack, 0, sizeof(double) * (size_t)(nrows * D));
+    for_rows(&J, attend_row_cb, nrows, nthreads);
+    return 0;
 }
 
 int orc_attn_rows_identity(const double *q, const double *k, const double *v,
