@@ -181,11 +181,19 @@ class Runner:
         # split-KV attention where the query tiles alone would leave SMs idle
         # (e.g. one streaming frame against a long cache); 1 for the video shapes
         self.window = (w.mask_block, w.win, w.sink) if w.mask == 3 else None
+        # windowed quantization: only the keys the step attends to are
+        # quantized (sage_quant_qk_window); attention runs on those
+        self.window_quant = bool(w.extra.get("window_quant"))
+        nkv_q = w.Nkv
+        if self.window_quant:
+            n_sink, lo, hi = sage.window_keys(sage.make_shape(w.B, w.H, w.Nq, w.Nkv, w.D),
+                                              *self.window)
+            nkv_q = n_sink + hi - lo
         if kv_splits == "auto":
             sms = torch.cuda.get_device_properties(device).multi_processor_count
-            nkv = w.Nkv
+            nkv = nkv_q
             if self.window:  # keys a query tile visits, at most
-                nkv = min(w.Nkv, w.sink + (w.win + 1) * w.mask_block + 128)
+                nkv = min(nkv_q, w.sink + (w.win + 1) * w.mask_block + 128)
             kv_splits = sage.suggest_kv_splits(w.B, w.H, w.Nq, nkv, sms)
         self.kv_splits = int(kv_splits)
         wr = rank_workload(w, rank)
@@ -199,7 +207,7 @@ class Runner:
         self.q = self.h_q.to(device)
         self.k = self.h_k.to(device)
         self.v = self.h_v.to(device)
-        self.shape = sage.make_shape(w.B, w.H, w.Nq, w.Nkv, w.D)
+        self.shape = sage.make_shape(w.B, w.H, w.Nq, nkv_q, w.D)
         self.qkv = sage.QuantizedQKV(self.shape, device)
         self.ws = torch.empty(max(sage.workspace_bytes(self.shape), 16), dtype=torch.uint8,
                               device=device)
@@ -216,7 +224,11 @@ class Runner:
         q, k, v, o = bufs if bufs is not None else (self.q, self.k, self.v, self.o)
         if ev is not None:
             ev[0].record(self.stream)
-        s.quant_qk(q, k, v, out=self.qkv, workspace=self.ws, stream=self.stream)
+        if self.window_quant:
+            s.quant_qk_window(q, k, v, *self.window, out=self.qkv, workspace=self.ws,
+                              stream=self.stream)
+        else:
+            s.quant_qk(q, k, v, out=self.qkv, workspace=self.ws, stream=self.stream)
         if ev is not None:
             ev[1].record(self.stream)
         s.attn_fwd(self.qkv, self.w.mask, self.w.mask_block, out=o, stream=self.stream,
@@ -424,16 +436,32 @@ def run_ours(args):
                          "step i overlap the kernels (second stream, double-buffered tensors)"}
 
     secondary = {}
-    if not args.no_secondary and w.name != synth.P480.name:
+    if not args.no_secondary:
         del runner
         torch.cuda.empty_cache()
-        r2 = Runner(synth.P480, rank, device)
-        t2 = time_steps(r2, args.steps, args.warmup, world, per_kernel=True)
-        secondary[synth.P480.name] = {
-            "value": aggregate_value(synth.P480.ops(), world, t2["ms"]), "unit": UNIT,
-            "ms_per_step": t2["ms"], "attn_ms": t2["attn_ms"], "quant_ms": t2["quant_ms"],
-            "attn_frac_of_peak": synth.P480.ops() / (t2["attn_ms"] / 1e3) / 1e12 / pk["i8_sustained"]}
-        del r2
+        # the other workloads of the metric: the 480p video shape and the
+        # streaming frame step (block-causal, and under the sliding window),
+        # each with the launch configuration `Runner` picks (KV splits where
+        # the query tiles alone would leave SMs idle)
+        for w2 in (synth.P480, synth.STREAMING, synth.STREAMING_WINDOW, synth.STREAMING_WINDOW_Q):
+            if w2.name == w.name:
+                continue
+            r2 = Runner(w2, rank, device)
+            t2 = time_steps(r2, args.steps, args.warmup, world, per_kernel=True)
+            ops2 = w2.ops()
+            secondary[w2.name] = {
+                "value": aggregate_value(ops2, world, t2["ms"]), "unit": UNIT,
+                "ms_per_step": round(t2["ms"], 4), "attn_ms": round(t2["attn_ms"], 4),
+                "quant_ms": round(t2["quant_ms"], 4),
+                "attn_kernel": attn_kernel_label(w2, r2.kv_splits),
+                "attn_tops": round(ops2 / (t2["attn_ms"] / 1e3) / 1e12, 2),
+                "attn_frac_of_peak": round(
+                    ops2 / (t2["attn_ms"] / 1e3) / 1e12 / pk["i8_sustained"], 4),
+                "attn_frac_of_burst_peak": round(
+                    ops2 / (t2["attn_ms"] / 1e3) / 1e12 / pk["i8_burst"], 4),
+                "ops_per_step": ops2, "mask": MASK_NAMES[w2.mask]}
+            del r2
+            torch.cuda.empty_cache()
 
     value = aggregate_value(ops_rank, world, t["ms"])
     achieved = ops_rank / (t["attn_ms"] / 1e3) / 1e12
@@ -745,6 +773,15 @@ def run_ceilings(args):
                     "per_sm_per_clock": round(best["per_sm_per_clock"], 2),
                     "per_second": best["per_second"], "ms": round(best["ms"], 4)})
     clk = clocks.stop()
+    # per SM per SM clock from the event-timed rate and the sampled SM clock
+    # (the per-block clock64 spans have been seen to advance at half the SM
+    # clock in these launches, so they are reported but not relied on)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mhz = (clk or {}).get("sm_mhz")
+    for r in out:
+        r["per_sm_per_clock_clock64"] = r.pop("per_sm_per_clock")
+        r["per_sm_per_sm_clock"] = (round(r["per_second"] / (sms * mhz * 1e6), 2)
+                                    if mhz else None)
     sustained = []
     if args.ceil_seconds > 0:
         # the attention's MMA shapes held for ceil_seconds each: back-to-back

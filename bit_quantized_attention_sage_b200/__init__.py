@@ -66,6 +66,10 @@ def lib():
         L.sage_quant_qk.argtypes = [P, P, P, P, P, P, SZ, P]
         L.sage_quant_qk_rope.restype = I
         L.sage_quant_qk_rope.argtypes = [P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.sage_window_keys.restype = I
+        L.sage_window_keys.argtypes = [P, I, I, I, P, P, P]
+        L.sage_quant_qk_window.restype = I
+        L.sage_quant_qk_window.argtypes = [P, P, P, P, I, I, I, P, P, P, P, P, P, SZ, P]
         L.sage_quant_qk_noalloc.restype = I
         L.sage_quant_qk_noalloc.argtypes = [P, P, P, P, P, P]
         L.sage_attn_fwd.restype = I
@@ -199,6 +203,52 @@ def quant_qk(q, k, v, out=None, workspace=None, stream=None, rope=None):
                                         *[_ptr(t) for t in rope], ctypes.byref(qs),
                                         _ptr(workspace), workspace.numel(), _stream(stream)),
                "sage_quant_qk_rope")
+    return out
+
+
+def window_keys(shape, frame, win, sink):
+    """sage_window_keys: (n_sink, lo, hi) -- a sliding-window step over a
+    cache of `shape` attends to keys [0, n_sink) and [lo, hi)."""
+    a, b, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().sage_window_keys(ctypes.byref(shape), int(frame), int(win), int(sink),
+                                  ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "sage_window_keys")
+    return a.value, b.value, c.value
+
+
+def quant_qk_window(q, k_cache, v_cache, frame, win, sink, rope=None, out=None, workspace=None,
+                    stream=None):
+    """sage_quant_qk_window: quantize only the keys a sliding-window step
+    attends to (the reference context and the window, gathered in cache
+    order).  q [B, H, Nq, D], k_cache / v_cache [B, H, Nkv, D] bf16 CUDA;
+    rope: None or (q_cos, q_sin, k_cos, k_sin) float32 [Nq, D/2] and
+    [Nkv', D/2] (the gathered keys' positions).  Returns QuantizedQKV of the
+    gathered shape (Nkv' = n_sink + hi - lo keys)."""
+    import torch
+    B, H, Nq, D = q.shape
+    cache = make_shape(B, H, Nq, k_cache.shape[2], D)
+    for t in (q, k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k_cache, v_cache must be contiguous bf16 CUDA tensors")
+    n_sink, lo, hi = window_keys(cache, frame, win, sink)
+    shape = make_shape(B, H, Nq, n_sink + hi - lo, D)
+    if rope is not None:
+        for t, n in zip(rope, (Nq, Nq, shape.Nkv, shape.Nkv)):
+            if (t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous()
+                    or tuple(t.shape) != (n, D // 2)):
+                raise ValueError("rotation tables must be contiguous float32 CUDA tensors "
+                                 "[Nq, D/2], [Nq, D/2], [Nkv', D/2], [Nkv', D/2]")
+    if out is None:
+        out = QuantizedQKV(shape, q.device)
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(shape), 16), dtype=torch.uint8,
+                                device=q.device)
+    qs = out.struct()
+    tabs = [None] * 4 if rope is None else [_ptr(t) for t in rope]
+    _check(lib().sage_quant_qk_window(_ptr(q), _ptr(k_cache), _ptr(v_cache), ctypes.byref(cache),
+                                      int(frame), int(win), int(sink), *tabs, ctypes.byref(qs),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sage_quant_qk_window")
     return out
 
 

@@ -30,11 +30,11 @@ constexpr long long kWaitBudget = 1ll << 31;  // ~1 s of SM clock per wait
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
-  std::once_flag once;
-  cudaError_t init_err = cudaSuccess;
+  bool ready = false;     // set-up succeeded on this device
   int* status = nullptr;  // device address of g_status
 };
 DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -56,20 +56,24 @@ EncodeTiledFn encode_fn() {
 }
 
 // Per-device one-time setup: the status word's device address and the
-// attention kernels' shared-memory attribute.
+// kernels' shared-memory attributes.  Only a complete, successful set-up is
+// kept; after a failure (which may be an unrelated error left by an earlier
+// launch) the next call tries again.
 DeviceState* device_state() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   DeviceState& d = g_dev[dev];
-  std::call_once(d.once, [&d] {
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (!d.ready) {
     void* p = nullptr;
-    d.init_err = cudaGetSymbolAddress(&p, g_status);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_status);
+    if (e == cudaSuccess) e = attn_prepare(128);
+    if (e == cudaSuccess) e = attn_prepare(64);
+    if (e == cudaSuccess) e = w8a8_prepare();
+    if (e != cudaSuccess) return nullptr;
     d.status = static_cast<int*>(p);
-    if (d.init_err == cudaSuccess) d.init_err = attn_prepare(128);
-    if (d.init_err == cudaSuccess) d.init_err = attn_prepare(64);
-    if (d.init_err == cudaSuccess) d.init_err = w8a8_prepare();
-  });
-  if (d.init_err != cudaSuccess) return nullptr;
+    d.ready = true;
+  }
   return &d;
 }
 
@@ -306,10 +310,35 @@ SAGE_EXPORT size_t sage_quant_workspace_bytes(const sage_shape* shape) {
 }
 
 namespace {
+// The keys a sliding-window step over a cache of `shape` attends to (the
+// union over its query rows): [0, *n_sink) and [*lo, *hi), *lo >= *n_sink.
+// The same row windows as the attention kernel's (queries are the newest Nq
+// of the Nkv tokens).
+void window_key_ranges(const sage_shape* s, int frame, int win, int sink, int* n_sink, int* lo,
+                       int* hi) {
+  const long long off = static_cast<long long>(s->Nkv) - s->Nq;
+  const long long se = std::min<long long>(sink, s->Nkv);
+  auto row = [&](long long g, long long* l, long long* h) {
+    if (g < se) {
+      *l = *h = se;
+      return;
+    }
+    const long long f = (g - se) / frame;
+    *l = se + std::max<long long>(f - win + 1, 0) * frame;
+    *h = std::min<long long>(se + (f + 1) * frame, s->Nkv);
+  };
+  long long l0, h0, l1, h1;
+  row(off, &l0, &h0);
+  row(off + s->Nq - 1, &l1, &h1);
+  *n_sink = static_cast<int>(se);
+  *lo = static_cast<int>(std::max(l0, se));
+  *hi = static_cast<int>(std::max(h1, std::max(l0, se)));
+}
+
 sage_status quant_common(const void* q_bf16, const void* k_bf16, const void* v_bf16,
                          const sage_shape* shape, const float* const rope[4],
                          const sage_qkv_quant* out, void* workspace, size_t ws_bytes,
-                         void* stream) {
+                         void* stream, int nkv_src = -1, int kv_split = -1, int kv_gap = 0) {
   if (!shape_ok(shape) || !qkv_ok(out)) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(workspace))
     return SAGE_ERR_INVALID_ARG;
@@ -337,6 +366,9 @@ sage_status quant_common(const void* q_bf16, const void* k_bf16, const void* v_b
   a.ws_ksum = static_cast<double*>(workspace);
   a.ws_vmax = reinterpret_cast<float*>(static_cast<char*>(workspace) + cells * 8);
   a.ws_vinv = reinterpret_cast<float*>(static_cast<char*>(workspace) + cells * 12);
+  a.Nkv_src = nkv_src < 0 ? a.Nkv : nkv_src;
+  a.kv_split = kv_split < 0 ? a.Nkv : kv_split;
+  a.kv_gap = kv_gap;
   if (rope) {
     a.q_cos = rope[0];
     a.q_sin = rope[1];
@@ -352,6 +384,36 @@ SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, co
                                       const sage_shape* shape, const sage_qkv_quant* out,
                                       void* workspace, size_t ws_bytes, void* stream) {
   return quant_common(q_bf16, k_bf16, v_bf16, shape, nullptr, out, workspace, ws_bytes, stream);
+}
+
+SAGE_EXPORT sage_status sage_window_keys(const sage_shape* shape, int frame, int win, int sink,
+                                         int* n_sink, int* lo, int* hi) {
+  if (!shape_ok(shape) || !n_sink || !lo || !hi || frame < 1 || win < 1 || sink < 0 ||
+      shape->Nkv < shape->Nq)
+    return SAGE_ERR_INVALID_ARG;
+  window_key_ranges(shape, frame, win, sink, n_sink, lo, hi);
+  return SAGE_OK;
+}
+
+SAGE_EXPORT sage_status sage_quant_qk_window(const void* q_bf16, const void* k_cache,
+                                             const void* v_cache, const sage_shape* cache_shape,
+                                             int frame, int win, int sink, const float* q_cos,
+                                             const float* q_sin, const float* k_cos,
+                                             const float* k_sin, const sage_qkv_quant* out,
+                                             void* workspace, size_t ws_bytes, void* stream) {
+  if (!shape_ok(cache_shape) || frame < 1 || win < 1 || sink < 0 ||
+      cache_shape->Nkv < cache_shape->Nq)
+    return SAGE_ERR_INVALID_ARG;
+  const int nrope = (q_cos != nullptr) + (q_sin != nullptr) + (k_cos != nullptr) + (k_sin != nullptr);
+  if (nrope != 0 && nrope != 4) return SAGE_ERR_INVALID_ARG;
+  int n_sink = 0, lo = 0, hi = 0;
+  window_key_ranges(cache_shape, frame, win, sink, &n_sink, &lo, &hi);
+  sage_shape g = *cache_shape;
+  g.Nkv = n_sink + (hi - lo);
+  if (g.Nkv < g.Nq) return SAGE_ERR_INVALID_ARG;
+  const float* rope[4] = {q_cos, q_sin, k_cos, k_sin};
+  return quant_common(q_bf16, k_cache, v_cache, &g, nrope ? rope : nullptr, out, workspace,
+                      ws_bytes, stream, cache_shape->Nkv, n_sink, lo - n_sink);
 }
 
 SAGE_EXPORT sage_status sage_quant_qk_rope(const void* q_bf16, const void* k_bf16,

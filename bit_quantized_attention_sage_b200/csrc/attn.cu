@@ -57,6 +57,12 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kBiasBits = 0x4B400000u;
 constexpr float kBias = 12582912.0f;
 constexpr uint32_t kNegInfBits = 0xFF800000u;
+// KV-tile columns >= kPolyFrom take the software exp2 (exp2_poly2), the rest
+// the exp2 unit
+#ifndef SAGE_POLY_FROM
+#define SAGE_POLY_FROM 128
+#endif
+constexpr int kPolyFrom = SAGE_POLY_FROM;
 
 // wait-site codes for the status word (kernel 1 = attention)
 enum : int {
@@ -430,14 +436,17 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
           const float2 sf = __fadd2_rn(make_float2(__uint_as_float(sv[j + e]), __uint_as_float(sv[j + e + 1])), nb2);
-          const float2 x = __ffma2_rn(sf, cc, nm2);
+          float2 x = __ffma2_rn(sf, cc, nm2);
+          if (c * 16 >= kPolyFrom) x = exp2_poly2(x);  // columns of the software exp2
           y[e] = x.x; y[e + 1] = x.y;
         }
+        if (c * 16 < kPolyFrom) {
 #pragma unroll
-        for (int e = 0; e < 4; e++) y[e] = ex2_approx(y[e]);
+          for (int e = 0; e < 4; e++) y[e] = ex2_approx(y[e]);
+        }
         acc[q4 & 1] = __fadd2_rn(acc[q4 & 1], make_float2(y[0], y[1]));
         acc[q4 & 1] = __fadd2_rn(acc[q4 & 1], make_float2(y[2], y[3]));
-        pk[q4] = __byte_perm(cvt_e4m3x2(y[0], y[1]), cvt_e4m3x2(y[2], y[3]), 0x5410);
+        pk[q4] = cvt_e4m3x4(y[0], y[1], y[2], y[3]);
       }
       *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
@@ -742,6 +751,7 @@ __global__ void __launch_bounds__(128) k_attn_merge(const AttnParams p) {
     p.lse[static_cast<size_t>(bh) * p.Nq + r] =
         seen ? (m + log2f(l) - 8.0f) * 0.69314718055994531f : -INFINITY;
 }
+
 
 }  // namespace
 

@@ -46,25 +46,23 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kSageNoallocScr
 
 constexpr int kMaxDevices = 64;
 
-struct ScratchState {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
-  unsigned char* ptr = nullptr;  // device address of g_noalloc_scratch
-};
-ScratchState g_scratch[kMaxDevices];
+// Device address of g_noalloc_scratch per device, once looked up.
+std::mutex g_scratch_mu;
+unsigned char* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch on the current device (set up once per
-// device); nullptr if the lookup failed.
+// Device address of the scratch on the current device; nullptr if the lookup
+// failed.  Only a successful lookup is kept: a failure (which may be an
+// unrelated error left by an earlier launch) is retried on the next call.
 unsigned char* scratch_address() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  ScratchState& s = g_scratch[dev];
-  std::call_once(s.once, [&s] {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    s.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (s.err == cudaSuccess) s.ptr = static_cast<unsigned char*>(p);
-  });
-  return s.err == cudaSuccess ? s.ptr : nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess)
+      g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  return g_scratch_ptr[dev];
 }
 
 inline bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -108,6 +106,9 @@ SAGE_EXPORT sage_status sage_quant_qk_noalloc(const void* q_bf16, const void* k_
   a.ws_ksum = reinterpret_cast<double*>(ws);
   a.ws_vmax = reinterpret_cast<float*>(ws + cells * 8);
   a.ws_vinv = reinterpret_cast<float*>(ws + cells * 12);
+  a.Nkv_src = a.Nkv;
+  a.kv_split = a.Nkv;
+  a.kv_gap = 0;
   return launch_quant(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SAGE_OK
                                                                            : SAGE_ERR_CUDA;
 }

@@ -95,10 +95,39 @@ __device__ __forceinline__ void rope_apply(float (&x)[8], const float4& c, const
   rot_pair(x[6], x[7], c.w, s.w);
 }
 
+// The 16-byte chunk `chunk` (row-major over the block's D / 8 chunks per row)
+// of K / V block `blk` of head `bh`, through the gather map.
+template <int D>
+__device__ __forceinline__ const uint4* kv_chunk(const uint16_t* src, const QuantArgs& a, int bh,
+                                                 int blk, int chunk) {
+  constexpr int kChunksPerRow = D / 8;
+  const int row = blk * kBlk + chunk / kChunksPerRow;
+  const int srow = row < a.kv_split ? row : row + a.kv_gap;
+  return reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * a.Nkv_src + srow) * D) +
+         chunk % kChunksPerRow;
+}
+
+// The INT8 code clamp(rne(x * inv), -127, 127) of one value, as the low byte
+// of the returned word.  With |x| <= a (the block absmax) and inv =
+// fp32(127 / a), |fp32(x * inv)| <= 127 (1 + 2^-24)^2 < 127.5, so the clamp
+// never acts and rne(y) is taken by adding 1.5 * 2^23: for |y| < 2^22 the
+// fp32 sum rounds y to the nearest integer, ties to even (the ulp there is
+// 1 and 1.5 * 2^23 is even), and its low byte is the two's-complement code.
+__device__ __forceinline__ uint32_t q_i8_word(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
+}
+
+// clamp(rne(x * inv), -127, 127) by the conversion unit: used when inv is
+// infinite (a block absmax below 127 / FLT_MAX), where the sum above is not.
 __device__ __forceinline__ int8_t q_i8(float x, float inv) {
   int q = __float2int_rn(__fmul_rn(x, inv));
   q = q > 127 ? 127 : (q < -127 ? -127 : q);
   return static_cast<int8_t>(q);
+}
+
+// Low bytes of four words -> one packed word (first word in the low byte).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  return __byte_perm(__byte_perm(w0, w1, 0x0040u), __byte_perm(w2, w3, 0x0040u), 0x5410u);
 }
 
 // Quantize the 64 x D block held as `ch` 16-byte chunks per thread (x[c][8],
@@ -128,10 +157,18 @@ __device__ __forceinline__ void quant_block_store(float (&x)[CH][8], int valid, 
     const int col = (chunk % kChunksPerRow) * 8;
     uint32_t lo = 0, hi = 0;
     if (row < valid && a != 0.0f) {
+      if (inv != INFINITY) {
+        uint32_t w[8];
 #pragma unroll
-      for (int e = 0; e < 4; e++) {
-        lo |= (static_cast<uint32_t>(static_cast<uint8_t>(q_i8(x[c][e], inv)))) << (8 * e);
-        hi |= (static_cast<uint32_t>(static_cast<uint8_t>(q_i8(x[c][e + 4], inv)))) << (8 * e);
+        for (int e = 0; e < 8; e++) w[e] = q_i8_word(x[c][e], inv);
+        lo = pack_low_bytes(w[0], w[1], w[2], w[3]);
+        hi = pack_low_bytes(w[4], w[5], w[6], w[7]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          lo |= static_cast<uint32_t>(static_cast<uint8_t>(q_i8(x[c][e], inv))) << (8 * e);
+          hi |= static_cast<uint32_t>(static_cast<uint8_t>(q_i8(x[c][e + 4], inv))) << (8 * e);
+        }
       }
     }
     *reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * D + col) = make_uint2(lo, hi);
@@ -188,9 +225,6 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
 
   if (blk < nkb && ROPE) {  // V block maxima, then sums of the rotated K block
     const int valid = min(kBlk, a.Nkv - blk * kBlk);
-    const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
-    const uint4* ksrc = reinterpret_cast<const uint4*>(a.k + base);
-    const uint4* vsrc = reinterpret_cast<const uint4*>(a.v + base);
     const size_t ws = (static_cast<size_t>(bh) * nkb + blk) * D;
     const int t = threadIdx.x;
     // every load of the block first: K chunks and their angles (kept in
@@ -202,14 +236,15 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
       const int chunk = c * kThreads + threadIdx.x;
       const int row = chunk / kChunksPerRow;
       if (row < valid) {
-        ku[c] = __ldg(ksrc + chunk);
+        ku[c] = __ldg(kv_chunk<D>(a.k, a, bh, blk, chunk));
         rope_load<D>(a.k_cos, a.k_sin, blk * kBlk + row, (chunk % kChunksPerRow) * 8, kc[c], ksn[c]);
       }
     }
 #pragma unroll
     for (int c = 0; c < CH; c++) {
       const int chunk = c * kThreads + threadIdx.x;
-      if (chunk / kChunksPerRow < valid) reinterpret_cast<uint4*>(ks)[chunk] = __ldg(vsrc + chunk);
+      if (chunk / kChunksPerRow < valid)
+        reinterpret_cast<uint4*>(ks)[chunk] = __ldg(kv_chunk<D>(a.v, a, bh, blk, chunk));
     }
     __syncthreads();
     if (t >= D && t < 2 * D) {  // max |V| of channel t - D
@@ -241,16 +276,13 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
     }
   } else if (blk < nkb) {  // K block sums and V block maxima
     const int valid = min(kBlk, a.Nkv - blk * kBlk);
-    const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
-    const uint4* ksrc = reinterpret_cast<const uint4*>(a.k + base);
-    const uint4* vsrc = reinterpret_cast<const uint4*>(a.v + base);
 #pragma unroll
     for (int c = 0; c < CH; c++) {
       const int chunk = c * kThreads + threadIdx.x;
       const int row = chunk / kChunksPerRow;
       if (row < valid) {
-        reinterpret_cast<uint4*>(ks)[chunk] = __ldg(ksrc + chunk);
-        reinterpret_cast<uint4*>(vsm)[chunk] = __ldg(vsrc + chunk);
+        reinterpret_cast<uint4*>(ks)[chunk] = __ldg(kv_chunk<D>(a.k, a, bh, blk, chunk));
+        reinterpret_cast<uint4*>(vsm)[chunk] = __ldg(kv_chunk<D>(a.v, a, bh, blk, chunk));
       }
     }
     __syncthreads();
@@ -325,23 +357,18 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
   const int nkv_pad = nkb * kBlk;
   const int valid = min(kBlk, a.Nkv - blk * kBlk);
-  const size_t base = (static_cast<size_t>(bh) * a.Nkv + static_cast<size_t>(blk) * kBlk) * D;
-
   // The V loads are issued first, together with the K loads, so that the
   // whole 64-token block of K and V is in flight at once.  Chunk c*256 + t
   // (8 channels of one token) belongs to thread t, as for K.
   uint4 vu[CH];
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.v + base);
 #pragma unroll
-    for (int c = 0; c < CH; c++) {
-      const int chunk = c * kThreads + threadIdx.x;
-      vu[c] = chunk / kChunksPerRow < valid ? __ldg(src + chunk) : make_uint4(0, 0, 0, 0);
-    }
+  for (int c = 0; c < CH; c++) {
+    const int chunk = c * kThreads + threadIdx.x;
+    vu[c] = chunk / kChunksPerRow < valid ? __ldg(kv_chunk<D>(a.v, a, bh, blk, chunk))
+                                          : make_uint4(0, 0, 0, 0);
   }
 
   {  // K - mean, block codes and scale
-    const uint4* src = reinterpret_cast<const uint4*>(a.k + base);
     const float* mu = a.k_mean + static_cast<size_t>(bh) * D;
     float x[CH][8];
     uint4 u[CH];
@@ -351,7 +378,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
       const int chunk = c * kThreads + threadIdx.x;
       const int row = chunk / kChunksPerRow;
       u[c] = make_uint4(0, 0, 0, 0);
-      if (row < valid) u[c] = __ldg(src + chunk);
+      if (row < valid) u[c] = __ldg(kv_chunk<D>(a.k, a, bh, blk, chunk));
       if constexpr (ROPE) {
         rc[c] = rs[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (row < valid)
@@ -401,6 +428,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
     }
   }
 }
+
 
 }  // namespace
 

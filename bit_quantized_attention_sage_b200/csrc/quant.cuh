@@ -28,6 +28,10 @@ struct QuantArgs {
   const float* q_sin;
   const float* k_cos;
   const float* k_sin;
+  // K / V rows: gathered row r (r < Nkv) is input row r if r < kv_split,
+  // else r + kv_gap, of Nkv_src rows per head (no gather: Nkv_src = Nkv,
+  // kv_split = Nkv, kv_gap = 0)
+  int Nkv_src, kv_split, kv_gap;
 };
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream);

@@ -465,6 +465,52 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// The recipe's software exp2 of two arguments, evaluated on the fma pipes
+// (the exp2 unit gives 16 results per clock per SM, half of what the 8-bit
+// tensor core consumes at D = 128, so a share of the exponentials is taken
+// off it).  Cody-Waite style reduction x = j + f with j = round-half-even(x)
+// (adding and subtracting 1.5 * 2^23) and |f| <= 1/2; a degree-3 polynomial
+// for 2^f whose coefficients were fitted for this library (minimax relative
+// error on [-1/2, 1/2], 2^-13.7 including the fp32 Horner evaluation); 2^j
+// added to the exponent field of the polynomial's bits.  x is first raised to
+// -125 so that the exponent stays normal (a masked key's -inf gives
+// 2^-125 p(0), whose e4m3 code is 0).  Every step is one fp32 operation
+// rounded to nearest-even or an integer add, so a CPU evaluation of the same
+// steps gives the same bits.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const float2 nmagic = make_float2(-12582912.0f, -12582912.0f);
+  const float2 neg1 = make_float2(-1.0f, -1.0f);
+  const float2 c0 = make_float2(__uint_as_float(0x3f7ffb49u), __uint_as_float(0x3f7ffb49u));
+  const float2 c1 = make_float2(__uint_as_float(0x3f31798du), __uint_as_float(0x3f31798du));
+  const float2 c2 = make_float2(__uint_as_float(0x3e786f0du), __uint_as_float(0x3e786f0du));
+  const float2 c3 = make_float2(__uint_as_float(0x3d61fbb0u), __uint_as_float(0x3d61fbb0u));
+  const float2 xc = make_float2(fmaxf(x.x, -125.0f), fmaxf(x.y, -125.0f));
+  const float2 t = __fadd2_rn(xc, magic);     // magic + j
+  const float2 jf = __fadd2_rn(t, nmagic);    // j
+  const float2 f = __ffma2_rn(jf, neg1, xc);  // xc - j, exact
+  float2 p = __ffma2_rn(c3, f, c2);
+  p = __ffma2_rn(p, f, c1);
+  p = __ffma2_rn(p, f, c0);
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Four fp32 values to four e4m3 codes packed in one word, a in bits 0-7, b in
+// 8-15, c in 16-23, d in 24-31 (round to nearest even, saturating to +-448):
+// two pair conversions whose 16-bit results are joined in the same
+// statement, so no separate byte permute is needed.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
 // Two fp32 values to two e4m3 codes (round to nearest even, saturating to
 // +-448): `lo` lands in bits 0-7, `hi` in bits 8-15.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {

@@ -121,6 +121,12 @@ STREAMING = Workload("streaming_b1h24_nq2040_nkv26520_d128_blockcausal2040", 1, 
 STREAMING_WINDOW = Workload("streaming_window_b1h24_nq2040_nkv26520_d128_frame2040_win4_sink2040",
                             1, 24, 2040, 26520, 128, mask=3, mask_block=2040, k_offset_var=4.0,
                             seed=1005, win=4, sink=2040)
+# the same step with the windowed quantization of the cache: only the
+# reference context and the window (10200 of the 26520 keys) are quantized
+STREAMING_WINDOW_Q = Workload(
+    "streaming_window_winquant_b1h24_nq2040_nkv26520_d128_frame2040_win4_sink2040",
+    1, 24, 2040, 26520, 128, mask=3, mask_block=2040, k_offset_var=4.0, seed=1005, win=4,
+    sink=2040, extra={"window_quant": True})
 P480 = Workload("video480p_b1h12_n32760_d128", 1, 12, 32760, 32760, 128, outlier_mag=20.0,
                 seed=1003)
 P720 = Workload("video720p_b1h40_n75600_d128", 1, 40, 75600, 75600, 128, outlier_mag=20.0,
@@ -143,4 +149,5 @@ def sweep():
     return pts
 
 
-WORKLOADS = {w.name: w for w in (TINY, STREAMING, STREAMING_WINDOW, P480, P720)}
+WORKLOADS = {w.name: w for w in (TINY, STREAMING, STREAMING_WINDOW, STREAMING_WINDOW_Q,
+                                  P480, P720)}

@@ -110,7 +110,8 @@ sage_status sage_quant_buffer_bytes(const sage_shape *shape, size_t sizes[7]);
 
 /* Device workspace sage_quant_qk needs for `shape` (bytes; 0 on an invalid
  * shape).  It holds per-64-token-block fp64 K channel sums and V channel
- * maxima: B*H*ceil(Nkv/64)*D*12 + B*H*D*4 bytes. */
+ * maxima, and the V inverse scales: B*H*ceil(Nkv/64)*D*12 + B*H*D*4 bytes.
+ * Its contents never need initialising. */
 size_t sage_quant_workspace_bytes(const sage_shape *shape);
 
 /* Quantize Q, K and V (all device, bf16, contiguous [B,H,N,D]).
@@ -138,7 +139,9 @@ size_t sage_quant_workspace_bytes(const sage_shape *shape);
  * `out` points to caller-allocated buffers sized by sage_quant_buffer_bytes;
  * `workspace` to at least sage_quant_workspace_bytes(shape) device bytes
  * (contents need not be initialised; they are overwritten).
- * Enqueues three kernels on `stream`.  Returns SAGE_OK or an error (above). */
+ * Enqueues three kernels on `stream`: the statistics of every 64-token
+ * block (and the Q codes), the per-head K mean and V scales, then the K and
+ * V codes.  Returns SAGE_OK or an error (above). */
 sage_status sage_quant_qk(const void *q_bf16, const void *k_bf16, const void *v_bf16,
                           const sage_shape *shape, const sage_qkv_quant *out,
                           void *workspace, size_t workspace_bytes, void *stream);
@@ -173,6 +176,47 @@ sage_status sage_quant_qk_rope(const void *q_bf16, const void *k_bf16, const voi
                                const float *q_sin, const float *k_cos, const float *k_sin,
                                const sage_qkv_quant *out, void *workspace,
                                size_t workspace_bytes, void *stream);
+
+/* The keys a sliding-window step attends to (the union over its query rows
+ * of the keys sage_attn_fwd_window lets them see): the reference context
+ * [0, *n_sink) and the window [*lo, *hi) of the cache of `shape` (queries are
+ * its newest Nq tokens).  *lo - *n_sink is a whole number of frames.
+ * Errors: SAGE_ERR_INVALID_ARG for a bad shape, a null output, frame or win
+ * below 1, sink below 0, or Nkv < Nq. */
+sage_status sage_window_keys(const sage_shape *shape, int frame, int win, int sink, int *n_sink,
+                             int *lo, int *hi);
+
+/* Windowed quantization of the streaming cache: sage_quant_qk (or, with the
+ * four angle tables, sage_quant_qk_rope) over only the keys a sliding-window
+ * step attends to.
+ *
+ * The pages' streaming decoder attends, at every step, to the persistent
+ * reference context and a fixed-length window of the cache ("Vidu S1"
+ * digest, section "Infra", sliding-window decoding paragraph), and keeps the
+ * cache before RoPE, re-applying RoPE at the current positions (RoPE
+ * Repositioning bullet).  Reading: the step's K mean and V channel scales are
+ * those of the keys it attends to, and only those keys are quantized.
+ *
+ *   q_bf16                 device bf16 [B, H, Nq, D]: the step's queries
+ *   k_cache, v_cache       device bf16 [B, H, Nkv, D]: the whole cache
+ *   cache_shape            B, H, Nq, Nkv (the cache's length), D
+ *   frame, win, sink       the window of sage_attn_fwd_window
+ *   q_cos ... k_sin        NULL (no rotation) or all four tables of
+ *                          sage_quant_qk_rope: q_* [Nq, D/2], k_* [Nkv', D/2]
+ *                          for the gathered keys' current positions
+ *   out, workspace         sized for the gathered shape (B, H, Nq, Nkv', D),
+ *                          Nkv' = n_sink + hi - lo of sage_window_keys
+ * Key r of the result is cache key r for r < n_sink and cache key
+ * r + (lo - n_sink) after, i.e. the reference context then the window, in
+ * cache order.  sage_attn_fwd_window with the same (frame, win, sink) on the
+ * result gives every query row the same keys as on the whole cache.
+ * Errors: as sage_quant_qk / sage_quant_qk_rope on the gathered shape, plus
+ * SAGE_ERR_INVALID_ARG for bad window parameters or only some angle tables. */
+sage_status sage_quant_qk_window(const void *q_bf16, const void *k_cache, const void *v_cache,
+                                 const sage_shape *cache_shape, int frame, int win, int sink,
+                                 const float *q_cos, const float *q_sin, const float *k_cos,
+                                 const float *k_sin, const sage_qkv_quant *out, void *workspace,
+                                 size_t workspace_bytes, void *stream);
 
 /* Size of the fixed device scratch array sage_quant_qk_noalloc uses: 16 MiB
  * on every GPU that loads the library, held until the process exits. */

@@ -68,6 +68,8 @@ def _load(path):
     L.orc_e4m3_encode_n.argtypes = [P, i64, P]
     L.orc_quant_head.restype = i32
     L.orc_quant_head.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P]
+    L.orc_quant_head_eq.restype = i32
+    L.orc_quant_head_eq.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P, P]
     L.orc_quant_head_rope.restype = i32
     L.orc_quant_head_rope.argtypes = [P, P, P, i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P]
     L.orc_qk_int32.restype = None
@@ -111,10 +113,44 @@ def _load(path):
                                              i64, P, i64, P, P, i32]
     L.orc_row_window_export.restype = None
     L.orc_row_window_export.argtypes = [i64, i64, i64, i32, i64, i64, i64, P]
+    L.orc_exp2_poly.restype = ctypes.c_float
+    L.orc_exp2_poly.argtypes = [ctypes.c_float]
+    L.orc_exp2_poly_n.restype = None
+    L.orc_exp2_poly_n.argtypes = [P, i64, P]
+    L.orc_set_exp2_poly_from.restype = None
+    L.orc_set_exp2_poly_from.argtypes = [i32]
+    L.orc_get_exp2_poly_from.restype = i32
+    L.orc_get_exp2_poly_from.argtypes = []
     L.orc_attn_rows_pert.restype = i32
     L.orc_attn_rows_pert.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, f64, P,
                                      f64, P, i64, P, P, P, i32]
     return L
+
+
+def exp2_poly(x):
+    """The recipe's software exp2 (``orc_exp2_poly``), elementwise on fp32."""
+    x = np.ascontiguousarray(x, np.float32)
+    y = np.empty_like(x)
+    lib().orc_exp2_poly_n(_p(x), x.size, _p(y))
+    return y
+
+
+def exp2_poly_from():
+    """The first KV-tile column whose exponentials use the software exp2."""
+    return int(lib().orc_get_exp2_poly_from())
+
+
+@contextlib.contextmanager
+def exp2_poly_columns(first):
+    """Within the block the oracle evaluates the exponentials of tile columns
+    >= `first` with the software exp2 (tkv or more: none); afterwards the
+    recipe's own value is restored.  Test-suite only."""
+    saved = exp2_poly_from()
+    lib().orc_set_exp2_poly_from(int(first))
+    try:
+        yield
+    finally:
+        lib().orc_set_exp2_poly_from(saved)
 
 
 def _p(a):
@@ -142,15 +178,19 @@ def e4m3_decode(codes):
 
 # ---------------------------------------------------------------- quantization
 
-def quant_head(q, k, v, rope=None):
+def quant_head(q, k, v, rope=None, eq=False):
     """Quantize one head.  q [nq, D], k/v [nkv, D] as uint16 bf16 bits.
 
     rope: None, or (q_cos, q_sin, k_cos, k_sin), float32 [nq, D/2] and
     [nkv, D/2]: Q and K are first rotated pairwise by those angles
     (``orc_quant_head_rope``).
+    eq: the channel-equalised variant (``orc_quant_head_eq``; no rotation):
+    channel d of Q is multiplied and channel d of the smoothed K divided by
+    2^eq_exp[d] before the block quantization.
 
     Returns a dict: q8 [nq_pad, D] int8, qs [nq_blk] f32, k8 [nkv_pad, D] int8,
-    ks [nkv_blk] f32, mu [D] f32, v8 [nkv, D] uint8 e4m3 codes, vs [D] f32.
+    ks [nkv_blk] f32, mu [D] f32, v8 [nkv, D] uint8 e4m3 codes, vs [D] f32
+    (and eq_exp [D] int8 with eq).
     """
     q = np.ascontiguousarray(q, np.uint16)
     k = np.ascontiguousarray(k, np.uint16)
@@ -163,7 +203,12 @@ def quant_head(q, k, v, rope=None):
                mu=np.empty(D, np.float32), v8=np.empty((nkv, D), np.uint8),
                vs=np.empty(D, np.float32))
     outs = [_p(out[key]) for key in ("q8", "qs", "k8", "ks", "mu", "v8", "vs")]
-    if rope is None:
+    if eq:
+        if rope is not None:
+            raise ValueError("the equalised variant takes no rotation")
+        out["eq_exp"] = np.empty(D, np.int8)
+        rc = lib().orc_quant_head_eq(_p(q), _p(k), _p(v), nq, nkv, D, *outs, _p(out["eq_exp"]))
+    elif rope is None:
         rc = lib().orc_quant_head(_p(q), _p(k), _p(v), nq, nkv, D, *outs)
     else:
         tabs = [np.ascontiguousarray(t, np.float32) for t in rope]
@@ -178,13 +223,13 @@ def quant_head(q, k, v, rope=None):
     return out
 
 
-def quant(q, k, v, rope=None):
+def quant(q, k, v, rope=None, eq=False):
     """Quantize [B, H, N, D] bf16-bit tensors head by head; returns stacked arrays.
-    rope: as for quant_head (the same tables for every batch entry and head)."""
+    rope, eq: as for quant_head (the same tables for every batch entry and head)."""
     B, H = q.shape[:2]
-    heads = [quant_head(q[b, h], k[b, h], v[b, h], rope) for b in range(B) for h in range(H)]
+    heads = [quant_head(q[b, h], k[b, h], v[b, h], rope, eq) for b in range(B) for h in range(H)]
     out = {}
-    for key in ("q8", "qs", "k8", "ks", "mu", "v8", "vs"):
+    for key in ("q8", "qs", "k8", "ks", "mu", "v8", "vs") + (("eq_exp",) if eq else ()):
         a = np.stack([hd[key] for hd in heads])
         out[key] = a.reshape((B, H) + a.shape[1:])
     return out
@@ -207,6 +252,23 @@ def row_window(i, nq, nkv, mask, mb, win=0, sink=0):
     out = np.empty(3, np.int64)
     lib().orc_row_window_export(i, nq, nkv, mask, mb, win, sink, _p(out))
     return tuple(int(x) for x in out)
+
+
+def window_keys(nq, nkv, frame, win, sink):
+    """The keys a sliding-window step attends to: the union over its nq query
+    rows (the newest nq of nkv cache tokens) of the visible keys, as indices
+    into the cache, ascending: the reference context [0, min(sink, nkv)) and
+    the window [lo(first row), hi(last row)).  Quantizing only these keys
+    (gathered in this order) is the windowed reading of the streaming cache;
+    the window attention over the gathered keys, with the same (frame, win,
+    sink), gives every query row the same visible keys (the gap removed
+    between the reference context and the window is a whole number of
+    frames)."""
+    se0, lo0, _ = row_window(0, nq, nkv, MASK_SLIDING_WINDOW, frame, win, sink)
+    se1, _, hi1 = row_window(nq - 1, nq, nkv, MASK_SLIDING_WINDOW, frame, win, sink)
+    se = min(int(sink), int(nkv))
+    lo = max(int(lo0), se)
+    return np.concatenate([np.arange(se), np.arange(lo, int(hi1))]).astype(np.int64)
 
 
 def _window(window):

@@ -28,6 +28,11 @@
  *   orc_e4m3_encode / decode : OCP OFP8 E4M3 special points + brute-force
  *                              nearest-even search + torch float8 cast.
  *   orc_quant_head           : quantizer invariants, numpy mean for mu.
+ *   orc_quant_head_eq        : the exponent rule restated with numpy frexp;
+ *                              dequantized scores within the INT8 bound of
+ *                              Q (K - mu)^T; balanced channels reproduce
+ *                              orc_quant_head bit for bit; accuracy against
+ *                              fp64 attention on outlier channels.
  *   orc_qk_int32             : numpy int64 brute force.
  *   orc_attn_rows (identity) : textbook softmax attention to 1e-12.
  *   orc_attn_rows (quant)    : closed forms (Q = 0, single visible key);
@@ -66,6 +71,23 @@
 #include <string.h>
 
 #define ORC_BLK 64 /* Q/K quantization block: 64 tokens */
+
+/* Compile-time switches used only by the test-suite, which builds separate
+ * copies of this library with them to show that its pins catch plausible
+ * mistakes (the product build defines neither):
+ *   ORC_PLANT = 1  the K scale of key j taken from block j / 128, not j / 64
+ *             = 2  l summed from the decoded e4m3 codes instead of from y
+ *             = 3  the slack not rescaled by alpha when the running max moves
+ *             = 4  the slack gap measured in code units instead of values
+ *             = 5  the slack not divided by l
+ *             = 6  equalisation: the smoothed K multiplied by 2^e, not divided
+ *             = 7  equalisation: e = ilogb(ak) - ilogb(aq), not half of it
+ *   ORC_PSCALE_UNFOLDED  the other admissible reading of the 2^8 P scale:
+ *             y = 2^8 * fp32(exp2(fmaf(S, c, -m))) instead of
+ *             y = fp32(exp2(fmaf(S, c, fp32(8 - m)))) */
+#ifndef ORC_PLANT
+#define ORC_PLANT 0
+#endif
 
 enum {
     ORC_MASK_NONE = 0,
@@ -245,22 +267,82 @@ static void rope_rows(float *x, long n, int D, const float *cs, const float *sn)
  * above applies to the rotated values (the K mean included); V is not
  * rotated.
  */
+/* floor(a / 2) for any int a. */
+static int floor_half(int a)
+{
+    return a >= 0 ? a / 2 : -((1 - a) / 2);
+}
+
+/* Channel equalisation of Q [nq, D] and the smoothed K [nkv, D], in place
+ * (a labelled accuracy variant, not the pages' recipe; the pages' per-block
+ * INT8 recipe is the default).  The scores sum_d Q[i,d] K[j,d] are unchanged
+ * in exact arithmetic when channel d of Q is multiplied and channel d of K
+ * divided by the same power of two.  With aq = max_n |Q[n,d]| and
+ * ak = max_n |K[n,d]|, the exponent is e = floor((ilogb(ak) - ilogb(aq)) / 2),
+ * clamped to [-ORC_EQ_MAX, ORC_EQ_MAX] (0 when either maximum is 0); after
+ * Q 2^e and K 2^-e the two channel maxima lie within a factor (1/2, 4) of each
+ * other, so a K channel with outliers no longer sets the scale of every K
+ * block alone.  Each product is one fp32 multiplication (exact unless it
+ * leaves the normal range). */
+#define ORC_EQ_MAX 32
+static void equalise_channels(float *xq, long nq, float *xk, long nkv, int D, int8_t *eq_exp)
+{
+    for (int d = 0; d < D; d++) {
+        float aq = 0.0f, ak = 0.0f;
+        for (long n = 0; n < nq; n++)
+            if (fabsf(xq[n * D + d]) > aq)
+                aq = fabsf(xq[n * D + d]);
+        for (long n = 0; n < nkv; n++)
+            if (fabsf(xk[n * D + d]) > ak)
+                ak = fabsf(xk[n * D + d]);
+        int e = 0;
+        if (aq > 0.0f && ak > 0.0f) {
+#if ORC_PLANT == 7
+            e = ilogbf(ak) - ilogbf(aq);
+#else
+            e = floor_half(ilogbf(ak) - ilogbf(aq));
+#endif
+            if (e > ORC_EQ_MAX)
+                e = ORC_EQ_MAX;
+            if (e < -ORC_EQ_MAX)
+                e = -ORC_EQ_MAX;
+        }
+        eq_exp[d] = (int8_t)e;
+#if ORC_PLANT == 6
+        const float up = ldexpf(1.0f, e), down = ldexpf(1.0f, e);
+#else
+        const float up = ldexpf(1.0f, e), down = ldexpf(1.0f, -e);
+#endif
+        for (long n = 0; n < nq; n++)
+            xq[n * D + d] = xq[n * D + d] * up;
+        for (long n = 0; n < nkv; n++)
+            xk[n * D + d] = xk[n * D + d] * down;
+    }
+}
+
 static int quant_head_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            long nq, long nkv, int D,
                            const float *q_cos, const float *q_sin,
                            const float *k_cos, const float *k_sin,
                            int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
-                           uint8_t *v8, float *vs)
+                           uint8_t *v8, float *vs, int8_t *eq_exp)
 {
     float *x = (float *)malloc(sizeof(float) * (size_t)((nq > nkv ? nq : nkv) * D));
-    if (!x)
+    float *xq = eq_exp ? (float *)malloc(sizeof(float) * (size_t)(nq * D)) : NULL;
+    if (!x || (eq_exp && !xq)) {
+        free(x);
+        free(xq);
         return 1;
-    /* Q */
+    }
+    /* Q (quantized at once, or kept for the equalisation) */
     for (long i = 0; i < nq * D; i++)
         x[i] = bf16_to_f32(q[i]);
     if (q_cos)
         rope_rows(x, nq, D, q_cos, q_sin);
-    quant_blocks_i8(x, nq, D, q8, qs);
+    if (eq_exp)
+        memcpy(xq, x, sizeof(float) * (size_t)(nq * D));
+    else
+        quant_blocks_i8(x, nq, D, q8, qs);
     /* K (rotated), then its channel mean in the canonical fp64 order */
     for (long i = 0; i < nkv * D; i++)
         x[i] = bf16_to_f32(k[i]);
@@ -282,6 +364,11 @@ static int quant_head_impl(const uint16_t *q, const uint16_t *k, const uint16_t 
     for (long r = 0; r < nkv; r++)
         for (int d = 0; d < D; d++)
             x[r * D + d] = x[r * D + d] - mu[d];
+    if (eq_exp) {
+        equalise_channels(xq, nq, x, nkv, D, eq_exp);
+        quant_blocks_i8(xq, nq, D, q8, qs);
+        free(xq);
+    }
     quant_blocks_i8(x, nkv, D, k8, ks);
     /* V per channel */
     for (int d = 0; d < D; d++) {
@@ -312,7 +399,20 @@ int orc_quant_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                    uint8_t *v8, float *vs)
 {
     return quant_head_impl(q, k, v, nq, nkv, D, NULL, NULL, NULL, NULL,
-                           q8, qs, k8, ks, mu, v8, vs);
+                           q8, qs, k8, ks, mu, v8, vs, NULL);
+}
+
+/* The channel-equalised variant (equalise_channels); eq_exp [D] receives the
+ * exponents e. */
+int orc_quant_head_eq(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                      long nq, long nkv, int D,
+                      int8_t *q8, float *qs, int8_t *k8, float *ks, float *mu,
+                      uint8_t *v8, float *vs, int8_t *eq_exp)
+{
+    if (!eq_exp)
+        return 2;
+    return quant_head_impl(q, k, v, nq, nkv, D, NULL, NULL, NULL, NULL,
+                           q8, qs, k8, ks, mu, v8, vs, eq_exp);
 }
 
 int orc_quant_head_rope(const uint16_t *q, const uint16_t *k, const uint16_t *v,
@@ -325,7 +425,7 @@ int orc_quant_head_rope(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     if (!q_cos || !q_sin || !k_cos || !k_sin)
         return 2;
     return quant_head_impl(q, k, v, nq, nkv, D, q_cos, q_sin, k_cos, k_sin,
-                           q8, qs, k8, ks, mu, v8, vs);
+                           q8, qs, k8, ks, mu, v8, vs, NULL);
 }
 
 /* Exact integer scores S[i,j] = sum_d q8[i,d] * k8[j,d] for rows i0..i0+ni-1
@@ -457,24 +557,69 @@ typedef struct {
      * uncertainty that the rounding slack is meant to cover */
     const int8_t *pert;
     double pert_eps;
+    /* tile columns >= poly_from take the software exp2 (orc_exp2_poly) */
+    int poly_from;
 } attn_job;
 
 static float exp2_f32(float x) { return (float)exp2((double)x); }
 
-/* Compile-time switches used only by the test-suite, which builds separate
- * copies of this library with them to show that its pins catch plausible
- * mistakes (the product build defines neither):
- *   ORC_PLANT = 1  the K scale of key j taken from block j / 128, not j / 64
- *             = 2  l summed from the decoded e4m3 codes instead of from y
- *             = 3  the slack not rescaled by alpha when the running max moves
- *             = 4  the slack gap measured in code units instead of values
- *             = 5  the slack not divided by l
- *   ORC_PSCALE_UNFOLDED  the other admissible reading of the 2^8 P scale:
- *             y = 2^8 * fp32(exp2(fmaf(S, c, -m))) instead of
- *             y = fp32(exp2(fmaf(S, c, fp32(8 - m)))) */
-#ifndef ORC_PLANT
-#define ORC_PLANT 0
+/* Software exp2: the recipe's exp2 for the tile columns >= poly_from (a
+ * reading: the target specification says only "exp2 in registers"; the
+ * device evaluates this share of the exponentials on its fma units instead
+ * of the exp2 unit, and both sides then agree bit for bit).
+ * Cody-Waite style reduction x = j + f with j = round-half-even(x) (adding
+ * and subtracting 1.5 * 2^23) and |f| <= 1/2, a degree-3 polynomial for 2^f
+ * fitted here (minimax relative error on [-1/2, 1/2]; 2^-13.7 including its
+ * fp32 Horner evaluation), and 2^j applied by adding j to the exponent field
+ * of the polynomial's bits.  x is first raised to -125 so that the exponent
+ * field stays normal (a masked key's -inf gives 2^-125 * p(0), whose e4m3
+ * code is 0).  Each step is one fp32 operation rounded to nearest-even or an
+ * integer add. */
+#define ORC_EXP2_C0 0x3f7ffb49u /* 0.999928057 */
+#define ORC_EXP2_C1 0x3f31798du /* 0.693260968 */
+#define ORC_EXP2_C2 0x3e786f0du /* 0.242611125 */
+#define ORC_EXP2_C3 0x3d61fbb0u /* 0.0551716685 */
+
+static float f32_of(uint32_t b)
+{
+    float f;
+    memcpy(&f, &b, 4);
+    return f;
+}
+
+float orc_exp2_poly(float x)
+{
+    const float magic = 12582912.0f; /* 1.5 * 2^23 */
+    const float xc = x > -125.0f ? x : -125.0f;
+    const float t = xc + magic;
+    const float jf = t - magic;
+    const float f = xc - jf;
+    const float p = fmaf(fmaf(fmaf(f32_of(ORC_EXP2_C3), f, f32_of(ORC_EXP2_C2)), f,
+                              f32_of(ORC_EXP2_C1)),
+                         f, f32_of(ORC_EXP2_C0));
+    uint32_t pb, tb;
+    memcpy(&pb, &p, 4);
+    memcpy(&tb, &t, 4);
+    return f32_of(pb + (tb << 23)); /* (t's bits << 23) = j << 23 modulo 2^32 */
+}
+
+void orc_exp2_poly_n(const float *x, long n, float *y)
+{
+    for (long i = 0; i < n; i++)
+        y[i] = orc_exp2_poly(x[i]);
+}
+
+/* The first tile column (0 .. tkv) whose exponentials use orc_exp2_poly; the
+ * recipe's value is ORC_EXP2_POLY_FROM (tkv or more: none).  The setter is
+ * for the tests that pin the polynomial's effect; set it before a call, not
+ * during one. */
+#ifndef ORC_EXP2_POLY_FROM
+#define ORC_EXP2_POLY_FROM 128
 #endif
+static int g_poly_from = ORC_EXP2_POLY_FROM;
+void orc_set_exp2_poly_from(int c) { g_poly_from = c; }
+int orc_get_exp2_poly_from(void) { return g_poly_from; }
+
 
 /* Width, in units of y = p*2^8, of the set of e4m3 codes that an fp32 value
  * within relative distance eps of y can round to; zero when that set is one
@@ -624,14 +769,18 @@ static void attend_range(const attn_job *J, long i, long se, long lo, long hi, c
             } else {
 #ifdef ORC_PSCALE_UNFOLDED
                 (void)nm8;
+                const int poly = 0;
                 float y = 256.0f * exp2_f32(fmaf((float)S[jj], c[jj], -mf));
 #else
                 float x = fmaf((float)S[jj], c[jj], nm8);
-                float y = exp2_f32(x);
+                const int poly = (j % tkv) >= J->poly_from;
+                float y = poly ? orc_exp2_poly(x) : exp2_f32(x);
 #endif
-                if (J->pert && J->pert[i * J->nkv + j] > 0)
+                /* the software exp2 is reproduced exactly: it has neither an
+                 * uncertainty (test hook) nor a slack */
+                if (!poly && J->pert && J->pert[i * J->nkv + j] > 0)
                     y = f32_at_most((double)y * (1.0 + J->pert_eps));
-                else if (J->pert && J->pert[i * J->nkv + j] < 0)
+                else if (!poly && J->pert && J->pert[i * J->nkv + j] < 0)
                     y = f32_at_least((double)y * (1.0 - J->pert_eps));
                 double w = orc_e4m3_decode(orc_e4m3_encode(y));
 #if ORC_PLANT == 2
@@ -639,7 +788,7 @@ static void attend_range(const attn_job *J, long i, long se, long lo, long hi, c
 #else
                 rowsum_f += y;
 #endif
-                double gap = sl ? e4m3_flip_gap((double)y, J->eps) : 0.0;
+                double gap = (sl && !poly) ? e4m3_flip_gap((double)y, J->eps) : 0.0;
                 for (int d = 0; d < D; d++) {
                     double vv = orc_e4m3_decode(J->v8[j * D + d]);
                     acc[d] += w * vv;
@@ -880,6 +1029,7 @@ int orc_attn_rows_bs(const int8_t *q8, const float *qs, const int8_t *k8, const 
     J.mask = mask;
     J.mb = mb;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.eps = eps;
     J.q8 = q8;
     J.qs = qs;
@@ -925,6 +1075,7 @@ int orc_attn_rows_identity_bs(const double *q, const double *k, const double *v,
     J.mask = mask;
     J.mb = mb;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.qd = q;
     J.kd = k;
     J.vd = v;
@@ -962,6 +1113,7 @@ int orc_attn_rows_split(const int8_t *q8, const float *qs, const int8_t *k8, con
     J.mask = mask;
     J.mb = mb;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.eps = eps;
     J.q8 = q8;
     J.qs = qs;
@@ -1001,6 +1153,7 @@ int orc_attn_rows_identity_split(const double *q, const double *k, const double 
     J.mask = mask;
     J.mb = mb;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.qd = q;
     J.kd = k;
     J.vd = v;
@@ -1045,6 +1198,7 @@ int orc_attn_rows_pert(const int8_t *q8, const float *qs, const int8_t *k8, cons
     J.mask = mask;
     J.mb = mb;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.eps = eps;
     J.q8 = q8;
     J.qs = qs;
@@ -1187,6 +1341,7 @@ int orc_attn_rows_win(const int8_t *q8, const float *qs, const int8_t *k8, const
     J.win = win;
     J.sink = sink;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.eps = eps;
     J.q8 = q8;
     J.qs = qs;
@@ -1224,6 +1379,7 @@ int orc_attn_rows_identity_win(const double *q, const double *k, const double *v
     J.win = win;
     J.sink = sink;
     J.tkv = tkv;
+    J.poly_from = g_poly_from;
     J.qd = q;
     J.kd = k;
     J.vd = v;

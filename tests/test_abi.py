@@ -198,3 +198,14 @@ def test_ceiling_arguments_are_rejected_before_any_launch(L):
     assert call(3, scratch=ctypes.c_void_p(4096), nbytes=1 << 19) == 1  # of at least 1 MiB
     assert call(3, scratch=ctypes.c_void_p(4104), nbytes=1 << 30) == 1  # 16-byte aligned
     assert call(0, cycles=None) == 1 and call(0, cycles=ctypes.c_void_p(4100)) == 1
+
+
+def test_noalloc_wrapper_refuses_oversized_shapes_before_any_launch(L):
+    # the Python wrapper checks the scratch size on the host and raises
+    # before it touches the tensors or the C entry point
+    class _Out:
+        shape = sage.make_shape(1, 40, 75600, 75600, 128)
+
+    assert sage.workspace_bytes(_Out.shape) > sage.NOALLOC_SCRATCH_BYTES
+    with pytest.raises(sage.SageError):
+        sage.quant_qk_noalloc(None, None, None, _Out())

@@ -57,6 +57,38 @@ def test_noalloc_matches_quant_qk_on_two_calls_in_a_row():
             assert torch.equal(out.bufs[name], ref.bufs[name]), name
 
 
+def test_noalloc_allocates_nothing():
+    # after a warm-up call (which looks up the scratch array's address), two
+    # more calls change neither the device's free memory nor torch's pool
+    w = synth.Workload("noalloc_mem", 1, 4, 500, 700, 128, k_offset_var=4.0, seed=73)
+    q, k, v = _inputs(w)
+    out = sage.QuantizedQKV(sage.make_shape(w.B, w.H, w.Nq, w.Nkv, w.D), q.device)
+    assert _noalloc(q, k, v, out) == 0
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for _ in range(2):
+        assert _noalloc(q, k, v, out) == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert sage.sync_status() == 0
+
+
+def test_python_wrapper_matches_quant_qk():
+    w = synth.Workload("noalloc_py", 1, 2, 200, 450, 64, outlier_mag=5.0, seed=74)
+    q, k, v = _inputs(w)
+    out = sage.QuantizedQKV(sage.make_shape(w.B, w.H, w.Nq, w.Nkv, w.D), q.device)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        sage.quant_qk_noalloc(q, k, v, out, stream=stream)
+    torch.cuda.current_stream().wait_stream(stream)
+    ref = sage.quant_qk(q, k, v)
+    assert sage.sync_status() == 0
+    for name in sage.BUFFERS:
+        assert torch.equal(out.bufs[name], ref.bufs[name]), name
+
+
 def test_noalloc_refuses_shapes_beyond_its_scratch():
     w = synth.P720  # needs about 72 MB of scratch, more than the fixed 16 MiB
     shape = sage.make_shape(w.B, w.H, w.Nq, w.Nkv, w.D)
