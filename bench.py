@@ -68,6 +68,10 @@ def parse():
                     help="time sage_quant_qk_rope (RoPE applied to Q and K inside the quantizer, "
                          "1D angles pos * 10000^(-2p/D)) against sage_quant_qk on the workload, "
                          "one JSON line")
+    ap.add_argument("--equalized", action="store_true",
+                    help="the channel-equalised quantization variant against the recipe on the "
+                         "workload: quantizer time and the accuracy of sampled rows against fp64 "
+                         "attention, one JSON line")
     ap.add_argument("--sweep-filter", default="",
                     help="only sweep points whose name contains this string")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -520,13 +524,13 @@ def run_ours(args):
 
 # ------------------------------------------------------------------ sweep
 
-def fp64_rows(w, q, k, v, rows):
+def fp64_rows(w, q, k, v, rows, b=0, h=0):
     """Textbook softmax attention in fp64 (torch, on the GPU) for the given
-    query rows of head (0, 0): the full-precision accuracy reference."""
+    query rows of head (b, h): the full-precision accuracy reference."""
     import torch
     rows = torch.as_tensor(rows, device=q.device, dtype=torch.int64)
-    qd = q[0, 0, rows].double()
-    kd, vd = k[0, 0].double(), v[0, 0].double()
+    qd = q[b, h, rows].double()
+    kd, vd = k[b, h].double(), v[b, h].double()
     s = (qd @ kd.T) / float(np.sqrt(w.D))
     g = rows + (w.Nkv - w.Nq)
     if w.mask == 1:
@@ -738,6 +742,70 @@ def run_rope(args):
         "table_bytes": 8 * (w.Nq + w.Nkv) * (w.D // 2)}), flush=True)
 
 
+def run_equalized(args):
+    """sage_quant_qk_equalized (a labelled accuracy variant outside the
+    recipe) against sage_quant_qk on the workload's seeded inputs: quantizer
+    time (CUDA events, inputs resident) and, for both, the accuracy of 64
+    sampled query rows of three heads against fp64 attention."""
+    import torch
+    import bit_quantized_attention_sage_b200 as sage
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    sage.lib()
+    w = synth.WORKLOADS[args.workload]
+    runner = Runner(w, 0, device)
+    q, k, v = runner.q, runner.k, runner.v
+    plain = sage.quant_qk(q, k, v)
+    eq = sage.quant_qk_equalized(q, k, v)
+    ws_p = torch.empty(max(sage.workspace_bytes(plain.shape), 16), dtype=torch.uint8, device=device)
+    ws_e = torch.empty(max(sage.equalized_workspace_bytes(eq.shape), 16), dtype=torch.uint8,
+                       device=device)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    t_plain = timed(lambda: sage.quant_qk(q, k, v, out=plain, workspace=ws_p))
+    t_eq = timed(lambda: sage.quant_qk_equalized(q, k, v, out=eq, workspace=ws_e))
+    rng = np.random.default_rng(w.seed)
+    heads = sorted(set([0, w.B * w.H - 1]) | set(rng.choice(w.B * w.H, 1).tolist()))
+    acc = {}
+    for name, qkv in (("recipe", plain), ("equalized", eq)):
+        o32 = torch.empty((w.B, w.H, w.Nq, w.D), dtype=torch.float32, device=device)
+        sage.attn_fwd(qkv, w.mask, w.mask_block, out=runner.o, o_f32=o32)
+        got, ref = [], []
+        for bh in heads:
+            b, h = divmod(bh, w.H)
+            rows = np.sort(np.random.default_rng(w.seed + bh).choice(w.Nq, size=min(64, w.Nq),
+                                                                     replace=False))
+            got.append(o32[b, h, torch.as_tensor(rows, device=device)].double())
+            ref.append(fp64_rows(w, q, k, v, rows, b, h))
+        got, ref = torch.cat(got), torch.cat(ref)
+        cos = float(torch.nn.functional.cosine_similarity(got.flatten(), ref.flatten(), dim=0))
+        rel = float((got - ref).abs().sum() / ref.abs().sum())
+        acc[name] = {"cos_vs_fp64": round(cos, 6), "relL1_vs_fp64": round(rel, 5)}
+        del o32
+    if sage.sync_status() != 0:
+        raise RuntimeError("device status error in the equalised quantizer run")
+    alg = 3 * w.B * w.H * (w.Nq + 2 * w.Nkv) * w.D
+    print(json.dumps({
+        "equalized_quantizer": w.name, "outlier_mag": w.outlier_mag,
+        "quant_ms": round(t_plain, 4), "quant_equalized_ms": round(t_eq, 4),
+        "quant_GBps_alg": round(alg / (t_plain / 1e3) / 1e9, 1),
+        "quant_equalized_GBps_alg": round(alg / (t_eq / 1e3) / 1e9, 1),
+        "rows": "64 sampled query rows of heads %s" % heads, **{
+            "%s_%s" % (n, key): val for n, d in acc.items() for key, val in d.items()}}),
+        flush=True)
+
+
 # ------------------------------------------------------------------ reference arm
 
 CEILING_PLAN = [  # kind, iters, MMA N, unit of one operation
@@ -849,6 +917,8 @@ def main():
         run_w8a8(args)
     elif args.rope:
         run_rope(args)
+    elif args.equalized:
+        run_equalized(args)
     elif args.ceilings:
         run_ceilings(args)
     else:

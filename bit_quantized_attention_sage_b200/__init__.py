@@ -66,6 +66,10 @@ def lib():
         L.sage_quant_qk.argtypes = [P, P, P, P, P, P, SZ, P]
         L.sage_quant_qk_rope.restype = I
         L.sage_quant_qk_rope.argtypes = [P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.sage_quant_equalized_workspace_bytes.restype = SZ
+        L.sage_quant_equalized_workspace_bytes.argtypes = [P]
+        L.sage_quant_qk_equalized.restype = I
+        L.sage_quant_qk_equalized.argtypes = [P, P, P, P, P, P, P, SZ, P]
         L.sage_window_keys.restype = I
         L.sage_window_keys.argtypes = [P, I, I, I, P, P, P]
         L.sage_quant_qk_window.restype = I
@@ -203,6 +207,38 @@ def quant_qk(q, k, v, out=None, workspace=None, stream=None, rope=None):
                                         *[_ptr(t) for t in rope], ctypes.byref(qs),
                                         _ptr(workspace), workspace.numel(), _stream(stream)),
                "sage_quant_qk_rope")
+    return out
+
+
+def equalized_workspace_bytes(shape):
+    """sage_quant_equalized_workspace_bytes."""
+    return int(lib().sage_quant_equalized_workspace_bytes(ctypes.byref(shape)))
+
+
+def quant_qk_equalized(q, k, v, out=None, eq_exp=None, workspace=None, stream=None):
+    """sage_quant_qk_equalized (a labelled accuracy variant outside the
+    recipe): channel d of Q times 2^e[d] and of the smoothed K times 2^-e[d]
+    before the block codes.  q, k, v bf16 CUDA [B, H, N, D]; eq_exp: None or
+    an int8 CUDA tensor [B, H, D] that receives e.  Returns QuantizedQKV."""
+    import torch
+    B, H, Nq, D = q.shape
+    shape = make_shape(B, H, Nq, k.shape[2], D)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if eq_exp is not None and (eq_exp.dtype != torch.int8 or not eq_exp.is_cuda
+                               or not eq_exp.is_contiguous() or tuple(eq_exp.shape) != (B, H, D)):
+        raise ValueError("eq_exp must be a contiguous int8 CUDA tensor [B, H, D]")
+    if out is None:
+        out = QuantizedQKV(shape, q.device)
+    if workspace is None:
+        workspace = torch.empty(max(equalized_workspace_bytes(shape), 16), dtype=torch.uint8,
+                                device=q.device)
+    qs = out.struct()
+    _check(lib().sage_quant_qk_equalized(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(shape),
+                                         ctypes.byref(qs), None if eq_exp is None else _ptr(eq_exp),
+                                         _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sage_quant_qk_equalized")
     return out
 
 

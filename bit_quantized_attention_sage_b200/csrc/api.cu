@@ -106,6 +106,14 @@ size_t workspace_bytes(const sage_shape* s) {
   return bh * (pad64(s->Nkv) / 64) * D * 12 + bh * D * 4;
 }
 
+// sage_quant_qk_equalized: the base workspace, then the per-block channel
+// maxima of |Q| and maxima and minima of K, then the factors 2^e and 2^-e.
+size_t eq_workspace_bytes(const sage_shape* s) {
+  const size_t bh = static_cast<size_t>(s->B) * s->H, D = s->D;
+  return workspace_bytes(s) +
+         bh * D * 4 * (pad64(s->Nq) / 64 + 2 * (pad64(s->Nkv) / 64) + 2);
+}
+
 bool qkv_ok(const sage_qkv_quant* q) {
   return q && aligned16(q->q_i8) && aligned16(q->q_scale) && aligned16(q->k_i8) &&
          aligned16(q->k_scale) && aligned16(q->k_mean) && aligned16(q->v_f8) &&
@@ -338,11 +346,13 @@ void window_key_ranges(const sage_shape* s, int frame, int win, int sink, int* n
 sage_status quant_common(const void* q_bf16, const void* k_bf16, const void* v_bf16,
                          const sage_shape* shape, const float* const rope[4],
                          const sage_qkv_quant* out, void* workspace, size_t ws_bytes,
-                         void* stream, int nkv_src = -1, int kv_split = -1, int kv_gap = 0) {
+                         void* stream, int nkv_src = -1, int kv_split = -1, int kv_gap = 0,
+                         bool eq = false, int8_t* eq_exp = nullptr) {
   if (!shape_ok(shape) || !qkv_ok(out)) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(workspace))
     return SAGE_ERR_INVALID_ARG;
-  if (ws_bytes < workspace_bytes(shape)) return SAGE_ERR_INVALID_ARG;
+  if (ws_bytes < (eq ? eq_workspace_bytes(shape) : workspace_bytes(shape)))
+    return SAGE_ERR_INVALID_ARG;
   if (rope)
     for (int i = 0; i < 4; i++)
       if (!aligned16(rope[i])) return SAGE_ERR_INVALID_ARG;
@@ -369,6 +379,17 @@ sage_status quant_common(const void* q_bf16, const void* k_bf16, const void* v_b
   a.Nkv_src = nkv_src < 0 ? a.Nkv : nkv_src;
   a.kv_split = kv_split < 0 ? a.Nkv : kv_split;
   a.kv_gap = kv_gap;
+  if (eq) {
+    const size_t qcells = static_cast<size_t>(a.BH) * (pad64(a.Nq) / 64) * a.D;
+    float* x = reinterpret_cast<float*>(static_cast<char*>(workspace) + workspace_bytes(shape));
+    a.eq = true;
+    a.ws_qmax = x;
+    a.ws_kmax = x + qcells;
+    a.ws_kmin = x + qcells + cells;
+    a.ws_eq_up = x + qcells + 2 * cells;
+    a.ws_eq_down = a.ws_eq_up + static_cast<size_t>(a.BH) * a.D;
+    a.eq_exp = eq_exp;
+  }
   if (rope) {
     a.q_cos = rope[0];
     a.q_sin = rope[1];
@@ -384,6 +405,18 @@ SAGE_EXPORT sage_status sage_quant_qk(const void* q_bf16, const void* k_bf16, co
                                       const sage_shape* shape, const sage_qkv_quant* out,
                                       void* workspace, size_t ws_bytes, void* stream) {
   return quant_common(q_bf16, k_bf16, v_bf16, shape, nullptr, out, workspace, ws_bytes, stream);
+}
+
+SAGE_EXPORT size_t sage_quant_equalized_workspace_bytes(const sage_shape* shape) {
+  return shape_ok(shape) ? eq_workspace_bytes(shape) : 0;
+}
+
+SAGE_EXPORT sage_status sage_quant_qk_equalized(const void* q_bf16, const void* k_bf16,
+                                                const void* v_bf16, const sage_shape* shape,
+                                                const sage_qkv_quant* out, int8_t* eq_exp,
+                                                void* workspace, size_t ws_bytes, void* stream) {
+  return quant_common(q_bf16, k_bf16, v_bf16, shape, nullptr, out, workspace, ws_bytes, stream, -1,
+                      -1, 0, true, eq_exp);
 }
 
 SAGE_EXPORT sage_status sage_window_keys(const sage_shape* shape, int frame, int win, int sink,

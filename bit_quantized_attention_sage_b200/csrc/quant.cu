@@ -176,7 +176,20 @@ __device__ __forceinline__ void quant_block_store(float (&x)[CH][8], int valid, 
   if (threadIdx.x == 0) *scale_out = scale;
 }
 
-template <int D, bool ROPE>
+// Channel maxima of |x| over the valid rows of a 64 x D bf16 block staged in
+// shared memory (thread t < D: channel t).
+template <int D>
+__device__ __forceinline__ float channel_absmax(const uint16_t* blk, int valid, int t) {
+  float m = 0.0f;
+  for (int r = 0; r < valid; r++)
+    m = fmaxf(m, fabsf(__uint_as_float(static_cast<uint32_t>(blk[r * D + t]) << 16)));
+  return m;
+}
+
+// pass 1.  EQ (channel equalisation): the Q codes wait for the per-channel
+// factors, so a Q block only records its channel maxima here, and a K block
+// also its channel maxima and minima.
+template <int D, bool ROPE, bool EQ>
 __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;  // chunks per thread
@@ -194,7 +207,21 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
   const int nqb = (a.Nq + kBlk - 1) / kBlk;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
 
-  if (blk < nqb) {  // Q block: codes and scale
+  if (EQ && blk < nqb) {  // Q block: channel maxima of |Q|
+    const int valid = min(kBlk, a.Nq - blk * kBlk);
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.q + (static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(blk) * kBlk) * D);
+#pragma unroll
+    for (int c = 0; c < CH; c++) {
+      const int chunk = c * kThreads + threadIdx.x;
+      if (chunk / kChunksPerRow < valid) reinterpret_cast<uint4*>(ks)[chunk] = __ldg(src + chunk);
+    }
+    __syncthreads();
+    if (threadIdx.x < D)
+      a.ws_qmax[(static_cast<size_t>(bh) * nqb + blk) * D + threadIdx.x] =
+          channel_absmax<D>(ks, valid, threadIdx.x);
+    __syncthreads();  // the staging area is reused by the K / V block
+  } else if (blk < nqb) {  // Q block: codes and scale
     const int valid = min(kBlk, a.Nq - blk * kBlk);
     const uint4* src = reinterpret_cast<const uint4*>(
         a.q + (static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(blk) * kBlk) * D);
@@ -290,17 +317,45 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
     const int t = threadIdx.x;
     if (t < D) {  // fp64 sum of channel t, ascending token order
       double s = 0.0;
-      for (int r = 0; r < valid; r++)
-        s = __dadd_rn(s, static_cast<double>(__uint_as_float(static_cast<uint32_t>(ks[r * D + t]) << 16)));
+      float mx = -INFINITY, mn = INFINITY;
+      for (int r = 0; r < valid; r++) {
+        const float x = __uint_as_float(static_cast<uint32_t>(ks[r * D + t]) << 16);
+        s = __dadd_rn(s, static_cast<double>(x));
+        if (EQ) {
+          mx = fmaxf(mx, x);
+          mn = fminf(mn, x);
+        }
+      }
       a.ws_ksum[ws + t] = s;
+      if (EQ) {
+        a.ws_kmax[ws + t] = mx;
+        a.ws_kmin[ws + t] = mn;
+      }
     } else if (t < 2 * D) {  // max |V| of channel t - D
-      const int d = t - D;
-      float m = 0.0f;
-      for (int r = 0; r < valid; r++)
-        m = fmaxf(m, fabsf(__uint_as_float(static_cast<uint32_t>(vsm[r * D + d]) << 16)));
-      a.ws_vmax[ws + d] = m;
+      a.ws_vmax[ws + t - D] = channel_absmax<D>(vsm, valid, t - D);
     }
   }
+}
+
+// floor(log2 x) of a finite x > 0 (normal or subnormal), from its bits.
+__device__ __forceinline__ int floor_log2(float x) {
+  const uint32_t b = __float_as_uint(x);
+  const int ef = static_cast<int>((b >> 23) & 0xFF);
+  return ef ? ef - 127 : (31 - __clz(static_cast<int>(b & 0x7FFFFF))) - 149;
+}
+
+constexpr int kEqMax = 32;  // |e| limit of the channel equalisation
+
+// Channel equalisation exponent of channel d (finalize, EQ): aq = max |Q|,
+// ak = max |fp32(K - mu)|, which, fp32 subtraction being monotone, is the
+// larger of |fp32(kmax - mu)| and |fp32(kmin - mu)|; e = floor((floor(log2
+// ak) - floor(log2 aq)) / 2) in [-kEqMax, kEqMax], 0 if either is 0.
+__device__ __forceinline__ int eq_exponent(float aq, float kmax, float kmin, float mu) {
+  const float ak = fmaxf(fabsf(__fsub_rn(kmax, mu)), fabsf(__fsub_rn(kmin, mu)));
+  if (!(aq > 0.0f) || !(ak > 0.0f)) return 0;
+  const int t = floor_log2(ak) - floor_log2(aq);
+  const int e = t >= 0 ? t / 2 : -((1 - t) / 2);
+  return e > kEqMax ? kEqMax : (e < -kEqMax ? -kEqMax : e);
 }
 
 // One CTA per (head, 32 channels).  The fp64 block sums of a channel must be
@@ -313,40 +368,69 @@ constexpr int kFinChunk = 128;  // blocks per staged chunk
 constexpr int kFinCh = 32;      // channels per CTA
 
 __global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
+  constexpr int kGroups = kThreads / kFinCh;  // 8 row groups
   __shared__ double part[kFinChunk][kFinCh];
-  __shared__ float vred[kThreads / kFinCh][kFinCh];
+  __shared__ float vred[kGroups][kFinCh];
+  __shared__ float xred[3][kGroups][kFinCh];   // equalisation: K max, K min, |Q| max
   const int D = a.D;
   const int bh = blockIdx.y;
   const int d0 = blockIdx.x * kFinCh;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
   const int lane = threadIdx.x % kFinCh;       // channel d0 + lane
   const int rowg = threadIdx.x / kFinCh;       // 0 .. 7
+  const bool eq = a.eq;
   double total = 0.0;
-  float m = 0.0f;
+  float m = 0.0f, kmx = -INFINITY, kmn = INFINITY, qmx = 0.0f;
   for (int b0 = 0; b0 < nkb; b0 += kFinChunk) {
     const int nb = min(kFinChunk, nkb - b0);
-    for (int r = rowg; r < nb; r += kThreads / kFinCh) {
+    for (int r = rowg; r < nb; r += kGroups) {
       const size_t w = (static_cast<size_t>(bh) * nkb + b0 + r) * D + d0 + lane;
       part[r][lane] = a.ws_ksum[w];
       m = fmaxf(m, a.ws_vmax[w]);
+      if (eq) {
+        kmx = fmaxf(kmx, a.ws_kmax[w]);
+        kmn = fminf(kmn, a.ws_kmin[w]);
+      }
     }
     __syncthreads();
     if (threadIdx.x < kFinCh)
       for (int r = 0; r < nb; r++) total = __dadd_rn(total, part[r][threadIdx.x]);
     __syncthreads();
   }
+  if (eq) {
+    const int nqb = (a.Nq + kBlk - 1) / kBlk;
+    for (int r = rowg; r < nqb; r += kGroups)
+      qmx = fmaxf(qmx, a.ws_qmax[(static_cast<size_t>(bh) * nqb + r) * D + d0 + lane]);
+    xred[0][rowg][lane] = kmx;
+    xred[1][rowg][lane] = kmn;
+    xred[2][rowg][lane] = qmx;
+  }
   vred[rowg][lane] = m;
   __syncthreads();
   if (threadIdx.x < kFinCh) {
-    for (int g = 1; g < kThreads / kFinCh; g++) m = fmaxf(m, vred[g][threadIdx.x]);
+    for (int g = 1; g < kGroups; g++) m = fmaxf(m, vred[g][threadIdx.x]);
     const int idx = bh * D + d0 + threadIdx.x;
-    a.k_mean[idx] = __double2float_rn(__ddiv_rn(total, static_cast<double>(a.Nkv)));
+    const float mu = __double2float_rn(__ddiv_rn(total, static_cast<double>(a.Nkv)));
+    a.k_mean[idx] = mu;
     a.v_scale[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 448.0f);
     a.ws_vinv[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(448.0f, m);
+    if (eq) {
+      for (int g = 1; g < kGroups; g++) {
+        kmx = fmaxf(kmx, xred[0][g][threadIdx.x]);
+        kmn = fminf(kmn, xred[1][g][threadIdx.x]);
+        qmx = fmaxf(qmx, xred[2][g][threadIdx.x]);
+      }
+      const int e = eq_exponent(qmx, kmx, kmn, mu);
+      a.ws_eq_up[idx] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);    // 2^e
+      a.ws_eq_down[idx] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+      if (a.eq_exp) a.eq_exp[idx] = static_cast<int8_t>(e);
+    }
   }
 }
 
-template <int D, bool ROPE>
+// pass 2.  EQ: the grid also covers the Q blocks, whose codes are taken
+// here from Q * 2^e; the smoothed K is multiplied by 2^-e before its codes.
+template <int D, bool ROPE, bool EQ>
 __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;
@@ -356,6 +440,27 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
   const int bh = ROPE ? blockIdx.x : blockIdx.y;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
   const int nkv_pad = nkb * kBlk;
+  if constexpr (EQ) {
+    const int nqb = (a.Nq + kBlk - 1) / kBlk;
+    if (blk < nqb) {  // Q * 2^e: block codes and scale
+      const int qvalid = min(kBlk, a.Nq - blk * kBlk);
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.q + (static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(blk) * kBlk) * D);
+      const float* up = a.ws_eq_up + static_cast<size_t>(bh) * D;
+      float x[CH][8];
+#pragma unroll
+      for (int c = 0; c < CH; c++) {
+        const int chunk = c * kThreads + threadIdx.x;
+        const int col = (chunk % kChunksPerRow) * 8;
+        unpack8(chunk / kChunksPerRow < qvalid ? __ldg(src + chunk) : make_uint4(0, 0, 0, 0), x[c]);
+#pragma unroll
+        for (int e = 0; e < 8; e++) x[c][e] = __fmul_rn(x[c][e], __ldg(up + col + e));
+      }
+      quant_block_store<D, CH>(x, qvalid, a.q_i8 + (static_cast<size_t>(bh) * nqb + blk) * kBlk * D,
+                               a.q_scale + static_cast<size_t>(bh) * nqb + blk, red);
+    }
+    if (blk >= nkb) return;  // uniform over the CTA
+  }
   const int valid = min(kBlk, a.Nkv - blk * kBlk);
   // The V loads are issued first, together with the K loads, so that the
   // whole 64-token block of K and V is in flight at once.  Chunk c*256 + t
@@ -392,6 +497,11 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
       if constexpr (ROPE) rope_apply(x[c], rc[c], rs[c]);
 #pragma unroll
       for (int e = 0; e < 8; e++) x[c][e] = __fsub_rn(x[c][e], __ldg(mu + col + e));
+      if constexpr (EQ) {
+        const float* down = a.ws_eq_down + static_cast<size_t>(bh) * D;
+#pragma unroll
+        for (int e = 0; e < 8; e++) x[c][e] = __fmul_rn(x[c][e], __ldg(down + col + e));
+      }
     }
     int8_t* codes = a.k_i8 + (static_cast<size_t>(bh) * nkb + blk) * kBlk * D;
     quant_block_store<D, CH>(x, valid, codes, a.k_scale + static_cast<size_t>(bh) * nkb + blk,
@@ -441,18 +551,23 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream) {
   const bool rope = a.q_cos != nullptr;
   const dim3 r1(a.BH, g1.x), r2(a.BH, g2.x);  // rotary variant: heads fastest
   if (rope && g1.x > 65535) return cudaErrorInvalidConfiguration;
+  if (rope && a.eq) return cudaErrorInvalidValue;  // not offered together
   if (a.D == 128) {
-    if (rope) k_quant_pass1<128, true><<<r1, kThreads, 0, stream>>>(a);
-    else k_quant_pass1<128, false><<<g1, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass1<128, true, false><<<r1, kThreads, 0, stream>>>(a);
+    else if (a.eq) k_quant_pass1<128, false, true><<<g1, kThreads, 0, stream>>>(a);
+    else k_quant_pass1<128, false, false><<<g1, kThreads, 0, stream>>>(a);
     k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
-    if (rope) k_quant_pass2<128, true><<<r2, kThreads, 0, stream>>>(a);
-    else k_quant_pass2<128, false><<<g2, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass2<128, true, false><<<r2, kThreads, 0, stream>>>(a);
+    else if (a.eq) k_quant_pass2<128, false, true><<<g1, kThreads, 0, stream>>>(a);
+    else k_quant_pass2<128, false, false><<<g2, kThreads, 0, stream>>>(a);
   } else {
-    if (rope) k_quant_pass1<64, true><<<r1, kThreads, 0, stream>>>(a);
-    else k_quant_pass1<64, false><<<g1, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass1<64, true, false><<<r1, kThreads, 0, stream>>>(a);
+    else if (a.eq) k_quant_pass1<64, false, true><<<g1, kThreads, 0, stream>>>(a);
+    else k_quant_pass1<64, false, false><<<g1, kThreads, 0, stream>>>(a);
     k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
-    if (rope) k_quant_pass2<64, true><<<r2, kThreads, 0, stream>>>(a);
-    else k_quant_pass2<64, false><<<g2, kThreads, 0, stream>>>(a);
+    if (rope) k_quant_pass2<64, true, false><<<r2, kThreads, 0, stream>>>(a);
+    else if (a.eq) k_quant_pass2<64, false, true><<<g1, kThreads, 0, stream>>>(a);
+    else k_quant_pass2<64, false, false><<<g2, kThreads, 0, stream>>>(a);
   }
   return cudaGetLastError();
 }

@@ -32,6 +32,17 @@ struct QuantArgs {
   // else r + kv_gap, of Nkv_src rows per head (no gather: Nkv_src = Nkv,
   // kv_split = Nkv, kv_gap = 0)
   int Nkv_src, kv_split, kv_gap;
+  // channel equalisation (sage_quant_qk_equalized; false: the recipe as is):
+  // per-block channel maxima of |Q| [BH, nqb, D], maxima and minima of K
+  // [BH, nkb, D], the per-channel factors 2^e and 2^-e [BH, D], and the
+  // optional exponent output e [BH, D]
+  bool eq;
+  float* ws_qmax;
+  float* ws_kmax;
+  float* ws_kmin;
+  float* ws_eq_up;
+  float* ws_eq_down;
+  int8_t* eq_exp;
 };
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream);

@@ -177,6 +177,37 @@ sage_status sage_quant_qk_rope(const void *q_bf16, const void *k_bf16, const voi
                                const sage_qkv_quant *out, void *workspace,
                                size_t workspace_bytes, void *stream);
 
+/* Device workspace sage_quant_qk_equalized needs for `shape` (bytes; 0 on an
+ * invalid shape): sage_quant_workspace_bytes(shape) + B*H*D*4*(ceil(Nq/64) +
+ * 2*ceil(Nkv/64) + 2).  Its contents never need initialising. */
+size_t sage_quant_equalized_workspace_bytes(const sage_shape *shape);
+
+/* Channel-equalised quantization: a labelled accuracy variant of
+ * sage_quant_qk, outside the pages' recipe (which sage_quant_qk computes).
+ *
+ * The pages present 8-bit attention as nearly lossless for video models
+ * (reportify.cn TurboDiffusion notes, "几乎无损"); with per-block INT8 codes a
+ * K channel that carries outliers sets the scale of every K block it lives in,
+ * and the INT8 error of Q K^T then dominates.  This variant, before the
+ * per-block INT8 codes, multiplies channel d of Q by 2^e[d] and divides
+ * channel d of the smoothed key fp32(K - mu) by 2^e[d] (each one fp32
+ * multiplication), which leaves every score unchanged in exact arithmetic:
+ *   aq = max_n |Q[n,d]|, ak = max_n |fp32(K[n,d] - mu[d])| (per b, h, d),
+ *   e = floor((floor(log2 ak) - floor(log2 aq)) / 2) clamped to [-32, 32],
+ *   e = 0 when aq or ak is 0.
+ * The K mean, the V codes and scales, and the layout of every output are
+ * those of sage_quant_qk; sage_attn_fwd and the other attention calls take
+ * the result unchanged.  Q is read twice (its channel maxima, then its codes).
+ *
+ *   q_bf16 ... out, stream  as for sage_quant_qk (no rotation)
+ *   eq_exp                  NULL, or device int8 [B, H, D]: receives e
+ *   workspace               at least sage_quant_equalized_workspace_bytes
+ * Enqueues three kernels.  Errors as sage_quant_qk. */
+sage_status sage_quant_qk_equalized(const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                                    const sage_shape *shape, const sage_qkv_quant *out,
+                                    int8_t *eq_exp, void *workspace, size_t workspace_bytes,
+                                    void *stream);
+
 /* The keys a sliding-window step attends to (the union over its query rows
  * of the keys sage_attn_fwd_window lets them see): the reference context
  * [0, *n_sink) and the window [*lo, *hi) of the cache of `shape` (queries are

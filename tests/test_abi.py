@@ -49,6 +49,10 @@ def test_buffer_and_workspace_sizes(L):
     assert b["k_mean"] == 2 * 128 * 4 and b["v_scale"] == 2 * 128 * 4
     assert b["v_f8"] == 2 * 128 * nkp
     assert sage.workspace_bytes(s) == 2 * 47 * 128 * 12 + 2 * 128 * 4
+    # equalised variant: + |Q| maxima per Q block, K maxima and minima per K
+    # block, the two factors per channel
+    assert sage.equalized_workspace_bytes(s) == (sage.workspace_bytes(s) +
+                                                 2 * 128 * 4 * (16 + 2 * 47 + 2))
 
 
 @pytest.mark.parametrize("shape", [(0, 1, 8, 8, 128), (1, 1, 8, 8, 96), (1, 1, 0, 8, 64),
@@ -58,6 +62,7 @@ def test_invalid_shapes(L, shape):
     sizes = (ctypes.c_size_t * 7)()
     assert L.sage_quant_buffer_bytes(ctypes.byref(s), sizes) == 1
     assert L.sage_quant_workspace_bytes(ctypes.byref(s)) == 0
+    assert L.sage_quant_equalized_workspace_bytes(ctypes.byref(s)) == 0
 
 
 def test_invalid_arguments_are_rejected_before_any_launch(L):
