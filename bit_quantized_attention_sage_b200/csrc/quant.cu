@@ -208,18 +208,41 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
 
   if (EQ && blk < nqb) {  // Q block: channel maxima of |Q|
+    // Thread t holds the 8 channels of group t mod (D/8) in CH rows; the
+    // lanes of a warp that share a group combine by shuffles, the warps
+    // through shared memory (rows past `valid` read as 0, which no maximum
+    // of magnitudes can exceed).
     const int valid = min(kBlk, a.Nq - blk * kBlk);
     const uint4* src = reinterpret_cast<const uint4*>(
         a.q + (static_cast<size_t>(bh) * a.Nq + static_cast<size_t>(blk) * kBlk) * D);
+    float mx[8];
+#pragma unroll
+    for (int e = 0; e < 8; e++) mx[e] = 0.0f;
 #pragma unroll
     for (int c = 0; c < CH; c++) {
       const int chunk = c * kThreads + threadIdx.x;
-      if (chunk / kChunksPerRow < valid) reinterpret_cast<uint4*>(ks)[chunk] = __ldg(src + chunk);
+      float x[8];
+      unpack8(chunk / kChunksPerRow < valid ? __ldg(src + chunk) : make_uint4(0, 0, 0, 0), x);
+#pragma unroll
+      for (int e = 0; e < 8; e++) mx[e] = fmaxf(mx[e], fabsf(x[e]));
+    }
+#pragma unroll
+    for (int o = kChunksPerRow; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; e++) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], o));
+    float* red8 = reinterpret_cast<float*>(stage);  // [warp][channel]
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    if (lane < kChunksPerRow) {
+#pragma unroll
+      for (int e = 0; e < 8; e++) red8[wp * D + lane * 8 + e] = mx[e];
     }
     __syncthreads();
-    if (threadIdx.x < D)
-      a.ws_qmax[(static_cast<size_t>(bh) * nqb + blk) * D + threadIdx.x] =
-          channel_absmax<D>(ks, valid, threadIdx.x);
+    if (threadIdx.x < D) {
+      float m = red8[threadIdx.x];
+#pragma unroll
+      for (int w2 = 1; w2 < kThreads / 32; w2++) m = fmaxf(m, red8[w2 * D + threadIdx.x]);
+      a.ws_qmax[(static_cast<size_t>(bh) * nqb + blk) * D + threadIdx.x] = m;
+    }
     __syncthreads();  // the staging area is reused by the K / V block
   } else if (blk < nqb) {  // Q block: codes and scale
     const int valid = min(kBlk, a.Nq - blk * kBlk);
