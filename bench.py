@@ -163,6 +163,26 @@ def kernel_hash():
     return h.hexdigest()[:16]
 
 
+def quant_kernel_hash():
+    h = hashlib.sha256()
+    for f in ("quant.cu", "quant.cuh", "sm100.cuh"):
+        h.update(open(os.path.join(ROOT, "bit_quantized_attention_sage_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_quant_traffic(workload):
+    """DRAM bytes of one sage_quant_qk call (its three kernels) on `workload`
+    from the committed ncu summary, if it was taken on the current quantizer
+    source and that workload; else None."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "quant_traffic.json")))
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_hash") != quant_kernel_hash() or rec.get("workload") != workload:
+        return None
+    return rec
+
+
 def recorded_traffic():
     """DRAM bytes per attention launch from the committed ncu summary, if it
     was taken on the current kernel source; else None."""
@@ -471,6 +491,7 @@ def run_ours(args):
     achieved = ops_rank / (t["attn_ms"] / 1e3) / 1e12
     # the dense kernel's record
     traffic = recorded_traffic() if kv_splits == 1 and w.mask != 3 else None
+    qtraffic = recorded_quant_traffic(w.name)
     # algorithmic bytes of sage_quant_qk: read bf16 (2 B) and write one 8-bit
     # code (1 B) per element of Q, K and V, plus the scales and the K mean
     quant_bytes = 3 * w.B * w.H * (w.Nq + 2 * w.Nkv) * w.D + 4 * w.B * w.H * (
@@ -499,7 +520,12 @@ def run_ours(args):
                            "peak": pk["hbm"], "unit": "GB/s",
                            "frac": round(quant_bytes / (t["quant_ms"] / 1e3) / 1e9 / pk["hbm"], 4),
                            "ms_per_step": round(t["quant_ms"], 4),
-                           "algorithmic_bytes": quant_bytes},
+                           "algorithmic_bytes": quant_bytes,
+                           # DRAM bytes the three kernels move (ncu, committed summary):
+                           # the second read of K and V included
+                           "traffic": qtraffic["bytes_per_call"] if qtraffic else None,
+                           "dram_GBps": round(qtraffic["bytes_per_call"] / (t["quant_ms"] / 1e3) / 1e9, 1)
+                           if qtraffic else None},
         "gpu_launches": (KERNELS_PER_STEP + (kv_splits > 1)) * args.steps,
         "clocks": clk,
         "e2e": e2e,
