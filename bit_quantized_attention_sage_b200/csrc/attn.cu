@@ -457,12 +457,17 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     // O holds the sum through tile it - 1 once that tile's P V has completed;
     // rescale the O row when the running max moved (never before the first P V)
     if (it > 0 && !warp_wait(&s.o_ready, (it - 1) & 1, w, kSiteSmO)) { ok = false; break; }
-    tc_fence_after();
-    if (it > 0 && __any_sync(kFull, alpha != 1.0f)) rescale_row<D>(tO, alpha);
+    // the tcgen05 fences order the rescale's TMEM accesses after the P V it
+    // waited for and before the next P V; a tile without a rescale touches
+    // no TMEM here and needs neither
+    if (it > 0 && __any_sync(kFull, alpha != 1.0f)) {
+      tc_fence_after();
+      rescale_row<D>(tO, alpha);
+      tc_fence_before();
+    }
     l = __fadd_rn(__fmul_rn(l, alpha), rs);
     m = m_new;
     kt = kt_next;
-    tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.p_full);
   }
