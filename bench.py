@@ -260,48 +260,90 @@ class Runner:
         if ev is not None:
             ev[2].record(self.stream)
 
+    # heads per end-to-end chunk: a multiple of 4, so that every per-head
+    # buffer slice (the 4-byte-per-block scale arrays included) starts on a
+    # 16-byte boundary
+    E2E_CHUNK_HEADS = 4
+
     def run_e2e(self, steps):
         """`steps` end-to-end steps: every step copies its Q, K, V from pinned
         host memory to the device, runs the path and copies O back to pinned
-        host memory.  Copies run on a second stream into double-buffered
-        device tensors, so the copies of step i+1 overlap the kernels of step
-        i; each step's own copies are still inside the caller's timed region
-        (the last D2H completes before the caller's end event)."""
-        torch = self.torch
-        if not hasattr(self, "dbuf"):
-            self.dbuf = [(self.q, self.k, self.v, self.o),
-                         tuple(torch.empty_like(t) for t in (self.q, self.k, self.v, self.o))]
+        host memory.  A step is cut into groups of E2E_CHUNK_HEADS heads (the
+        heads are independent problems): the copies run on a copy stream
+        into double-buffered device tensors, so the H2D of one group overlaps
+        the kernels of the previous one, and each group's O is copied back as
+        soon as its kernels finish; consecutive groups run on two compute
+        streams, so that one group's kernels start while the previous group's
+        last CTAs finish.  Every step's own copies are inside the
+        caller's timed region (the last D2H completes before its end event)."""
+        torch, s, w = self.torch, self.sage, self.w
+        bh = w.B * w.H
+        hc = self.E2E_CHUNK_HEADS if bh % self.E2E_CHUNK_HEADS == 0 else bh
+        chunks = [(h0, h0 + hc) for h0 in range(0, bh, hc)]
+        if not hasattr(self, "ebuf"):
+            dev = self.q.device
+
+            def cdev(t):
+                return torch.empty((1, hc) + tuple(t.shape[2:]), dtype=t.dtype, device=dev)
+            self.ebuf = [tuple(cdev(t) for t in (self.q, self.k, self.v, self.o)) for _ in range(2)]
             self.h_o2 = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
             self.copy_stream = torch.cuda.Stream()
+            # two compute streams, alternating groups, so that one group's
+            # kernels fill the SMs the previous group's last CTAs leave idle;
+            # each has its own quantized buffers and workspaces
+            self.e_streams = [self.stream, torch.cuda.Stream()]
+            e_shape = s.make_shape(1, hc, self.shape.Nq, self.shape.Nkv, self.shape.D)
+            self.e_qkv = [s.QuantizedQKV(e_shape, dev) for _ in range(2)]
+            self.e_ws = [torch.empty(max(s.workspace_bytes(e_shape), 16), dtype=torch.uint8,
+                                     device=dev) for _ in range(2)]
+            self.e_split_ws = [None, None]
+            if self.kv_splits > 1:
+                self.e_split_ws = [torch.empty(s.attn_split_workspace_bytes(e_shape, self.kv_splits),
+                                               dtype=torch.uint8, device=dev) for _ in range(2)]
         cs, st = self.copy_stream, self.stream
-        h_out = (self.h_o, self.h_o2)
+        h_in = [t.view(1, bh, t.shape[2], t.shape[3]) for t in (self.h_q, self.h_k, self.h_v)]
+        h_out = [t.view(1, bh, t.shape[2], t.shape[3]) for t in (self.h_o, self.h_o2)]
         ev = torch.cuda.Event
         in_ready = [ev(), ev()]
-        done = [ev(), ev()]      # kernels of the step that used buffer set i finished
-        out_read = [ev(), ev()]  # D2H of buffer set i finished
+        done = [ev(), ev()]      # kernels that used buffer set j finished
+        out_read = [ev(), ev()]  # D2H of buffer set j finished
+        units = [(i, c) for i in range(steps) for c in range(len(chunks))]
         cs.wait_stream(st)
+        self.e_streams[1].wait_stream(st)
 
-        def h2d(i):
+        def h2d(u):
+            j = u % 2
+            h0, h1 = chunks[units[u][1]]
             with torch.cuda.stream(cs):
-                if i >= 2:
-                    cs.wait_event(done[i % 2])
-                for d, h in zip(self.dbuf[i % 2][:3], (self.h_q, self.h_k, self.h_v)):
-                    d.copy_(h, non_blocking=True)
-                in_ready[i % 2].record(cs)
+                if u >= 2:
+                    cs.wait_event(out_read[j])  # buffer set j's O is read back (and its kernels done)
+                for d, h in zip(self.ebuf[j][:3], h_in):
+                    d.copy_(h[:, h0:h1], non_blocking=True)
+                in_ready[j].record(cs)
 
-        h2d(0)
-        for i in range(steps):
-            if i + 1 < steps:
-                h2d(i + 1)
-            st.wait_event(in_ready[i % 2])
-            if i >= 2:
-                st.wait_event(out_read[i % 2])
-            self.step(bufs=self.dbuf[i % 2])
-            done[i % 2].record(st)
+        if units:
+            h2d(0)
+        for u, (i, c) in enumerate(units):
+            j = u % 2
+            h0, h1 = chunks[c]
+            if u + 1 < len(units):
+                h2d(u + 1)
+            est = self.e_streams[j]
+            est.wait_event(in_ready[j])
+            q, k, v, o = self.ebuf[j]
+            if self.window_quant:
+                s.quant_qk_window(q, k, v, *self.window, out=self.e_qkv[j], workspace=self.e_ws[j],
+                                  stream=est)
+            else:
+                s.quant_qk(q, k, v, out=self.e_qkv[j], workspace=self.e_ws[j], stream=est)
+            s.attn_fwd(self.e_qkv[j], w.mask, w.mask_block, out=o, stream=est,
+                       kv_splits=self.kv_splits, workspace=self.e_split_ws[j], window=self.window)
+            done[j].record(est)
             with torch.cuda.stream(cs):
-                cs.wait_event(done[i % 2])
-                h_out[i % 2].copy_(self.dbuf[i % 2][3], non_blocking=True)
-                out_read[i % 2].record(cs)
+                cs.wait_event(done[j])
+                h_out[i % 2][:, h0:h1].copy_(o, non_blocking=True)
+                out_read[j].record(cs)
+        st.wait_stream(self.e_streams[1])
         st.wait_stream(cs)
 
     def h2d_bytes(self):
@@ -456,8 +498,10 @@ def run_ours(args):
         e2e = {"value": aggregate_value(ops_rank, world, te["ms"]), "unit": UNIT,
                "h2d_bytes_per_step": runner.h2d_bytes(), "d2h_bytes_per_step": runner.d2h_bytes(),
                "ms_per_step": te["ms"],
-               "copies": "pinned host <-> device every step; the H2D of step i+1 and the D2H of "
-                         "step i overlap the kernels (second stream, double-buffered tensors)"}
+               "copies": "pinned host <-> device every step, in groups of %d heads: the H2D of "
+                         "one group and the D2H of the previous one overlap its kernels (copy "
+                         "stream, double-buffered group tensors, groups alternating on two "
+                         "compute streams)" % runner.E2E_CHUNK_HEADS}
 
     secondary = {}
     if not args.no_secondary:
