@@ -24,9 +24,9 @@
 //               pattern 0x4B400000 before each Q K^T, so the int32 result
 //               0x4B400000 + S reads as the fp32 value 1.5*2^23 + S exactly
 //               (no conversion unit, no integer add).  Per tile: load the
-//               score row from TMEM and re-seed it, take the masked max per
-//               64-key scale group with a tree of 3-input maxima, update the
-//               running max, y = exp2(fma(S, c, 8 - m)) (P scale 2^8 folded
+//               score row from TMEM, take the masked max per 64-key scale
+//               group with a tree of 3-input maxima, update the running max,
+//               re-seed the row, y = exp2(fma(S, c, 8 - m)) (P scale 2^8 folded
 //               into the exponent) with packed fp32x2 arithmetic, row sum,
 //               e4m3(y) into the swizzled shared-memory P buffer of the
 //               tile's parity, then (once P V of the previous tile has
@@ -348,7 +348,6 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     uint32_t sv[128];  // 0x4B400000 + S: the fp32 value 1.5 * 2^23 + S
     tmem_ld128(tS, sv);
     const bool more = it + 1 < nk;
-    if (more) tmem_fill128_x8_nowait(tS, kBiasBits);  // seed for the next tile
 
     // scale of each 64-key group of the tile; the next tile's K scales are
     // loaded now so that their latency is hidden behind this tile
@@ -413,6 +412,9 @@ __device__ __forceinline__ void softmax_rows(Smem<D>& s, const AttnParams& p, ui
     // not be -inf * 0 = NaN)
     const float ce0 = c0 > 0.0f ? c0 : FLT_MIN, ce1 = c1 > 0.0f ? c1 : FLT_MIN;
 
+    // re-seed S for the next tile (issued here, just before its wait: placed
+    // ahead of the maximum it measured 2.8 % slower)
+    if (more) tmem_fill128_x8_nowait(tS, kBiasBits);
     // the seed has landed; the MMA issuer may now write S of the next tile
     if (more) tmem_wait_st();
     tc_fence_before();

@@ -336,20 +336,6 @@ __device__ __forceinline__ void tmem_fill32_x8_nowait(uint32_t taddr, uint32_t v
       : "memory");
 }
 
-// Fill 64 columns with one value as eight x8 stores, without waiting.
-__device__ __forceinline__ void tmem_fill64_x8_nowait(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+0], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+8], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+16], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+24], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+32], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+40], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+48], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+56], {%1,%1,%1,%1,%1,%1,%1,%1};\n\t" ::"r"(taddr), "r"(v)
-      : "memory");
-}
-
 // Fill 128 columns with one value as sixteen x8 stores, without waiting
 // (a store reads a run of consecutive registers, so narrow stores need only
 // eight copies of the value).
