@@ -12,7 +12,7 @@
 //   pass1    one CTA per (head, 64-token block): Q block codes + scale; fp64
 //            per-channel sums of the K block in ascending token order; V
 //            block per-channel maxima.
-//   finalize one CTA per (head, 32 channels): ascending sum of the block
+//   finalize one CTA per (head, 8 channels): ascending sum of the block
 //            sums -> k_mean; max of the block maxima -> v_scale, 448/absmax.
 //   pass2    one CTA per (head, 64-token block): K - mean block codes + scale;
 //            V codes, token-major like the K codes ([B,H,Nkv_pad,D]).
@@ -381,34 +381,36 @@ __device__ __forceinline__ int eq_exponent(float aq, float kmax, float kmin, flo
   return e > kEqMax ? kEqMax : (e < -kEqMax ? -kEqMax : e);
 }
 
-// One CTA per (head, 32 channels).  The fp64 block sums of a channel must be
+// One CTA per (head, 8 channels).  The fp64 block sums of a channel must be
 // added one after the other in ascending block order (the canonical order
-// that makes the mean reproducible), so the CTA stages chunks of block sums
-// in shared memory with coalesced loads by all its threads, and then one
-// thread per channel adds its chunk in order.  The V block maxima are
-// reduced on the fly (max is order-free).
-constexpr int kFinChunk = 128;  // blocks per staged chunk
-constexpr int kFinCh = 32;      // channels per CTA
+// that makes the mean reproducible): the CTA stages up to 512 block sums
+// per channel in shared memory with loads spread over all its threads, then
+// one thread per channel adds them in order (shared-memory reads issued
+// eight ahead of the additions, so that the chain of fp64 additions is the
+// only serial part).  The V block maxima and the equalisation maxima are
+// order-free: every thread reduces the blocks it loaded, then the CTA
+// combines its 32 partial maxima per channel.
+constexpr int kFinCh = 8;                      // channels per CTA
+constexpr int kFinRows = kThreads / kFinCh;    // 32 threads per channel
+constexpr int kFinChunk = 512;                 // blocks per staged chunk
 
 __global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
-  constexpr int kGroups = kThreads / kFinCh;  // 8 row groups
-  __shared__ double part[kFinChunk][kFinCh];
-  __shared__ float vred[kGroups][kFinCh];
-  __shared__ float xred[3][kGroups][kFinCh];   // equalisation: K max, K min, |Q| max
+  __shared__ double part[kFinChunk][kFinCh];   // 32 KB
+  __shared__ float red[4][kFinRows][kFinCh];   // V max; K max, K min, |Q| max (equalisation)
   const int D = a.D;
   const int bh = blockIdx.y;
   const int d0 = blockIdx.x * kFinCh;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
-  const int lane = threadIdx.x % kFinCh;       // channel d0 + lane
-  const int rowg = threadIdx.x / kFinCh;       // 0 .. 7
+  const int ch = threadIdx.x % kFinCh;         // channel d0 + ch
+  const int rl = threadIdx.x / kFinCh;         // 0 .. 31
   const bool eq = a.eq;
   double total = 0.0;
   float m = 0.0f, kmx = -INFINITY, kmn = INFINITY, qmx = 0.0f;
   for (int b0 = 0; b0 < nkb; b0 += kFinChunk) {
     const int nb = min(kFinChunk, nkb - b0);
-    for (int r = rowg; r < nb; r += kGroups) {
-      const size_t w = (static_cast<size_t>(bh) * nkb + b0 + r) * D + d0 + lane;
-      part[r][lane] = a.ws_ksum[w];
+    for (int r = rl; r < nb; r += kFinRows) {
+      const size_t w = (static_cast<size_t>(bh) * nkb + b0 + r) * D + d0 + ch;
+      part[r][ch] = a.ws_ksum[w];
       m = fmaxf(m, a.ws_vmax[w]);
       if (eq) {
         kmx = fmaxf(kmx, a.ws_kmax[w]);
@@ -416,32 +418,41 @@ __global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
       }
     }
     __syncthreads();
-    if (threadIdx.x < kFinCh)
-      for (int r = 0; r < nb; r++) total = __dadd_rn(total, part[r][threadIdx.x]);
+    if (threadIdx.x < kFinCh) {
+      int r = 0;
+      for (; r + 8 <= nb; r += 8) {
+        double v[8];
+#pragma unroll
+        for (int e = 0; e < 8; e++) v[e] = part[r + e][threadIdx.x];
+#pragma unroll
+        for (int e = 0; e < 8; e++) total = __dadd_rn(total, v[e]);
+      }
+      for (; r < nb; r++) total = __dadd_rn(total, part[r][threadIdx.x]);
+    }
     __syncthreads();
   }
   if (eq) {
     const int nqb = (a.Nq + kBlk - 1) / kBlk;
-    for (int r = rowg; r < nqb; r += kGroups)
-      qmx = fmaxf(qmx, a.ws_qmax[(static_cast<size_t>(bh) * nqb + r) * D + d0 + lane]);
-    xred[0][rowg][lane] = kmx;
-    xred[1][rowg][lane] = kmn;
-    xred[2][rowg][lane] = qmx;
+    for (int r = rl; r < nqb; r += kFinRows)
+      qmx = fmaxf(qmx, a.ws_qmax[(static_cast<size_t>(bh) * nqb + r) * D + d0 + ch]);
+    red[1][rl][ch] = kmx;
+    red[2][rl][ch] = kmn;
+    red[3][rl][ch] = qmx;
   }
-  vred[rowg][lane] = m;
+  red[0][rl][ch] = m;
   __syncthreads();
-  if (threadIdx.x < kFinCh) {
-    for (int g = 1; g < kGroups; g++) m = fmaxf(m, vred[g][threadIdx.x]);
+  if (threadIdx.x < kFinCh) {  // rl = 0, ch = threadIdx.x
+    for (int g = 1; g < kFinRows; g++) m = fmaxf(m, red[0][g][threadIdx.x]);
     const int idx = bh * D + d0 + threadIdx.x;
     const float mu = __double2float_rn(__ddiv_rn(total, static_cast<double>(a.Nkv)));
     a.k_mean[idx] = mu;
     a.v_scale[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(m, 448.0f);
     a.ws_vinv[idx] = (m == 0.0f) ? 0.0f : __fdiv_rn(448.0f, m);
     if (eq) {
-      for (int g = 1; g < kGroups; g++) {
-        kmx = fmaxf(kmx, xred[0][g][threadIdx.x]);
-        kmn = fminf(kmn, xred[1][g][threadIdx.x]);
-        qmx = fmaxf(qmx, xred[2][g][threadIdx.x]);
+      for (int g = 1; g < kFinRows; g++) {
+        kmx = fmaxf(kmx, red[1][g][threadIdx.x]);
+        kmn = fminf(kmn, red[2][g][threadIdx.x]);
+        qmx = fmaxf(qmx, red[3][g][threadIdx.x]);
       }
       const int e = eq_exponent(qmx, kmx, kmn, mu);
       a.ws_eq_up[idx] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);    // 2^e
