@@ -82,6 +82,13 @@ def test_two_gloo_ranks(tmp_path):
     assert r[0]["seed"] != r[1]["seed"] and r[0]["q_sum"] != r[1]["q_sum"]
     line = json.loads(r[0]["ref_out"].strip())
     assert line["impl"] == "reference" and line["n_gpus"] == world
+    # the reference arm reports the GPU arm's metric, unit and direction on
+    # the same workload, its own CPU baseline and an e2e with no copies
+    assert (line["metric"], line["unit"], line["higher_is_better"]) == (bench.METRIC, bench.UNIT, True)
+    assert line["config"]["workload"] == synth.TINY.name
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
     assert r[1]["ref_out"] == ""  # other ranks exit without work
 
 
