@@ -6,6 +6,8 @@
   the oracle, unsplit and in split-KV form with more ranges than KV tiles.
 * A block-sparse call over 6144 KV tiles (786432 keys, the most its tile
   bitmap holds): sampled rows match the oracle's block-sparse form.
+* The rotary quantizer at its token limit, 65535 blocks of 64 keys (its
+  grid puts the blocks on the y dimension): bit-exact with the oracle.
 """
 import numpy as np
 import pytest
@@ -21,6 +23,7 @@ pytestmark = pytest.mark.gpu
 
 MAX_HEADS = 65535
 MAX_SPARSE_KEYS = 6144 * 128
+MAX_ROPE_TOKENS = 65535 * 64
 
 
 def test_most_heads_one_token_each():
@@ -71,3 +74,19 @@ def test_block_sparse_at_its_tile_limit():
     with pytest.raises(RuntimeError):
         sage.attn_fwd(qkv2, 0, 0, block_mask=bm2)
     assert sage.sync_status() == 0
+
+
+def test_rotary_quantizer_at_its_token_limit():
+    rng = np.random.default_rng(4194240)
+    nq, nkv, D = 64, MAX_ROPE_TOKENS, 64
+    q = synth.f32_to_bf16_bits(rng.standard_normal((1, 1, nq, D), dtype=np.float32))
+    k = synth.f32_to_bf16_bits(rng.standard_normal((1, 1, nkv, D), dtype=np.float32))
+    v = synth.f32_to_bf16_bits(rng.standard_normal((1, 1, nkv, D), dtype=np.float32))
+    ang_q = rng.uniform(-np.pi, np.pi, (nq, D // 2))
+    ang_k = rng.uniform(-np.pi, np.pi, (nkv, D // 2)).astype(np.float32)
+    tabs = (np.cos(ang_q).astype(np.float32), np.sin(ang_q).astype(np.float32),
+            np.cos(ang_k), np.sin(ang_k))
+    qkv = sage.quant_qk(to_dev(q), to_dev(k), to_dev(v),
+                        rope=[torch.from_numpy(t).cuda() for t in tabs])
+    assert sage.sync_status() == 0
+    check_quant_head(qkv, 0, 0, oracle.quant_head(q[0, 0], k[0, 0], v[0, 0], rope=tabs))
