@@ -37,6 +37,16 @@ namespace sage {
 
 namespace {
 
+// Programmatic dependent launch.  finalize and pass 2 are launched with
+// programmatic stream serialization, so their CTAs may be scheduled while
+// the previous kernel's last CTAs still run; grid_dep_wait holds them until
+// that grid has completed and its writes are visible.  grid_dep_trigger lets
+// the next kernel launch once every CTA of this grid has passed it.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 constexpr int kBlk = 64;
 constexpr int kThreads = 256;
 
@@ -191,6 +201,7 @@ __device__ __forceinline__ float channel_absmax(const uint16_t* blk, int valid, 
 // also its channel maxima and minima.
 template <int D, bool ROPE, bool EQ>
 __global__ void __launch_bounds__(kThreads) k_quant_pass1(QuantArgs a) {
+  grid_dep_trigger();
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;  // chunks per thread
   __shared__ float red[kThreads / 32];
@@ -395,6 +406,8 @@ constexpr int kFinRows = kThreads / kFinCh;    // 32 threads per channel
 constexpr int kFinChunk = 512;                 // blocks per staged chunk
 
 __global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
+  grid_dep_wait();
+  grid_dep_trigger();
   __shared__ double part[kFinChunk][kFinCh];   // 32 KB
   __shared__ float red[4][kFinRows][kFinCh];   // V max; K max, K min, |Q| max (equalisation)
   const int D = a.D;
@@ -466,6 +479,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_finalize(QuantArgs a) {
 // here from Q * 2^e; the smoothed K is multiplied by 2^-e before its codes.
 template <int D, bool ROPE, bool EQ>
 __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
+  grid_dep_wait();
   constexpr int kChunksPerRow = D / 8;
   constexpr int CH = kBlk * kChunksPerRow / kThreads;
   __shared__ float red[kThreads / 32];
@@ -576,6 +590,23 @@ __global__ void __launch_bounds__(kThreads) k_quant_pass2(QuantArgs a) {
 
 }  // namespace
 
+// a launch of `kernel` that may begin before the previous kernel of the
+// stream has finished (the kernel waits for it in grid_dep_wait)
+template <typename Kernel>
+cudaError_t launch_after(Kernel kernel, dim3 grid, cudaStream_t stream, const QuantArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream) {
   const int nqb = (a.Nq + kBlk - 1) / kBlk;
   const int nkb = (a.Nkv + kBlk - 1) / kBlk;
@@ -586,23 +617,29 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t stream) {
   const dim3 r1(a.BH, g1.x), r2(a.BH, g2.x);  // rotary variant: heads fastest
   if (rope && g1.x > 65535) return cudaErrorInvalidConfiguration;
   if (rope && a.eq) return cudaErrorInvalidValue;  // not offered together
+  cudaError_t e = cudaSuccess;
   if (a.D == 128) {
     if (rope) k_quant_pass1<128, true, false><<<r1, kThreads, 0, stream>>>(a);
     else if (a.eq) k_quant_pass1<128, false, true><<<g1, kThreads, 0, stream>>>(a);
     else k_quant_pass1<128, false, false><<<g1, kThreads, 0, stream>>>(a);
-    k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
-    if (rope) k_quant_pass2<128, true, false><<<r2, kThreads, 0, stream>>>(a);
-    else if (a.eq) k_quant_pass2<128, false, true><<<g1, kThreads, 0, stream>>>(a);
-    else k_quant_pass2<128, false, false><<<g2, kThreads, 0, stream>>>(a);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_after(k_quant_finalize, gf, stream, a);
+    if (e == cudaSuccess)
+      e = rope   ? launch_after(k_quant_pass2<128, true, false>, r2, stream, a)
+          : a.eq ? launch_after(k_quant_pass2<128, false, true>, g1, stream, a)
+                 : launch_after(k_quant_pass2<128, false, false>, g2, stream, a);
   } else {
     if (rope) k_quant_pass1<64, true, false><<<r1, kThreads, 0, stream>>>(a);
     else if (a.eq) k_quant_pass1<64, false, true><<<g1, kThreads, 0, stream>>>(a);
     else k_quant_pass1<64, false, false><<<g1, kThreads, 0, stream>>>(a);
-    k_quant_finalize<<<gf, kThreads, 0, stream>>>(a);
-    if (rope) k_quant_pass2<64, true, false><<<r2, kThreads, 0, stream>>>(a);
-    else if (a.eq) k_quant_pass2<64, false, true><<<g1, kThreads, 0, stream>>>(a);
-    else k_quant_pass2<64, false, false><<<g2, kThreads, 0, stream>>>(a);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_after(k_quant_finalize, gf, stream, a);
+    if (e == cudaSuccess)
+      e = rope   ? launch_after(k_quant_pass2<64, true, false>, r2, stream, a)
+          : a.eq ? launch_after(k_quant_pass2<64, false, true>, g1, stream, a)
+                 : launch_after(k_quant_pass2<64, false, false>, g2, stream, a);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
