@@ -133,17 +133,25 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=2)
+        return self.summarize(self.lines)
+
+    @staticmethod
+    def summarize(lines):
+        """Median SM clock of the busy samples (above half the maximum clock),
+        the maximum clock and every throttle reason seen active, from
+        nvidia-smi csv lines of FIELDS; None without a usable sample."""
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
+                clk, clk_max = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
+            sm.append(clk)
+            mx = max(mx, clk_max)
             for n, val in zip(names, parts[5:9]):
                 if val.lower() == "active":
                     reasons.add(n)
